@@ -1,0 +1,384 @@
+#!/usr/bin/env python
+"""Benchmark of the FP8 vision-encoder attention path on B200.
+
+One step = one dynamic-scaling forward of the 8192-token, 16-head,
+head_dim-128 workload: amax ring update -> per-tensor e4m3 quantize of
+Q/K/V -> varlen FP8 attention (BF16 out) -> per-token-group e4m3 quantize of
+the attention output viewed as [8192, 2048].  Inputs are seeded synthetic
+BF16 (N(0,1), 1% of channels x8) for 20 forwards, resident in HBM, rotated
+step by step (2.0 GB > 126 MB L2).
+
+Prints one JSON line: metric = counted attention TFLOP/s (4*S^2*D*H per
+image), whole job over all ranks, plus the attention kernel's roofline, the
+oracle's CPU baseline, an end-to-end number through host buffers, clocks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU: launched under torch.distributed.run, one rank per GPU; every
+rank runs its own replica of the workload (weak scaling, no collective on
+the data path); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "FP8 varlen attention TFLOP/s (counted 4*S^2*D*H) over the full step"
+UNIT = "TFLOP/s"
+WORKLOAD = "c2"
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _source_sha(path):
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def _traffic(kernel_src: str, workload: str):
+    """DRAM bytes per launch recorded from an ncu capture, if it was taken on
+    the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        e = d.get(workload)
+        if e and e.get("source_sha") == _source_sha(kernel_src):
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+    return None
+
+
+def _oracle_rows_time(w, codes, desc, rows_budget_s: float, seed: int):
+    """Time the oracle's attention on seeded (token, head) rows until the
+    budget is spent; returns (counted FLOPs, seconds, rows)."""
+    import oracle
+    import synth
+    cu = synth.cu_seqlens(w.seg_lens)
+    rng = np.random.default_rng(seed)
+    flops, secs, rows = 0.0, 0.0, 0
+    batch = 8
+    while secs < rows_budget_s:
+        toks = rng.integers(0, w.tokens, size=batch).astype(np.int64)
+        hs = rng.integers(0, w.heads, size=batch).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.attn_pairs(*codes, *desc, cu, w.heads, w.head_dim, w.softmax_scale, toks, hs)
+        secs += time.perf_counter() - t0
+        for t in toks:
+            seg = int(np.searchsorted(cu, t, side="right") - 1)
+            S = int(cu[seg + 1] - cu[seg])
+            flops += 4.0 * S * w.head_dim
+        rows += batch
+    return flops, secs, rows
+
+
+def _oracle_inputs(w):
+    import oracle
+    q, k, v = w.qkv(0)
+    desc = list(oracle.Ring().update([oracle.amax_bf16(x) for x in (q, k, v)]))
+    codes = [oracle.quantize_per_tensor(x, d).reshape(w.tokens, w.heads, w.head_dim)
+             for x, d in zip((q, k, v), desc)]
+    return codes, desc
+
+
+def run_reference(args):
+    """The oracle (plain single-threaded C) as the reference arm."""
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    import synth
+    w = synth.WORKLOADS[args.workload]
+    codes, desc = _oracle_inputs(w)
+    per_step = args.ref_step_seconds
+    for _ in range(args.warmup):
+        _oracle_rows_time(w, codes, desc, per_step / 4, seed=1)
+    tot_f, tot_s, tot_rows = 0.0, 0.0, 0
+    for s in range(args.steps):
+        f, sec, rows = _oracle_rows_time(w, codes, desc, per_step, seed=100 + s)
+        tot_f += f
+        tot_s += sec
+        tot_rows += rows
+    value = tot_f / tot_s / 1e12
+    sample = (f"{tot_rows} seeded (token, head) query rows of forward 0's attention "
+              f"({tot_rows / args.steps:.0f} per step; amax/quantize stages excluded)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": _config(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(w):
+    return {"workload": w.name, "seq_lens": list(w.seg_lens), "heads": w.heads,
+            "head_dim": w.head_dim, "forwards": len(w.seeds),
+            "step": "amax ring + quantize q/k/v + attention (bf16 out) + group quant (128)",
+            "l2": "inputs rotate over 20 forwards (2.0 GB > 126 MB L2)",
+            "parallelism": "replicas"}
+
+
+def run_ours(args):
+    import torch
+    import fp8_quantized_vit_b200 as fv
+    import synth
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dist = None
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    w = synth.WORKLOADS[args.workload]
+    T, H, D = w.tokens, w.heads, w.head_dim
+    n_fwd = len(w.seeds)
+    ctx = fv.Context(local)
+    dev = torch.device("cuda", local)
+
+    # inputs: all forwards resident in HBM
+    inputs = []
+    for f in range(n_fwd):
+        qkv = w.qkv(f)
+        inputs.append([torch.from_numpy(x.view(np.int16)).view(torch.bfloat16)
+                       .reshape(T, H, D).to(dev) for x in qkv])
+    cu = torch.from_numpy(synth.cu_seqlens(w.seg_lens)).to(dev)
+    max_s = max(w.seg_lens)
+    ring = fv.new_ring(dev)
+    desc = torch.zeros(3, dtype=torch.float32, device=dev)
+    q8, k8, v8 = (torch.empty((T, H, D), dtype=torch.uint8, device=dev) for _ in range(3))
+    out = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    xq = torch.empty((T, H * D), dtype=torch.uint8, device=dev)
+    xs = torch.empty((T, H * D // 128), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+
+    def step(i, timed=False):
+        q, k, v = inputs[i % n_fwd]
+        fv.fp8_amax_ring_update(q, k, v, ring, desc, ctx=ctx)
+        fv.fp8_quantize_qkv_per_tensor(q, k, v, desc, q8, k8, v8, ctx=ctx)
+        if timed:
+            ev_a[i].record(stream)
+        fv.fp8_varlen_attn_fwd(q8, k8, v8, desc[0:1], desc[1:2], desc[2:3], cu, max_s,
+                               w.softmax_scale, out, ctx=ctx)
+        if timed:
+            ev_b[i].record(stream)
+        fv.per_token_group_quant_fp8(out.view(T, H * D), 128, xq, xs, ctx=ctx)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    st, site = ctx.check()
+    if st != fv.OK:
+        raise RuntimeError(f"device fault during warm-up: {fv.status_string(st)} site {site}")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(i, timed=True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    elapsed_ms = t0.elapsed_time(t1)
+    attn_ms = [a.elapsed_time(b) for a, b in zip(ev_a, ev_b)]
+    st, site = ctx.check()
+    if st != fv.OK:
+        raise RuntimeError(f"device fault: {fv.status_string(st)} site {site}")
+
+    if dist:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    flops_step = w.attn_flops()
+    value = ws * flops_step * args.steps / (elapsed_ms * 1e-3) / 1e12
+    attn_avg_s = statistics.mean(attn_ms) * 1e-3
+    attn_tflops = flops_step / attn_avg_s / 1e12
+
+    # end to end through host buffers: pinned BF16 q/k/v in, quantized
+    # attention output (codes + group scales) back, copies inside the timing.
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    host_in = [[t.cpu().pin_memory() for t in inputs[f]] for f in range(min(n_fwd, e2e_steps))]
+    host_xq = torch.empty(xq.shape, dtype=xq.dtype).pin_memory()
+    host_xs = torch.empty(xs.shape, dtype=xs.dtype).pin_memory()
+    dq, dk, dv = (torch.empty((T, H, D), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        hq, hk, hv = host_in[i % len(host_in)]
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        fv.fp8_amax_ring_update(dq, dk, dv, ring, desc, ctx=ctx)
+        fv.fp8_quantize_qkv_per_tensor(dq, dk, dv, desc, q8, k8, v8, ctx=ctx)
+        fv.fp8_varlen_attn_fwd(q8, k8, v8, desc[0:1], desc[1:2], desc[2:3], cu, max_s,
+                               w.softmax_scale, out, ctx=ctx)
+        fv.per_token_group_quant_fp8(out.view(T, H * D), 128, xq, xs, ctx=ctx)
+        host_xq.copy_(xq, non_blocking=True)
+        host_xs.copy_(xs, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = ws * flops_step * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    h2d = 3 * T * H * D * 2
+    d2h = xq.numel() + xs.numel() * 4
+
+    peaks = _peaks()
+    fp8_peak = 2.0 * peaks["bf16"]  # dense FP8 = 2 x dense BF16 (nominal ratio)
+    traffic = _traffic(os.path.join(ROOT, "fp8_quantized_vit_b200", "csrc", "attn.cu"),
+                       args.workload)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3 (fp32 accumulate)",
+        "data": "synthetic", "config": _config(w),
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>",
+                     "achieved": attn_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
+                     "frac": attn_tflops / fp8_peak, "traffic": traffic,
+                     "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16']} x 2 (fp8/bf16)",
+                     "kernel_ms": attn_avg_s * 1e3},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        codes, dsc = _oracle_inputs(w)
+        f, sec, rows = _oracle_rows_time(w, codes, dsc, args.cpu_seconds, seed=7)
+        line["cpu_baseline"] = {
+            "value": f / sec / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{rows} seeded (token, head) query rows of forward 0's attention "
+                      f"({sec:.1f} s single-threaded; amax/quantize stages excluded)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    ctx.close()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=1.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

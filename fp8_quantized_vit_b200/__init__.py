@@ -1,0 +1,320 @@
+"""Python binding of libfp8vit.so -- the B200 FP8 vision-encoder attention path.
+
+Argument marshalling only: every step of the path runs in the CUDA kernels
+behind the C ABI (``include/fp8vit.h``); PyTorch supplies device memory and
+the current CUDA stream.  The library must be built (``__graft_entry__.build``
+or ``python -m fp8_quantized_vit_b200._build``); there is no fallback.
+
+Entry points (same names as the C ABI):
+  fp8_amax_ring_update, fp8_quantize_qkv_per_tensor, fp8_varlen_attn_fwd,
+  per_token_group_quant_fp8, fp8_static_scales_load, fp8_static_scales_save,
+  fp8_descale_from_amax, fp8_ring_read_amax, ring_init
+and ``FP8EncoderAttention``, which chains them for one attention layer
+(dynamic ring or static scales, BF16 or FP8 output, optional group quant).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp8vit.so")
+
+OK, EINVAL, EUNSUPPORTED, ECUDA, EIO, EPARSE, ENOTFOUND, ETIMEOUT = range(8)
+RING_BYTES = 256
+E4M3_MAX = 448.0
+
+_P, _I32, _I64, _F32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+
+_SIGNATURES = {
+    "fp8vit_create": (_I32, [_I32, ctypes.POINTER(_P)]),
+    "fp8vit_destroy": (_I32, [_P]),
+    "fp8vit_check": (_I32, [_P, _P, ctypes.POINTER(_I32)]),
+    "fp8vit_status_string": (ctypes.c_char_p, [_I32]),
+    "fp8vit_version": (_I32, []),
+    "fp8vit_ring_init": (_I32, [_P, _P]),
+    "fp8_amax_ring_update": (_I32, [_P, _P, _P, _P, _I64, _P, _P, _P]),
+    "fp8_ring_read_amax": (_I32, [_P, _P, _P]),
+    "fp8_quantize_qkv_per_tensor": (_I32, [_P, _P, _P, _P, _I64, _P, _P, _P, _P, _P]),
+    "fp8_varlen_attn_fwd": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I64, _I32, _I32,
+                                   _F32, _P, _I32, _P, _P]),
+    "per_token_group_quant_fp8": (_I32, [_P, _P, _I64, _I64, _I32, _P, _P, _P]),
+    "fp8_static_scales_load": (_I32, [ctypes.c_char_p, ctypes.c_char_p, _P]),
+    "fp8_static_scales_save": (_I32, [ctypes.c_char_p, _I32, ctypes.POINTER(ctypes.c_char_p),
+                                      _P, _F32]),
+    "fp8_descale_from_amax": (_F32, [_F32]),
+}
+
+_lib = None
+
+
+class FP8VitError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+def lib():
+    """The loaded libfp8vit.so; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m fp8_quantized_vit_b200._build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().fp8vit_status_string(status).decode()
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise FP8VitError(status, what)
+
+
+def _stream(stream=None) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _ptr(t: torch.Tensor | None, dtype=None, name: str = "tensor") -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    return t.data_ptr()
+
+
+_FP8 = (torch.uint8, torch.float8_e4m3fn)
+
+
+class Context:
+    """A library context on one device (status word + amax scratch)."""
+
+    def __init__(self, device: int | None = None):
+        if device is None:
+            device = torch.cuda.current_device()
+        h = _P()
+        _check(lib().fp8vit_create(device, ctypes.byref(h)), "fp8vit_create")
+        self.handle = h.value
+        self.device = device
+
+    def check(self, stream=None) -> tuple[int, int]:
+        """Synchronize and return (status, site) of the first device fault."""
+        site = _I32(0)
+        st = lib().fp8vit_check(self.handle, _stream(stream), ctypes.byref(site))
+        return st, site.value
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lib().fp8vit_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+_default_ctx: dict[int, Context] = {}
+
+
+def default_context() -> Context:
+    dev = torch.cuda.current_device()
+    if dev not in _default_ctx:
+        _default_ctx[dev] = Context(dev)
+    return _default_ctx[dev]
+
+
+def _ctx(ctx):
+    return (ctx or default_context()).handle
+
+
+# ---- ring ------------------------------------------------------------------------
+
+def new_ring(device=None) -> torch.Tensor:
+    """A zeroed ring state (64 x float32 = 256 bytes) on the device."""
+    r = torch.empty(RING_BYTES // 4, dtype=torch.float32, device=device or "cuda")
+    ring_init(r)
+    return r
+
+
+def ring_init(ring: torch.Tensor, stream=None):
+    _check(lib().fp8vit_ring_init(_ptr(ring, torch.float32, "ring"), _stream(stream)),
+           "fp8vit_ring_init")
+
+
+def fp8_amax_ring_update(q, k, v, ring, descale3, ctx=None, stream=None):
+    n = q.numel()
+    if k.numel() != n or v.numel() != n:
+        raise ValueError("q, k, v must have the same number of elements")
+    _check(lib().fp8_amax_ring_update(
+        _ctx(ctx), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+        _ptr(v, torch.bfloat16, "v"), n, _ptr(ring, torch.float32, "ring"),
+        _ptr(descale3, torch.float32, "descale3"), _stream(stream)), "fp8_amax_ring_update")
+    return descale3
+
+
+def fp8_ring_read_amax(ring, stream=None) -> list[float]:
+    out = (ctypes.c_float * 3)()
+    _check(lib().fp8_ring_read_amax(_ptr(ring, torch.float32, "ring"), out, _stream(stream)),
+           "fp8_ring_read_amax")
+    return [float(x) for x in out]
+
+
+# ---- quantizers ----------------------------------------------------------------------
+
+def fp8_quantize_qkv_per_tensor(q, k, v, descale3, q8, k8, v8, ctx=None, stream=None):
+    n = q.numel()
+    for t in (k, v, q8, k8, v8):
+        if t.numel() != n:
+            raise ValueError("all tensors must have the same number of elements")
+    _check(lib().fp8_quantize_qkv_per_tensor(
+        _ctx(ctx), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+        _ptr(v, torch.bfloat16, "v"), n, _ptr(descale3, torch.float32, "descale3"),
+        _ptr(q8, _FP8, "q8"), _ptr(k8, _FP8, "k8"), _ptr(v8, _FP8, "v8"), _stream(stream)),
+        "fp8_quantize_qkv_per_tensor")
+    return q8, k8, v8
+
+
+def per_token_group_quant_fp8(x, group, xq, scales, ctx=None, stream=None):
+    if x.dim() != 2:
+        raise ValueError("x must be [m, n]")
+    m, n = x.shape
+    if xq.numel() != m * n or scales.numel() != (m * (n // group) if group > 0 else -1):
+        raise ValueError("output sizes do not match [m, n] and [m, n/group]")
+    _check(lib().per_token_group_quant_fp8(
+        _ctx(ctx), _ptr(x, torch.bfloat16, "x"), m, n, group, _ptr(xq, _FP8, "xq"),
+        _ptr(scales, torch.float32, "scales"), _stream(stream)), "per_token_group_quant_fp8")
+    return xq, scales
+
+
+# ---- attention ----------------------------------------------------------------------
+
+def fp8_varlen_attn_fwd(q8, k8, v8, q_descale, k_descale, v_descale, cu_seqlens, max_seqlen,
+                        softmax_scale, out, output_scale=None, ctx=None, stream=None):
+    """q8/k8/v8: e4m3 [T, H, D]; out: BF16 [T, H, D], or e4m3 with output_scale."""
+    if q8.dim() != 3:
+        raise ValueError("q8 must be [T, H, D]")
+    T, H, D = q8.shape
+    if k8.shape != q8.shape or v8.shape != q8.shape or out.shape != q8.shape:
+        raise ValueError("q8, k8, v8 and out must have the same [T, H, D] shape")
+    fp8_out = output_scale is not None
+    _check(lib().fp8_varlen_attn_fwd(
+        _ctx(ctx), _ptr(q8, _FP8, "q8"), _ptr(k8, _FP8, "k8"), _ptr(v8, _FP8, "v8"),
+        _ptr(q_descale, torch.float32, "q_descale"), _ptr(k_descale, torch.float32, "k_descale"),
+        _ptr(v_descale, torch.float32, "v_descale"), _ptr(cu_seqlens, torch.int32, "cu_seqlens"),
+        cu_seqlens.numel() - 1, int(max_seqlen), T, H, D, float(softmax_scale),
+        _ptr(out, _FP8 if fp8_out else torch.bfloat16, "out"), 1 if fp8_out else 0,
+        _ptr(output_scale, torch.float32, "output_scale"), _stream(stream)),
+        "fp8_varlen_attn_fwd")
+    return out
+
+
+# ---- static scales ------------------------------------------------------------------
+
+def fp8_static_scales_load(path: str, layer: str) -> tuple[float, float, float]:
+    out = (ctypes.c_float * 3)()
+    _check(lib().fp8_static_scales_load(path.encode(), layer.encode(), out),
+           f"fp8_static_scales_load({layer})")
+    return float(out[0]), float(out[1]), float(out[2])
+
+
+def fp8_static_scales_save(path: str, layers, qkv_amax, margin: float = 1.5):
+    import numpy as np
+    names = (ctypes.c_char_p * len(layers))(*[s.encode() for s in layers])
+    vals = np.ascontiguousarray(np.asarray(qkv_amax, dtype=np.float32).reshape(len(layers), 3))
+    _check(lib().fp8_static_scales_save(path.encode(), len(layers), names, vals.ctypes.data,
+                                        float(margin)), "fp8_static_scales_save")
+
+
+def fp8_descale_from_amax(v: float) -> float:
+    return float(lib().fp8_descale_from_amax(float(v)))
+
+
+# ---- one attention layer ---------------------------------------------------------------
+
+class FP8EncoderAttention:
+    """One ViT-encoder attention layer on the FP8 path.
+
+    Holds the layer's scale state (a device ring for dynamic scaling, or
+    static descales), and runs
+        [amax ring update] -> per-tensor quantize -> varlen FP8 attention
+        [-> per-token-group quantize of the BF16 output]
+    on the current stream.  Intermediate FP8 buffers are allocated once per
+    token count and reused (no allocation per call at steady state).
+    """
+
+    def __init__(self, num_heads: int, head_dim: int, softmax_scale: float | None = None,
+                 static_amax=None, margin: float = 1.5, device=None, ctx: Context | None = None):
+        self.H, self.D = num_heads, head_dim
+        self.softmax_scale = (float(torch.tensor(head_dim ** -0.5, dtype=torch.float32))
+                              if softmax_scale is None else softmax_scale)
+        self.device = torch.device(device or "cuda")
+        self.ctx = ctx or default_context()
+        self.descale = torch.zeros(3, dtype=torch.float32, device=self.device)
+        self.ring = None
+        if static_amax is None:
+            self.ring = new_ring(self.device)
+        else:
+            self.set_static_amax(static_amax, margin=None)
+        self._bufs = {}
+
+    @classmethod
+    def from_scale_file(cls, path: str, layer: str, num_heads: int, head_dim: int, **kw):
+        vals = fp8_static_scales_load(path, layer)
+        obj = cls(num_heads, head_dim, static_amax=vals, **kw)
+        return obj
+
+    def set_static_amax(self, values, margin: float | None = None):
+        """Use static scales.  ``values`` are in the amax domain (already
+        including the save margin, as stored in a scale file); pass ``margin``
+        to apply one here instead."""
+        import numpy as np
+        v = np.asarray(values, dtype=np.float32)
+        if margin is not None:
+            v = (v * np.float32(margin)).astype(np.float32)
+        d = [fp8_descale_from_amax(float(x)) for x in v]
+        self.descale.copy_(torch.tensor(d, dtype=torch.float32))
+        self.ring = None
+
+    def _buffers(self, T: int, fp8_out: bool):
+        key = (T, fp8_out)
+        if key not in self._bufs:
+            shape = (T, self.H, self.D)
+            mk = lambda dt: torch.empty(shape, dtype=dt, device=self.device)
+            self._bufs[key] = dict(q8=mk(torch.uint8), k8=mk(torch.uint8), v8=mk(torch.uint8),
+                                   out=mk(torch.uint8 if fp8_out else torch.bfloat16))
+        return self._bufs[key]
+
+    def forward(self, q, k, v, cu_seqlens, max_seqlen: int, output_scale=None, out=None):
+        """q, k, v: BF16 [T, H, D] on the device; cu_seqlens: int32 [B+1].
+        Returns the attention output (BF16, or e4m3 codes if output_scale)."""
+        T = q.shape[0]
+        b = self._buffers(T, output_scale is not None)
+        if self.ring is not None:
+            fp8_amax_ring_update(q, k, v, self.ring, self.descale, ctx=self.ctx)
+        fp8_quantize_qkv_per_tensor(q, k, v, self.descale, b["q8"], b["k8"], b["v8"],
+                                    ctx=self.ctx)
+        o = b["out"] if out is None else out
+        fp8_varlen_attn_fwd(b["q8"], b["k8"], b["v8"], self.descale[0:1], self.descale[1:2],
+                            self.descale[2:3], cu_seqlens, max_seqlen, self.softmax_scale, o,
+                            output_scale=output_scale, ctx=self.ctx)
+        return o
+
+    __call__ = forward

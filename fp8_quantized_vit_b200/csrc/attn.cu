@@ -1,0 +1,497 @@
+// Non-causal varlen FP8 flash attention for sm_100a (vLLM docs "FP8 ViT
+// Encoder Attention": per-tensor FP8 Q/K/V, packed images attend only within
+// themselves; vLLM issue "fused fp8 output for FlashAttention 3": an
+// output_scale epilogue that writes e4m3).
+//
+// One CTA = one (image, head, 128-row query tile).  Warp roles:
+//   warp 0      TMA producer: Q once, then K/V tiles of 128 keys into an
+//               NS-stage shared-memory ring (SWIZZLE_32B, 32-byte boxes).
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer:
+//               S = Q K^T (kind::f8f6f4, K-major A and B) into TMEM,
+//               O += P V  (A = P from TMEM, B = V MN-major from smem).
+//   warps 2..5  softmax + epilogue, one query row per thread (TMEM lane):
+//               row max, exp2, row sum in registers; P written back to TMEM
+//               as two e4m3 terms (hi + lo) so that the PV product keeps
+//               ~8 mantissa bits while running on FP8 tensor cores; O is
+//               rescaled in TMEM when the row max rises.
+// head_dim 72 is padded inside the kernel: the QK contraction runs over 96
+// bytes starting at the head's offset rounded down to 16 bytes (TMA needs a
+// 16-byte aligned x coordinate); bytes of the window outside the head are
+// zeroed in Q, so the neighbouring head's K bytes contribute exactly 0.  PV
+// runs with N = 80 and the epilogue picks the head's 72 columns.
+#include <math.h>
+
+#include "fp8vit_internal.cuh"
+
+namespace {
+
+constexpr int kBM = 128;          // query rows per CTA (MMA M)
+constexpr int kBN = 128;          // keys per KV tile
+constexpr int kThreads = 192;     // 6 warps
+constexpr int kTmemCols = 256;
+constexpr uint32_t kTmemS = 0;    // S columns [0,128); P hi/lo written over [0,64)
+constexpr uint32_t kTmemO = 128;  // O accumulator columns [128, 128 + NPV)
+constexpr int kBox = 32;          // bytes per TMA box row (one SW32 atom row)
+constexpr int kTileBytes = kBox * 128;  // one [128 rows x 32 B] box
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+template <int D>
+struct Cfg;
+template <>
+struct Cfg<72> {
+    static constexpr int KB = 3;    // 32-byte k-blocks of the QK contraction (96 bytes)
+    static constexpr int VA = 3;    // 32-byte V column blocks loaded (96 bytes)
+    static constexpr int NPV = 80;  // PV MMA N (covers head bytes [0,72) or [8,80))
+    static constexpr int NS = 3;    // K/V pipeline stages
+};
+template <>
+struct Cfg<128> {
+    static constexpr int KB = 4;
+    static constexpr int VA = 4;
+    static constexpr int NPV = 128;
+    static constexpr int NS = 2;
+};
+
+template <int D>
+struct Smem {
+    static constexpr int Q = 0;
+    static constexpr int K = Q + Cfg<D>::KB * kTileBytes;
+    static constexpr int V = K + Cfg<D>::NS * Cfg<D>::KB * kTileBytes;
+    static constexpr int BAR = V + Cfg<D>::NS * Cfg<D>::VA * kTileBytes;
+    static constexpr int TOTAL = BAR + 256;
+    static constexpr int ALLOC = TOTAL + 1024;  // slack for 1024-byte alignment
+};
+
+// Shared-memory matrix descriptors (tcgen05 "version 1" format), 32-byte
+// swizzle.  K-major: rows of 32 bytes, 8-row groups 256 bytes apart (SBO).
+// MN-major: 32-byte atoms along N, 4096 bytes apart (LBO); 8-key groups
+// 256 bytes apart (SBO).
+__device__ __forceinline__ uint64_t desc_k_sw32(uint32_t addr) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(256 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)6 << 61);
+}
+__device__ __forceinline__ uint64_t desc_mn_sw32(uint32_t addr) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)(kTileBytes >> 4) << 16) |
+           ((uint64_t)(256 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)6 << 61);
+}
+
+// Instruction descriptor, kind::f8f6f4: e4m3 x e4m3 -> f32, M = 128.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int n, bool b_mn_major) {
+    return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(n >> 3) << 17) |
+           ((uint32_t)(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void tmem_ld32_sync(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld8_sync(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7])
+        : "r"(taddr)
+        : "memory");
+}
+
+// Quantize 4 probabilities (scaled to (0, 256]) into one hi word and one lo
+// word: hi = e4m3(p), lo = e4m3(p - hi); hi + lo carries ~8 mantissa bits.
+__device__ __forceinline__ void p_split4(float p0, float p1, float p2, float p3, uint32_t& hi,
+                                         uint32_t& lo) {
+    const uint16_t h01 = f32x2_to_e4m3x2(p0, p1);
+    const uint16_t h23 = f32x2_to_e4m3x2(p2, p3);
+    const float2 b01 = e4m3x2_to_f32x2(h01);
+    const float2 b23 = e4m3x2_to_f32x2(h23);
+    const uint16_t l01 = f32x2_to_e4m3x2(p0 - b01.x, p1 - b01.y);
+    const uint16_t l23 = f32x2_to_e4m3x2(p2 - b23.x, p3 - b23.y);
+    hi = (uint32_t)h01 | ((uint32_t)h23 << 16);
+    lo = (uint32_t)l01 | ((uint32_t)l23 << 16);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 2)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ dq_p,
+                    const float* __restrict__ dk_p, const float* __restrict__ dv_p,
+                    const int32_t* __restrict__ cu, int32_t max_seqlen, int64_t total_tokens,
+                    int32_t num_heads, float sm_scale, void* __restrict__ out, int32_t out_fp8,
+                    const float* __restrict__ out_scale_p, fp8vit_scratch* __restrict__ scr) {
+    using C = Cfg<D>;
+    using L = Smem<D>;
+    constexpr int NS = C::NS;
+
+    const int qt = blockIdx.x, h = blockIdx.y, seg = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    const int32_t seg_start = cu[seg];
+    const int32_t seg_end = cu[seg + 1];
+    const int32_t seg_len = seg_end - seg_start;
+    if (seg_start < 0 || seg_len < 0 || seg_len > max_seqlen || (int64_t)seg_end > total_tokens) {
+        if (threadIdx.x == 0 && qt == 0 && h == 0)
+            fp8vit_report(scr, FP8VIT_EINVAL, SITE_ATTN_SEQLENS);
+        return;
+    }
+    const int q0 = qt * kBM;
+    if (q0 >= seg_len) return;
+    const int n_kv = (seg_len + kBN - 1) / kBN;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sQ = smem_u32(sm + L::Q);
+    const uint32_t sK = smem_u32(sm + L::K);
+    const uint32_t sV = smem_u32(sm + L::V);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR);
+    const uint32_t bar0 = smem_u32(bars);
+    // barrier indices
+    const uint32_t b_q_full = bar0 + 8 * 0;
+    const uint32_t b_q_ready = bar0 + 8 * 1;
+    const uint32_t b_s_full = bar0 + 8 * 2;
+    const uint32_t b_p_full = bar0 + 8 * 3;
+    const uint32_t b_o_ready = bar0 + 8 * 4;
+    auto b_k_full = [&](int s) { return bar0 + 8 * (5 + s); };
+    auto b_v_full = [&](int s) { return bar0 + 8 * (5 + NS + s); };
+    auto b_kv_empty = [&](int s) { return bar0 + 8 * (5 + 2 * NS + s); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::BAR + 8 * (5 + 3 * NS));
+    volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
+
+    if (threadIdx.x == 0) {
+        mbar_init(b_q_full, 1);
+        mbar_init(b_q_ready, 128);
+        mbar_init(b_s_full, 1);
+        mbar_init(b_p_full, 128);
+        mbar_init(b_o_ready, 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(b_k_full(s), 1);
+            mbar_init(b_v_full(s), 1);
+            mbar_init(b_kv_empty(s), 1);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // x coordinate (bytes) of the head's window: head offset rounded down to 16.
+    const int32_t x0 = (h * D) & ~15;
+    const int col_off = h * D - x0;  // 0, or 8 for odd heads at D = 72
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+            mbar_arrive_expect_tx(b_q_full, C::KB * kTileBytes);
+            for (int kb = 0; kb < C::KB; ++kb)
+                tma_load_2d(sQ + kb * kTileBytes, &tm_q, x0 + kBox * kb, seg_start + q0, b_q_full);
+            int issued = 0;
+            for (int j = 0; j < n_kv; ++j) {
+                const int s = j % NS;
+                if (j >= NS &&
+                    !mbar_wait_bounded(b_kv_empty(s), ((j / NS) - 1) & 1, abort_flag, scr,
+                                       SITE_ATTN_WAIT_EMPTY, kTimeoutNs))
+                    break;
+                const int32_t row = seg_start + j * kBN;
+                mbar_arrive_expect_tx(b_k_full(s), C::KB * kTileBytes);
+                for (int kb = 0; kb < C::KB; ++kb)
+                    tma_load_2d(sK + (s * C::KB + kb) * kTileBytes, &tm_k, x0 + kBox * kb, row,
+                                b_k_full(s));
+                mbar_arrive_expect_tx(b_v_full(s), C::VA * kTileBytes);
+                for (int a = 0; a < C::VA; ++a)
+                    tma_load_2d(sV + (s * C::VA + a) * kTileBytes, &tm_v, x0 + kBox * a, row,
+                                b_v_full(s));
+                ++issued;
+            }
+            // Drain: every issued copy must land before the CTA may exit.
+            mbar_wait_bounded(b_q_full, 0, abort_flag, scr, SITE_ATTN_DRAIN, kTimeoutNs);
+            for (int j = issued - 1; j >= 0 && j >= issued - NS; --j) {
+                const int s = j % NS;
+                mbar_wait_bounded(b_k_full(s), (j / NS) & 1, abort_flag, scr, SITE_ATTN_DRAIN,
+                                  kTimeoutNs);
+                mbar_wait_bounded(b_v_full(s), (j / NS) & 1, abort_flag, scr, SITE_ATTN_DRAIN,
+                                  kTimeoutNs);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_e4m3(kBN, false);
+            constexpr uint32_t idesc_pv = idesc_e4m3(C::NPV, true);
+            const uint32_t tS = tmem + kTmemS, tO = tmem + kTmemO;
+            bool ok = mbar_wait_bounded(b_q_ready, 0, abort_flag, scr, SITE_ATTN_WAIT_QREADY,
+                                        kTimeoutNs);
+            int committed = 0;  // number of o_ready commits issued
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int s = j % NS;
+                const uint32_t ph = (j / NS) & 1;
+                if (!mbar_wait_bounded(b_k_full(s), ph, abort_flag, scr, SITE_ATTN_WAIT_K,
+                                       kTimeoutNs))
+                    break;
+                // S may be overwritten only after PV of the previous tile has
+                // read P out of it.
+                if (j > 0 && !mbar_wait_bounded(b_o_ready, (j - 1) & 1, abort_flag, scr,
+                                                SITE_ATTN_WAIT_O, kTimeoutNs))
+                    break;
+                tc_fence_after();
+#pragma unroll
+                for (int kb = 0; kb < C::KB; ++kb)
+                    umma_f8_ss(tS, desc_k_sw32(sQ + kb * kTileBytes),
+                               desc_k_sw32(sK + (s * C::KB + kb) * kTileBytes), idesc_qk,
+                               kb > 0 ? 1u : 0u);
+                umma_commit(b_s_full);
+                if (!mbar_wait_bounded(b_v_full(s), ph, abort_flag, scr, SITE_ATTN_WAIT_V,
+                                       kTimeoutNs))
+                    break;
+                if (!mbar_wait_bounded(b_p_full, j & 1, abort_flag, scr, SITE_ATTN_WAIT_P,
+                                       kTimeoutNs))
+                    break;
+                tc_fence_after();
+                const uint32_t vbase = sV + s * C::VA * kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < kBN / 32; ++kk) {
+                    const uint64_t bdesc = desc_mn_sw32(vbase + kk * 32 * kBox);
+                    umma_f8_ts(tO, tS + 16 * kk, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_f8_ts(tO, tS + 16 * kk + 8, bdesc, idesc_pv, 1u);
+                }
+                umma_commit(b_o_ready);
+                umma_commit(b_kv_empty(s));
+                ++committed;
+            }
+            // Never leave MMAs in flight: wait for the last commit.
+            if (committed > 0)
+                mbar_wait_bounded(b_o_ready, (committed - 1) & 1, abort_flag, scr,
+                                  SITE_ATTN_DRAIN, kTimeoutNs);
+        }
+    } else {
+        // ---------------- softmax + epilogue (warps 2..5) ----------------
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;  // query row in the tile == TMEM lane
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        const uint32_t tS = lane_base + kTmemS, tO = lane_base + kTmemO;
+        const float dq = *dq_p, dk = *dk_p, dv = *dv_p;
+        const float scale_log2 = sm_scale * dq * dk * 1.4426950408889634f;
+
+        bool ok = mbar_wait_bounded(b_q_full, 0, abort_flag, scr, SITE_ATTN_WAIT_Q, kTimeoutNs);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (ok && D == 72) {
+            // Zero the window bytes outside this head: [72,96) for even heads,
+            // [0,8) and [80,96) for odd heads.  SW32 layout: row r of k-block
+            // kb at kb*4096 + r*32, 16-byte chunk c stored at chunk c ^ ((r>>2)&1).
+            uint8_t* q = sm + L::Q;
+            const int sw = (row >> 2) & 1;
+            uint8_t* kb2 = q + 2 * kTileBytes + row * kBox;
+            *reinterpret_cast<uint4*>(kb2 + ((1 ^ sw) << 4)) = make_uint4(0, 0, 0, 0);
+            if (col_off == 0)
+                *reinterpret_cast<uint2*>(kb2 + ((0 ^ sw) << 4) + 8) = make_uint2(0, 0);
+            else
+                *reinterpret_cast<uint2*>(q + row * kBox + ((0 ^ sw) << 4)) = make_uint2(0, 0);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(b_q_ready);
+
+        float m_run = -INFINITY, l_run = 0.0f;
+        for (int j = 0; ok && j < n_kv; ++j) {
+            ok = mbar_wait_bounded(b_s_full, j & 1, abort_flag, scr, SITE_ATTN_WAIT_S, kTimeoutNs);
+            ok = __all_sync(0xFFFFFFFFu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            const int nvalid = min(kBN, seg_len - j * kBN);
+            // pass 1: row max over the valid keys
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < kBN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32_sync(tS + 32 * c, r);
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (32 * c + i < nvalid) mx = fmaxf(mx, __uint_as_float(r[i]));
+            }
+            const float m_new = fmaxf(m_run, mx);
+            const bool need = (j > 0) && (m_new > m_run);
+            if (__any_sync(0xFFFFFFFFu, need)) {
+                ok = mbar_wait_bounded(b_o_ready, (j - 1) & 1, abort_flag, scr, SITE_ATTN_WAIT_O,
+                                       kTimeoutNs);
+                ok = __all_sync(0xFFFFFFFFu, ok);
+                if (!ok) break;
+                tc_fence_after();
+                const float alpha = need ? ex2_approx((m_run - m_new) * scale_log2) : 1.0f;
+#pragma unroll
+                for (int c = 0; c < C::NPV / 8; ++c) {
+                    uint32_t r[8];
+                    tmem_ld8_sync(tO + 8 * c, r);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                    tmem_st8(tO + 8 * c, r);
+                }
+                tmem_wait_st();
+                l_run *= alpha;
+            }
+            m_run = m_new;
+            // p = 2^(s*scale_log2 - m*scale_log2 + 8): probabilities scaled to (0, 256]
+            const float bias = m_new * scale_log2 - 8.0f;
+#pragma unroll
+            for (int c = 0; c < kBN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32_sync(tS + 32 * c, r);
+                float p[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    p[i] = (32 * c + i < nvalid)
+                               ? ex2_approx(fmaf(__uint_as_float(r[i]), scale_log2, -bias))
+                               : 0.0f;
+                    l_run += p[i];
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int w = 0; w < 8; ++w)
+                    p_split4(p[4 * w], p[4 * w + 1], p[4 * w + 2], p[4 * w + 3], pk[w], pk[8 + w]);
+                tmem_st16(tS + 16 * c, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(b_p_full);
+        }
+        // epilogue
+        if (ok) {
+            ok = mbar_wait_bounded(b_o_ready, (n_kv - 1) & 1, abort_flag, scr, SITE_ATTN_WAIT_O,
+                                   kTimeoutNs);
+            ok = __all_sync(0xFFFFFFFFu, ok);
+        }
+        if (ok) {
+            tc_fence_after();
+            const bool valid = (q0 + row) < seg_len;
+            const float inv = __fdiv_rn(dv, l_run);
+            const int64_t tok = (int64_t)seg_start + q0 + row;
+            const int64_t off = (tok * num_heads + h) * D;
+            const float oscale = out_fp8 ? *out_scale_p : 1.0f;
+#pragma unroll
+            for (int c = 0; c < D / 8; ++c) {
+                uint32_t r[8];
+                tmem_ld8_sync(tO + col_off + 8 * c, r);
+                float o[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) o[i] = __uint_as_float(r[i]) * inv;
+                if (!valid) continue;
+                if (out_fp8) {
+                    uint32_t w0 = (uint32_t)f32x2_to_e4m3x2(__fdiv_rn(o[0], oscale), __fdiv_rn(o[1], oscale)) |
+                                  ((uint32_t)f32x2_to_e4m3x2(__fdiv_rn(o[2], oscale), __fdiv_rn(o[3], oscale)) << 16);
+                    uint32_t w1 = (uint32_t)f32x2_to_e4m3x2(__fdiv_rn(o[4], oscale), __fdiv_rn(o[5], oscale)) |
+                                  ((uint32_t)f32x2_to_e4m3x2(__fdiv_rn(o[6], oscale), __fdiv_rn(o[7], oscale)) << 16);
+                    *reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(out) + off + 8 * c) =
+                        make_uint2(w0, w1);
+                } else {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        __nv_bfloat162 b = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
+                        w[i] = *reinterpret_cast<uint32_t*>(&b);
+                    }
+                    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out) + off + 8 * c) =
+                        make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+bool encode_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_bytes) {
+    fp8vit_encode_tiled_fn enc = fp8vit_get_encode_tiled();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    const cuuint32_t box[2] = {(cuuint32_t)kBox, (cuuint32_t)kBM};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+fp8vit_status launch(fp8vit_ctx* ctx, const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
+                     const float* dq, const float* dk, const float* dv, const int32_t* cu,
+                     int32_t num_seqs, int32_t max_seqlen, int64_t T, int32_t H, float sm_scale,
+                     void* out, int32_t out_fp8, const float* out_scale, cudaStream_t st) {
+    CUtensorMap mq, mk, mv;
+    const int64_t row_bytes = (int64_t)H * D;
+    if (!encode_map(&mq, q8, T, row_bytes) || !encode_map(&mk, k8, T, row_bytes) ||
+        !encode_map(&mv, v8, T, row_bytes))
+        return FP8VIT_ECUDA;
+    static bool attr_set[2] = {false, false};  // per template instance (one device set-up)
+    auto kern = attn_fwd_kernel<D>;
+    if (!attr_set[D == 128]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Smem<D>::ALLOC) != cudaSuccess)
+            return FP8VIT_ECUDA;
+        attr_set[D == 128] = true;
+    }
+    dim3 grid((unsigned)((max_seqlen + kBM - 1) / kBM), (unsigned)H, (unsigned)num_seqs);
+    kern<<<grid, kThreads, Smem<D>::ALLOC, st>>>(mq, mk, mv, dq, dk, dv, cu, max_seqlen, T, H,
+                                                 sm_scale, out, out_fp8, out_scale,
+                                                 ctx->d_scratch);
+    return cudaGetLastError() == cudaSuccess ? FP8VIT_OK : FP8VIT_ECUDA;
+}
+
+inline bool misaligned(const void* p, uintptr_t a) {
+    return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0;
+}
+
+}  // namespace
+
+extern "C" fp8vit_status fp8_varlen_attn_fwd(
+    fp8vit_ctx* ctx, const uint8_t* d_q8, const uint8_t* d_k8, const uint8_t* d_v8,
+    const float* d_q_descale, const float* d_k_descale, const float* d_v_descale,
+    const int32_t* d_cu_seqlens, int32_t num_seqs, int32_t max_seqlen, int64_t total_tokens,
+    int32_t num_heads, int32_t head_dim, float softmax_scale, void* d_out, int32_t out_dtype,
+    const float* d_output_scale, void* stream) {
+    if (!ctx || !d_q8 || !d_k8 || !d_v8 || !d_q_descale || !d_k_descale || !d_v_descale ||
+        !d_cu_seqlens || !d_out)
+        return FP8VIT_EINVAL;
+    if (num_seqs < 0 || max_seqlen < 0 || total_tokens < 0 || total_tokens > INT32_MAX ||
+        num_heads < 1)
+        return FP8VIT_EINVAL;
+    if (!(softmax_scale > 0.0f) || !isfinite(softmax_scale)) return FP8VIT_EINVAL;
+    if (out_dtype != 0 && out_dtype != 1) return FP8VIT_EINVAL;
+    if ((out_dtype == 1) != (d_output_scale != nullptr)) return FP8VIT_EINVAL;
+    if (head_dim != 72 && head_dim != 128) return FP8VIT_EUNSUPPORTED;
+    if (((int64_t)num_heads * head_dim) % 16 != 0) return FP8VIT_EUNSUPPORTED;
+    if (misaligned(d_q8, 16) || misaligned(d_k8, 16) || misaligned(d_v8, 16) ||
+        misaligned(d_out, out_dtype == 0 ? 16 : 8) || misaligned(d_cu_seqlens, 4))
+        return FP8VIT_EINVAL;
+    if (num_heads > 65535 || num_seqs > 65535) return FP8VIT_EUNSUPPORTED;
+    if (num_seqs == 0 || max_seqlen == 0 || total_tokens == 0) return FP8VIT_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (head_dim == 72)
+        return launch<72>(ctx, d_q8, d_k8, d_v8, d_q_descale, d_k_descale, d_v_descale,
+                          d_cu_seqlens, num_seqs, max_seqlen, total_tokens, num_heads,
+                          softmax_scale, d_out, out_dtype, d_output_scale, st);
+    return launch<128>(ctx, d_q8, d_k8, d_v8, d_q_descale, d_k_descale, d_v_descale, d_cu_seqlens,
+                       num_seqs, max_seqlen, total_tokens, num_heads, softmax_scale, d_out,
+                       out_dtype, d_output_scale, st);
+}

@@ -1,0 +1,266 @@
+// HBM-bound kernels of the path:
+//   amax_ring_kernel   -- amax of q, k, v + 16-slot ring update + descales
+//                         (vLLM "FP8 ViT Encoder Attention", Usage: dynamic scaling)
+//   quant3_kernel      -- per-tensor e4m3 quantization of q, k, v
+//                         (same page, intro: Q/K/V quantized right before attention)
+//   group_quant_kernel -- per-token-group e4m3 quantization with fp32 scales
+//                         (atrex-bench "#025 per_token_group_quant_fp8")
+// All three stream 16-byte vectors with grid-stride loops sized to the SM
+// count, and round with the hardware RNE-satfinite e4m3 conversion after an
+// IEEE fp32 division (x / scale, as the pages' definitions divide).
+#include "fp8vit_internal.cuh"
+
+namespace {
+
+constexpr int kAmaxThreads = 512;
+constexpr int kQuantThreads = 256;
+constexpr int kGroupThreads = 256;
+
+// Per-lane |x| max of two packed bf16 values: clear the sign bits, then an
+// unsigned max on each 16-bit half.  For non-NaN bf16, the order of the
+// magnitude bit patterns is the order of the magnitudes.
+__device__ __forceinline__ uint32_t absmax2(uint32_t acc, uint32_t w) {
+    return __vmaxu2(acc, w & 0x7FFF7FFFu);
+}
+
+__device__ __forceinline__ uint32_t absmax_vec(uint32_t acc, const uint4& x) {
+    acc = absmax2(acc, x.x);
+    acc = absmax2(acc, x.y);
+    acc = absmax2(acc, x.z);
+    return absmax2(acc, x.w);
+}
+
+__global__ void __launch_bounds__(kAmaxThreads) amax_ring_kernel(
+    const uint4* __restrict__ q, const uint4* __restrict__ k, const uint4* __restrict__ v,
+    int64_t n_elems, fp8vit_ring* __restrict__ ring, float* __restrict__ descale3,
+    fp8vit_scratch* __restrict__ scr) {
+    const int64_t nvec = n_elems >> 3;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const uint4* src[3] = {q, k, v};
+    uint32_t m[3];
+#pragma unroll
+    for (int t = 0; t < 3; ++t) {
+        const uint4* p = src[t];
+        uint32_t a0 = 0, a1 = 0;
+        int64_t i = i0;
+        for (; i + 3 * stride < nvec; i += 4 * stride) {
+            uint4 x0 = __ldcs(p + i);
+            uint4 x1 = __ldcs(p + i + stride);
+            uint4 x2 = __ldcs(p + i + 2 * stride);
+            uint4 x3 = __ldcs(p + i + 3 * stride);
+            a0 = absmax_vec(a0, x0);
+            a1 = absmax_vec(a1, x1);
+            a0 = absmax_vec(a0, x2);
+            a1 = absmax_vec(a1, x3);
+        }
+        for (; i < nvec; i += stride) a0 = absmax_vec(a0, __ldcs(p + i));
+        const int tail = (int)(n_elems & 7);
+        if (blockIdx.x == 0 && (int)threadIdx.x < tail) {
+            const uint16_t* ps = reinterpret_cast<const uint16_t*>(p);
+            a0 = absmax2(a0, ps[(nvec << 3) + threadIdx.x]);
+        }
+        a0 = __vmaxu2(a0, a1);
+        m[t] = max(a0 & 0xFFFFu, a0 >> 16);
+    }
+    __shared__ uint32_t red[3][kAmaxThreads / 32];
+    __shared__ int is_last;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int t = 0; t < 3; ++t) {
+        uint32_t w = __reduce_max_sync(0xFFFFFFFFu, m[t]);
+        if (lane == 0) red[t][warp] = w;
+    }
+    __syncthreads();
+    if (warp == 0) {
+#pragma unroll
+        for (int t = 0; t < 3; ++t) {
+            uint32_t x = lane < (int)(blockDim.x >> 5) ? red[t][lane] : 0u;
+            x = __reduce_max_sync(0xFFFFFFFFu, x);
+            if (lane == 0) atomicMax(&scr->amax_bits[t], x);
+        }
+        if (lane == 0) {
+            __threadfence();
+            unsigned ticket = atomicAdd(&scr->arrivals, 1u);
+            is_last = (ticket == gridDim.x - 1);
+        }
+    }
+    __syncthreads();
+    if (!is_last || threadIdx.x != 0) return;
+    // Last CTA: every other CTA's atomicMax is visible.  Read and clear the
+    // scratch for the next launch, then run the ring rule.
+    __threadfence();
+    float amax[3];
+#pragma unroll
+    for (int t = 0; t < 3; ++t) amax[t] = bf16_bits_to_f32(atomicExch(&scr->amax_bits[t], 0u));
+    atomicExch(&scr->arrivals, 0u);
+    int32_t p = ring->pos;
+    p = ((p % 16) + 16) % 16;
+#pragma unroll
+    for (int t = 0; t < 3; ++t) ring->hist[t][p] = amax[t];
+    ring->pos = (p + 1) & 15;
+#pragma unroll
+    for (int t = 0; t < 3; ++t) {
+        float mx = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) mx = ring->hist[t][j] > mx ? ring->hist[t][j] : mx;
+        float d = __fdiv_rn(mx, 448.0f);
+        descale3[t] = d > 1e-10f ? d : 1e-10f;
+    }
+}
+
+// 8 bf16 (one 16-byte vector) / scale -> 8 e4m3 codes (8 bytes).
+__device__ __forceinline__ uint2 quant8(const uint4& x, float s) {
+    uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t c[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float lo = __fdiv_rn(__uint_as_float(w[i] << 16), s);
+        float hi = __fdiv_rn(__uint_as_float(w[i] & 0xFFFF0000u), s);
+        c[i] = f32x2_to_e4m3x2(lo, hi);
+    }
+    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+__global__ void __launch_bounds__(kQuantThreads) quant3_kernel(
+    const uint4* __restrict__ q, const uint4* __restrict__ k, const uint4* __restrict__ v,
+    int64_t n_elems, const float* __restrict__ descale3, uint2* __restrict__ q8,
+    uint2* __restrict__ k8, uint2* __restrict__ v8) {
+    const int64_t nvec = n_elems >> 3;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const uint4* src[3] = {q, k, v};
+    uint2* dst[3] = {q8, k8, v8};
+#pragma unroll
+    for (int t = 0; t < 3; ++t) {
+        const float s = descale3[t];
+        const uint4* p = src[t];
+        uint2* o = dst[t];
+        int64_t i = i0;
+        for (; i + stride < nvec; i += 2 * stride) {
+            uint4 x0 = __ldcs(p + i);
+            uint4 x1 = __ldcs(p + i + stride);
+            __stcs(o + i, quant8(x0, s));
+            __stcs(o + i + stride, quant8(x1, s));
+        }
+        if (i < nvec) __stcs(o + i, quant8(__ldcs(p + i), s));
+        const int tail = (int)(n_elems & 7);
+        if (blockIdx.x == 0 && (int)threadIdx.x < tail) {
+            const uint16_t* ps = reinterpret_cast<const uint16_t*>(p);
+            uint8_t* os = reinterpret_cast<uint8_t*>(o);
+            const int64_t e = (nvec << 3) + threadIdx.x;
+            float y = __fdiv_rn(bf16_bits_to_f32(ps[e]), s);
+            os[e] = (uint8_t)(f32x2_to_e4m3x2(y, 0.0f) & 0xFF);
+        }
+    }
+}
+
+// LPG = lanes per group = group / 8; each lane owns one 16-byte vector of
+// its group; a warp covers 32 / LPG groups per iteration.
+template <int LPG>
+__global__ void __launch_bounds__(kGroupThreads) group_quant_kernel(
+    const uint4* __restrict__ x, int64_t total_groups, uint2* __restrict__ xq,
+    float* __restrict__ scales) {
+    constexpr int kGPW = 32 / LPG;
+    const int lane = threadIdx.x & 31;
+    const int sub = lane / LPG, gl = lane % LPG;
+    const int64_t warp_id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t g0 = warp_id * kGPW; g0 < total_groups; g0 += nwarps * kGPW) {
+        const int64_t g = g0 + sub;
+        const bool valid = g < total_groups;
+        uint4 xv = valid ? __ldcs(x + g * LPG + gl) : make_uint4(0, 0, 0, 0);
+        uint32_t a = absmax_vec(0u, xv);
+        a = max(a & 0xFFFFu, a >> 16);
+#pragma unroll
+        for (int off = LPG / 2; off > 0; off >>= 1)
+            a = max(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+        float s = __fdiv_rn(bf16_bits_to_f32(a), 448.0f);
+        s = s > 1e-10f ? s : 1e-10f;
+        if (valid) {
+            __stcs(xq + g * LPG + gl, quant8(xv, s));
+            if (gl == 0) scales[g] = s;
+        }
+    }
+}
+
+inline bool misaligned(const void* p, uintptr_t a) {
+    return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0;
+}
+
+inline int grid_for(int64_t work_items, int threads, int per_thread, int max_blocks) {
+    int64_t b = (work_items + (int64_t)threads * per_thread - 1) / ((int64_t)threads * per_thread);
+    if (b < 1) b = 1;
+    if (b > max_blocks) b = max_blocks;
+    return (int)b;
+}
+
+}  // namespace
+
+extern "C" {
+
+fp8vit_status fp8_amax_ring_update(fp8vit_ctx* ctx, const uint16_t* d_q, const uint16_t* d_k,
+                                   const uint16_t* d_v, int64_t n_elems, void* d_ring,
+                                   float* d_descale3, void* stream) {
+    if (!ctx || !d_q || !d_k || !d_v || !d_ring || !d_descale3 || n_elems < 0)
+        return FP8VIT_EINVAL;
+    if (misaligned(d_q, 16) || misaligned(d_k, 16) || misaligned(d_v, 16) ||
+        misaligned(d_ring, 16) || misaligned(d_descale3, 4))
+        return FP8VIT_EINVAL;
+    const int grid = grid_for(n_elems >> 3, kAmaxThreads, 8, 4 * ctx->num_sms);
+    amax_ring_kernel<<<grid, kAmaxThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const uint4*>(d_q), reinterpret_cast<const uint4*>(d_k),
+        reinterpret_cast<const uint4*>(d_v), n_elems, reinterpret_cast<fp8vit_ring*>(d_ring),
+        d_descale3, ctx->d_scratch);
+    return cudaGetLastError() == cudaSuccess ? FP8VIT_OK : FP8VIT_ECUDA;
+}
+
+fp8vit_status fp8_quantize_qkv_per_tensor(fp8vit_ctx* ctx, const uint16_t* d_q,
+                                          const uint16_t* d_k, const uint16_t* d_v,
+                                          int64_t n_elems, const float* d_descale3, uint8_t* d_q8,
+                                          uint8_t* d_k8, uint8_t* d_v8, void* stream) {
+    if (!ctx || !d_q || !d_k || !d_v || !d_descale3 || !d_q8 || !d_k8 || !d_v8 || n_elems < 0)
+        return FP8VIT_EINVAL;
+    if (misaligned(d_q, 16) || misaligned(d_k, 16) || misaligned(d_v, 16) ||
+        misaligned(d_q8, 8) || misaligned(d_k8, 8) || misaligned(d_v8, 8) ||
+        misaligned(d_descale3, 4))
+        return FP8VIT_EINVAL;
+    const int grid = grid_for(n_elems >> 3, kQuantThreads, 4, 8 * ctx->num_sms);
+    quant3_kernel<<<grid, kQuantThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const uint4*>(d_q), reinterpret_cast<const uint4*>(d_k),
+        reinterpret_cast<const uint4*>(d_v), n_elems, d_descale3, reinterpret_cast<uint2*>(d_q8),
+        reinterpret_cast<uint2*>(d_k8), reinterpret_cast<uint2*>(d_v8));
+    return cudaGetLastError() == cudaSuccess ? FP8VIT_OK : FP8VIT_ECUDA;
+}
+
+fp8vit_status per_token_group_quant_fp8(fp8vit_ctx* ctx, const uint16_t* d_x, int64_t m,
+                                        int64_t n, int32_t group, uint8_t* d_xq,
+                                        float* d_scales, void* stream) {
+    if (!ctx || !d_x || !d_xq || !d_scales || m < 0 || n < 0 || group <= 0) return FP8VIT_EINVAL;
+    if (n % group != 0) return FP8VIT_EINVAL;
+    if (group != 16 && group != 32 && group != 64 && group != 128 && group != 256)
+        return FP8VIT_EUNSUPPORTED;
+    if (misaligned(d_x, 16) || misaligned(d_xq, 8) || misaligned(d_scales, 4))
+        return FP8VIT_EINVAL;
+    if (m != 0 && n > INT64_MAX / m) return FP8VIT_EINVAL;
+    const int64_t total_groups = m * (n / group);
+    if (total_groups == 0) return FP8VIT_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int lpg = group / 8;
+    const int64_t gpw = 32 / (lpg > 0 ? lpg : 1);
+    const int grid = grid_for((total_groups + gpw - 1) / gpw * 32, kGroupThreads, 4,
+                              8 * ctx->num_sms);
+    const uint4* x = reinterpret_cast<const uint4*>(d_x);
+    uint2* xq = reinterpret_cast<uint2*>(d_xq);
+    switch (group) {
+        case 16: group_quant_kernel<2><<<grid, kGroupThreads, 0, st>>>(x, total_groups, xq, d_scales); break;
+        case 32: group_quant_kernel<4><<<grid, kGroupThreads, 0, st>>>(x, total_groups, xq, d_scales); break;
+        case 64: group_quant_kernel<8><<<grid, kGroupThreads, 0, st>>>(x, total_groups, xq, d_scales); break;
+        case 128: group_quant_kernel<16><<<grid, kGroupThreads, 0, st>>>(x, total_groups, xq, d_scales); break;
+        case 256: group_quant_kernel<32><<<grid, kGroupThreads, 0, st>>>(x, total_groups, xq, d_scales); break;
+        default: return FP8VIT_EUNSUPPORTED;
+    }
+    return cudaGetLastError() == cudaSuccess ? FP8VIT_OK : FP8VIT_ECUDA;
+}
+
+}  // extern "C"

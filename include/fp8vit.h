@@ -1,0 +1,187 @@
+/*
+ * fp8vit.h -- C ABI of libfp8vit.so, the B200 (sm_100a) FP8 vision-encoder
+ * attention path.
+ *
+ * What the path computes (web sources cited by title and section):
+ *   - vLLM docs "FP8 ViT Encoder Attention", intro and Usage: BF16 Q/K/V are
+ *     quantized to FP8 e4m3 with one scale per tensor right before the
+ *     attention call.  Without a scale file the scale is dynamic: a 16-entry
+ *     circular buffer of the observed Q/K/V amax drives the per-forward
+ *     scale.  With a scale file (section "Scale File Format", saved with the
+ *     --mm-encoder-fp8-scale-save-margin of 1.5) the scales are static.
+ *     Packed variable-length image batches attend without crossing images.
+ *   - vLLM issue "[Feature]: Add support for fused fp8 output to FlashAttention
+ *     3", Description: an output_scale argument makes attention write FP8.
+ *   - atrex-bench "#025 per_token_group_quant_fp8", Reference Implementation:
+ *     the per-token-group quantizer that feeds an FP8 o-proj.
+ *
+ * Conventions (every entry point):
+ *   - A pointer named d_* is DEVICE memory, allocated and owned by the caller.
+ *     The library allocates device memory only in fp8vit_create (its context
+ *     scratch) and nothing per call.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Device work is enqueued asynchronously on it; the call returns
+ *     after the launch.
+ *   - BF16 tensors are uint16_t bit patterns; FP8 tensors are uint8_t e4m3fn
+ *     codes (OCP E4M3: bias 7, max +-448, no infinities, NaN = S.1111.111).
+ *   - Activation layout: packed [T, H, D] row-major (== [T, H*D]); T counts
+ *     the tokens of all images.
+ *   - "descale" is the dequantisation multiplier of a per-tensor FP8 tensor:
+ *     value ~= code * descale, descale = max(amax / 448, 1e-10) (the group
+ *     quantizer page calls the same quantity "scales").
+ *   - Host-side argument checks return at once with FP8VIT_EINVAL (null or
+ *     misaligned pointer, negative or overflowing size) or
+ *     FP8VIT_EUNSUPPORTED (a shape the kernels do not implement).  Faults the
+ *     GPU detects (bad cu_seqlens, a bounded wait that timed out) are
+ *     recorded in the context's device status word; fp8vit_check() returns
+ *     the first one.
+ */
+#ifndef FP8VIT_H
+#define FP8VIT_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP8VIT_OK = 0,
+    FP8VIT_EINVAL = 1,       /* bad argument (host) or bad cu_seqlens (device)      */
+    FP8VIT_EUNSUPPORTED = 2, /* shape/mode not implemented (e.g. head_dim not 72/128) */
+    FP8VIT_ECUDA = 3,        /* a CUDA runtime/driver call failed                    */
+    FP8VIT_EIO = 4,          /* scale file could not be opened/written               */
+    FP8VIT_EPARSE = 5,       /* scale file is not the documented JSON format          */
+    FP8VIT_ENOTFOUND = 6,    /* layer name absent from the scale file                */
+    FP8VIT_ETIMEOUT = 7      /* a bounded wait inside a kernel gave up                */
+} fp8vit_status;
+
+typedef struct fp8vit_ctx fp8vit_ctx;
+
+/* ---- context ------------------------------------------------------------ */
+
+/* Create a context on CUDA device `device` (made current by the call).  The
+ * context owns a device status word and the amax reduction scratch used by
+ * fp8_amax_ring_update.  One context must not be used by two streams at the
+ * same time (the scratch is shared).  *out is NULL on failure. */
+fp8vit_status fp8vit_create(int32_t device, fp8vit_ctx** out);
+
+/* Free the context's device memory.  NULL is accepted. */
+fp8vit_status fp8vit_destroy(fp8vit_ctx* ctx);
+
+/* Synchronize `stream`, then return and clear the first fault recorded on the
+ * device since the last check (FP8VIT_OK if none).  *site, if not NULL,
+ * receives a kernel-specific location code of that fault (0 if none). */
+fp8vit_status fp8vit_check(fp8vit_ctx* ctx, void* stream, int32_t* site);
+
+const char* fp8vit_status_string(fp8vit_status s);
+
+/* Library ABI version (major * 100 + minor). */
+int32_t fp8vit_version(void);
+
+/* ---- dynamic scaling: amax ring (vLLM "FP8 ViT Encoder Attention", Usage) --- */
+
+/* Size in bytes of one ring state: float hist[3][16] (rows q, k, v), then an
+ * int32 write position shared by the three rows, padded to 256 bytes. */
+#define FP8VIT_RING_BYTES 256
+
+/* Zero a ring state (all slots 0, position 0) on `stream`. */
+fp8vit_status fp8vit_ring_init(void* d_ring, void* stream);
+
+/* One forward of dynamic scaling for q, k and v in a single launch:
+ *   amax_t = max |x_t| over all n_elems elements of tensor t (exact);
+ *   hist[t][pos] = amax_t for t = q, k, v;  pos = (pos + 1) mod 16;
+ *   d_descale3[t] = max(max_j hist[t][j] / 448, 1e-10)   (fp32 division).
+ * The current forward's amax is in the ring before its scale is taken.
+ * d_q, d_k, d_v: BF16 [n_elems], 16-byte aligned.  d_ring: FP8VIT_RING_BYTES
+ * bytes, 16-byte aligned.  d_descale3: float[3] written.  Nothing returns to
+ * the host (no synchronisation). */
+fp8vit_status fp8_amax_ring_update(fp8vit_ctx* ctx, const uint16_t* d_q, const uint16_t* d_k,
+                                   const uint16_t* d_v, int64_t n_elems, void* d_ring,
+                                   float* d_descale3, void* stream);
+
+/* Host helper for the calibrate-once workflow (vLLM "FP8 ViT Encoder
+ * Attention", "Calibrate-Once, Reuse Workflow"): synchronize `stream`, copy
+ * the ring state to the host and return max_j hist[t][j] for t = q, k, v. */
+fp8vit_status fp8_ring_read_amax(const void* d_ring, float out_amax3[3], void* stream);
+
+/* ---- per-tensor quantization (vLLM "FP8 ViT Encoder Attention", intro) ---- */
+
+/* x8 = e4m3_rn_satfinite(float(x) / descale_t) for t = q, k, v, with an IEEE
+ * fp32 division, round-to-nearest-even and saturation to +-448.  d_descale3:
+ * float[3] (q, k, v) in device memory, e.g. from fp8_amax_ring_update or the
+ * static scales.  Inputs BF16 [n_elems] 16-byte aligned; outputs e4m3 codes
+ * [n_elems], 8-byte aligned. */
+fp8vit_status fp8_quantize_qkv_per_tensor(fp8vit_ctx* ctx, const uint16_t* d_q,
+                                          const uint16_t* d_k, const uint16_t* d_v,
+                                          int64_t n_elems, const float* d_descale3, uint8_t* d_q8,
+                                          uint8_t* d_k8, uint8_t* d_v8, void* stream);
+
+/* ---- varlen FP8 attention (vLLM "FP8 ViT Encoder Attention"; vLLM issue
+ *      "fused fp8 output for FlashAttention 3") ------------------------------ */
+
+/* Non-causal attention over cu_seqlens-packed images, FP8 QK^T and PV on the
+ * tensor cores with fp32 accumulation and online softmax:
+ *   for each image i, head h and query row r of image i:
+ *     s_j = softmax_scale * dq * dk * <q8[r,h,:], k8[j,h,:]>   (keys j of image i)
+ *     o[r,h,:] = sum_j softmax(s)_j * dv * v8[j,h,:]
+ * d_q8, d_k8, d_v8: e4m3 [total_tokens, num_heads, head_dim], 16-byte aligned.
+ * d_q_descale, d_k_descale, d_v_descale: one float each, device memory.
+ * d_cu_seqlens: int32 [num_seqs + 1], non-decreasing, cu[num_seqs] <=
+ *   total_tokens, every image length <= max_seqlen (checked on the device;
+ *   a violation records FP8VIT_EINVAL and skips that image).  Images of
+ *   length 0 are allowed.
+ * head_dim: 72 or 128 (others: FP8VIT_EUNSUPPORTED).  Any num_heads >= 1.
+ * out_dtype 0: d_out is BF16 [total_tokens, num_heads, head_dim] and
+ *   d_output_scale must be NULL.
+ * out_dtype 1: d_out is e4m3 [same shape], out = e4m3_rn_satfinite(o /
+ *   *d_output_scale), d_output_scale a device float.
+ * Rows of d_out outside [cu[0], cu[num_seqs]) are not written. */
+fp8vit_status fp8_varlen_attn_fwd(fp8vit_ctx* ctx, const uint8_t* d_q8, const uint8_t* d_k8,
+                                  const uint8_t* d_v8, const float* d_q_descale,
+                                  const float* d_k_descale, const float* d_v_descale,
+                                  const int32_t* d_cu_seqlens, int32_t num_seqs,
+                                  int32_t max_seqlen, int64_t total_tokens, int32_t num_heads,
+                                  int32_t head_dim, float softmax_scale, void* d_out,
+                                  int32_t out_dtype, const float* d_output_scale, void* stream);
+
+/* ---- per-token-group quantizer (atrex-bench "#025 per_token_group_quant_fp8",
+ *      Reference Implementation) --------------------------------------------- */
+
+/* For each row r < m and each group g of `group` consecutive columns of the
+ * row-major BF16 matrix d_x [m, n]:
+ *   amax = max |x|;  scale = max(amax / 448, 1e-10)  (fp32 division)
+ *   d_xq[r, c] = e4m3_rn_satfinite(x[r, c] / scale)  (fp32 division)
+ *   d_scales[r, g] = scale                            (fp32, [m, n/group])
+ * group in {16, 32, 64, 128, 256}; n % group == 0 (else FP8VIT_EINVAL).
+ * d_x 16-byte aligned, d_xq 8-byte aligned, d_scales 4-byte aligned. */
+fp8vit_status per_token_group_quant_fp8(fp8vit_ctx* ctx, const uint16_t* d_x, int64_t m,
+                                        int64_t n, int32_t group, uint8_t* d_xq,
+                                        float* d_scales, void* stream);
+
+/* ---- static scales (vLLM "FP8 ViT Encoder Attention", "Scale File Format"
+ *      and the 1.5 save margin) -------------------------------------------- */
+
+/* Read the q, k, v numbers of `layer` from the JSON scale file at `path`:
+ *   { "<layer>": {"q": a, "k": b, "v": c}, ... }
+ * with "q_scale"/"k_scale"/"v_scale" accepted as aliases (both spellings
+ * with different values is FP8VIT_EPARSE).  The numbers are in the amax
+ * domain (margin x observed amax); fp8_descale_from_amax turns one into a
+ * descale.  Host only; no CUDA call. */
+fp8vit_status fp8_static_scales_load(const char* path, const char* layer, float out_qkv[3]);
+
+/* Write the scale file for n_layers layers: layer i gets
+ * {"q": margin*qkv_amax[3i], "k": margin*qkv_amax[3i+1], "v": margin*qkv_amax[3i+2]}
+ * (fp32 products, printed so they read back exactly).  Host only. */
+fp8vit_status fp8_static_scales_save(const char* path, int32_t n_layers,
+                                     const char* const* layers, const float* qkv_amax,
+                                     float margin);
+
+/* max(v / 448, 1e-10) in fp32: the descale for a value v of the amax domain. */
+float fp8_descale_from_amax(float v);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8VIT_H */

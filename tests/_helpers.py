@@ -1,0 +1,63 @@
+"""Shared test helpers: error metrics, row sampling, device transfers."""
+from __future__ import annotations
+
+import numpy as np
+
+import synth
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    return synth.bf16_to_float(np.ascontiguousarray(bits)).astype(np.float64)
+
+
+def bf16_half_ulp(ref: np.ndarray) -> np.ndarray:
+    """Half the bfloat16 spacing at |ref| (the rounding error bound of a
+    correctly rounded bf16 result)."""
+    a = np.abs(ref)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    ulp = np.exp2(e - 7)
+    return np.where(a > 0, 0.5 * ulp, 0.0)
+
+
+def attn_errors(got: np.ndarray, ref: np.ndarray) -> dict:
+    """max-abs, mean-abs, excess over bf16 output rounding, cosine."""
+    got = got.astype(np.float64).ravel()
+    ref = ref.astype(np.float64).ravel()
+    d = np.abs(got - ref)
+    excess = np.maximum(0.0, d - bf16_half_ulp(ref))
+    cos = float(np.dot(got, ref) / (np.linalg.norm(got) * np.linalg.norm(ref) + 1e-300))
+    return dict(max_abs=float(d.max()), mean_abs=float(d.mean()), max_excess=float(excess.max()),
+                cos=cos)
+
+
+# The attention gate: max-abs 3e-2 (measured as excess over the bf16 rounding
+# of the exact result), mean-abs 3e-3, cosine >= 0.999.
+ATTN_MAX_EXCESS = 3e-2
+ATTN_MEAN_ABS = 3e-3
+ATTN_COS = 0.999
+
+
+def assert_attn_close(got, ref, what=""):
+    e = attn_errors(got, ref)
+    assert e["max_excess"] <= ATTN_MAX_EXCESS, (what, e)
+    assert e["mean_abs"] <= ATTN_MEAN_ABS, (what, e)
+    assert e["cos"] >= ATTN_COS, (what, e)
+    return e
+
+
+def sample_pairs(cu: np.ndarray, heads: int, per_seg: int, seed: int):
+    """(token, head) pairs per segment: first/last rows, rows around the
+    128-row tile edges, and random rows; heads cycle so all are covered."""
+    rng = np.random.default_rng(seed)
+    toks, hs = [], []
+    for i in range(len(cu) - 1):
+        a, b = int(cu[i]), int(cu[i + 1])
+        L = b - a
+        if L <= 0:
+            continue
+        fixed = {0, L - 1, min(127, L - 1), min(128, L - 1), L // 2, max(0, L - 129)}
+        rows = sorted(fixed) + list(rng.integers(0, L, size=max(0, per_seg - len(fixed))))
+        for n, r in enumerate(rows):
+            toks.append(a + int(r))
+            hs.append(int((n + i) % heads) if n < heads else int(rng.integers(0, heads)))
+    return np.array(toks, dtype=np.int64), np.array(hs, dtype=np.int32)

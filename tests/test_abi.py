@@ -1,0 +1,151 @@
+"""CPU checks of the C-ABI library: it loads, exports every symbol the header
+declares, and its host-only entry points (status strings, descale rule,
+scale-file reader/writer, argument checks) behave as documented.  No CUDA
+compute is launched here."""
+import ctypes
+import json
+import os
+import re
+
+import numpy as np
+import pytest
+
+import fp8_quantized_vit_b200 as fv
+from fp8_quantized_vit_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8vit.h")
+GOLDEN = os.path.join(ROOT, "tests", "golden", "scale_file_example.json")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    _build.build()
+    yield
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([A-Za-z_][A-Za-z0-9_]*)\s*\(",
+                       text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "defined")))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for n in ["fp8_amax_ring_update", "fp8_quantize_qkv_per_tensor", "fp8_varlen_attn_fwd",
+              "per_token_group_quant_fp8", "fp8_static_scales_load", "fp8_static_scales_save",
+              "fp8_descale_from_amax", "fp8vit_create", "fp8vit_check"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(fv.LIB_PATH)
+    missing = [n for n in _declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    monkeypatch.setattr(fv, "_lib", None)
+    monkeypatch.setattr(fv, "LIB_PATH", os.path.join(ROOT, "does-not-exist.so"))
+    with pytest.raises(RuntimeError):
+        fv.lib()
+
+
+def test_version_and_status_strings():
+    assert fv.lib().fp8vit_version() >= 100
+    for s in range(8):
+        assert fv.status_string(s)
+    assert fv.status_string(fv.ETIMEOUT).startswith("bounded wait")
+
+
+def test_descale_from_amax():
+    assert fv.fp8_descale_from_amax(224.0) == 0.5
+    assert fv.fp8_descale_from_amax(0.0) == float(np.float32(1e-10))
+    assert fv.fp8_descale_from_amax(198.0) == float(np.float32(198.0) / np.float32(448.0))
+
+
+def test_scale_file_golden_example():
+    # vLLM "FP8 ViT Encoder Attention", Scale File Format: the printed example.
+    assert fv.fp8_static_scales_load(GOLDEN, "visual.blocks.0.attn.attn") == (224.0, 198.0, 210.0)
+    assert fv.fp8_static_scales_load(GOLDEN, "visual.blocks.1.attn.attn") == (218.0, 195.0, 207.0)
+    d = [fv.fp8_descale_from_amax(x) for x in (224.0, 198.0, 210.0)]
+    assert d[0] == 0.5
+
+
+def test_scale_file_aliases_and_errors(tmp_path):
+    p = tmp_path / "s.json"
+    p.write_text(json.dumps({"a": {"q_scale": 1.5, "k_scale": 2.0, "v_scale": 3.25},
+                             "b": {"q": 1, "k": 2, "v": 3, "extra": [1, {"x": None}]}}))
+    assert fv.fp8_static_scales_load(str(p), "a") == (1.5, 2.0, 3.25)
+    assert fv.fp8_static_scales_load(str(p), "b") == (1.0, 2.0, 3.0)
+    with pytest.raises(fv.FP8VitError) as e:
+        fv.fp8_static_scales_load(str(p), "missing")
+    assert e.value.status == fv.ENOTFOUND
+    with pytest.raises(fv.FP8VitError) as e:
+        fv.fp8_static_scales_load(str(tmp_path / "nope.json"), "a")
+    assert e.value.status == fv.EIO
+    bad = tmp_path / "bad.json"
+    for text in ['{"a": {"q": 1, "k": 2}}',                      # v missing
+                 '{"a": {"q": 1, "q_scale": 2, "k": 1, "v": 1}}',  # conflicting alias
+                 '{"a": {"q": 1, "k": 2, "v": 3}',                 # truncated
+                 '{"a": {"q": "x", "k": 2, "v": 3}}',              # not a number
+                 '{"a": {"q": 1, "k": 2, "v": 3}} trailing']:
+        bad.write_text(text)
+        with pytest.raises(fv.FP8VitError) as e:
+            fv.fp8_static_scales_load(str(bad), "a")
+        assert e.value.status == fv.EPARSE, text
+    # both spellings with the same value are accepted
+    bad.write_text('{"a": {"q": 1, "q_scale": 1.0, "k": 2, "v": 3}}')
+    assert fv.fp8_static_scales_load(str(bad), "a") == (1.0, 2.0, 3.0)
+
+
+def test_scale_file_round_trip_with_margin(tmp_path):
+    rng = np.random.default_rng(1)
+    amax = (rng.random((3, 3)) * 40).astype(np.float32)
+    layers = [f"visual.blocks.{i}.attn.attn" for i in range(3)]
+    p = str(tmp_path / "cal.json")
+    fv.fp8_static_scales_save(p, layers, amax, margin=1.5)
+    json.load(open(p))  # valid JSON
+    for i, name in enumerate(layers):
+        got = fv.fp8_static_scales_load(p, name)
+        want = tuple(float(np.float32(1.5) * a) for a in amax[i])
+        assert got == want
+
+
+def test_host_argument_checks_need_no_gpu():
+    lib = fv.lib()
+    fake_ctx = ctypes.create_string_buffer(64)
+    dummy = ctypes.c_void_p(0x10000)  # never dereferenced: the checks return first
+    # null context / pointers
+    assert lib.fp8_varlen_attn_fwd(None, dummy, dummy, dummy, dummy, dummy, dummy, dummy, 1, 8,
+                                   8, 2, 72, 0.1, dummy, 0, None, None) == fv.EINVAL
+    # head_dim outside {72, 128}
+    assert lib.fp8_varlen_attn_fwd(fake_ctx, dummy, dummy, dummy, dummy, dummy, dummy, dummy, 1,
+                                   8, 8, 2, 64, 0.1, dummy, 0, None, None) == fv.EUNSUPPORTED
+    # odd head count at head_dim 72: a token row is not a multiple of 16 bytes
+    assert lib.fp8_varlen_attn_fwd(fake_ctx, dummy, dummy, dummy, dummy, dummy, dummy, dummy, 1,
+                                   8, 8, 3, 72, 0.1, dummy, 0, None, None) == fv.EUNSUPPORTED
+    # FP8 output needs an output scale and BF16 output must not get one
+    assert lib.fp8_varlen_attn_fwd(fake_ctx, dummy, dummy, dummy, dummy, dummy, dummy, dummy, 1,
+                                   8, 8, 2, 72, 0.1, dummy, 1, None, None) == fv.EINVAL
+    assert lib.fp8_varlen_attn_fwd(fake_ctx, dummy, dummy, dummy, dummy, dummy, dummy, dummy, 1,
+                                   8, 8, 2, 72, 0.1, dummy, 0, dummy, None) == fv.EINVAL
+    # non-positive softmax scale
+    assert lib.fp8_varlen_attn_fwd(fake_ctx, dummy, dummy, dummy, dummy, dummy, dummy, dummy, 1,
+                                   8, 8, 2, 72, 0.0, dummy, 0, None, None) == fv.EINVAL
+    # misaligned q8
+    odd = ctypes.c_void_p(0x10001)
+    assert lib.fp8_varlen_attn_fwd(fake_ctx, odd, dummy, dummy, dummy, dummy, dummy, dummy, 1,
+                                   8, 8, 2, 72, 0.1, dummy, 0, None, None) == fv.EINVAL
+    # group quant: n not a multiple of group, unsupported group
+    assert lib.per_token_group_quant_fp8(fake_ctx, dummy, 4, 200, 128, dummy, dummy,
+                                         None) == fv.EINVAL
+    assert lib.per_token_group_quant_fp8(None, dummy, 4, 256, 128, dummy, dummy,
+                                         None) == fv.EINVAL
+    # quantizers: negative size, misaligned input
+    assert lib.fp8_quantize_qkv_per_tensor(fake_ctx, dummy, dummy, dummy, -1, dummy, dummy,
+                                           dummy, dummy, None) == fv.EINVAL
+    assert lib.fp8_amax_ring_update(fake_ctx, odd, dummy, dummy, 8, dummy, dummy,
+                                    None) == fv.EINVAL

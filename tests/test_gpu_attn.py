@@ -1,0 +1,212 @@
+"""GPU parity of the varlen FP8 attention kernel against the fp64 oracle.
+
+Inputs: the oracle quantizes the seeded BF16 tensors (static 1.5 margin or
+the dynamic ring), and the same e4m3 bytes and descales go to the kernel.
+Small shapes (several tiles and ragged tails, 1..3 images, odd and even
+heads, head_dim 72 and 128) compare every output; the workload shapes
+compare sampled (token, head) rows the oracle computes one by one.
+Gate: max-abs 3e-2 measured as excess over the bf16 rounding of the exact
+result, mean-abs 3e-3, cosine >= 0.999.  FP8 output: every code within one
+e4m3 step of the oracle's code."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from _helpers import (assert_attn_close, attn_errors, bf16_bits_to_f64, sample_pairs)
+
+pytestmark = pytest.mark.gpu
+
+fv = pytest.importorskip("fp8_quantized_vit_b200")
+
+
+@pytest.fixture(scope="module")
+def ctx():
+    assert torch.cuda.is_available()
+    return fv.Context()
+
+
+def _dev(a: np.ndarray, dtype=None) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    return (t.view(dtype) if dtype is not None else t).cuda()
+
+
+def _prepare(lens, H, D, seed, mode="static"):
+    """Seeded BF16 q/k/v -> oracle e4m3 codes + descales."""
+    cu = synth.cu_seqlens(lens)
+    T = int(cu[-1])
+    keys = [synth.stream_key(seed, 0, t) for t in range(3)]
+    bf = [synth.bf16_tensor(k, T, H * D) for k in keys]
+    amax = [oracle.amax_bf16(x) for x in bf]
+    if mode == "static":
+        desc = [oracle.descale_from_amax(np.float32(1.5) * np.float32(a)) for a in amax]
+    else:
+        desc = list(oracle.Ring().update(amax))
+    codes = [oracle.quantize_per_tensor(x, d).reshape(T, H, D) for x, d in zip(bf, desc)]
+    return cu, codes, desc
+
+
+def _run_gpu(ctx, cu, codes, desc, H, D, max_seqlen, output_scale=None):
+    T = codes[0].shape[0]
+    q8, k8, v8 = (_dev(c) for c in codes)
+    d = [torch.tensor([x], dtype=torch.float32, device="cuda") for x in desc]
+    cu_d = _dev(cu)
+    if output_scale is None:
+        out = torch.full((T, H, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+        fv.fp8_varlen_attn_fwd(q8, k8, v8, d[0], d[1], d[2], cu_d, max_seqlen,
+                               np.float32(1.0 / math.sqrt(D)), out, ctx=ctx)
+    else:
+        out = torch.full((T, H, D), 0x7F, dtype=torch.uint8, device="cuda")
+        os_d = torch.tensor([output_scale], dtype=torch.float32, device="cuda")
+        fv.fp8_varlen_attn_fwd(q8, k8, v8, d[0], d[1], d[2], cu_d, max_seqlen,
+                               np.float32(1.0 / math.sqrt(D)), out, output_scale=os_d, ctx=ctx)
+    st, site = ctx.check()
+    assert st == fv.OK, (fv.status_string(st), site)
+    return out
+
+
+def _gpu_bf16_to_f64(out: torch.Tensor) -> np.ndarray:
+    return bf16_bits_to_f64(out.view(torch.int16).cpu().numpy().view(np.uint16))
+
+
+SMALL = [
+    ((1,), 2, 72), ((2,), 2, 128), ((127,), 2, 72), ((128,), 2, 128), ((129,), 4, 72),
+    ((300, 1, 77), 2, 72), ((256, 129), 2, 128), ((5, 0, 200), 2, 72), ((513,), 2, 128),
+]
+
+
+@pytest.mark.parametrize("lens,H,D", SMALL)
+def test_small_shapes_full_oracle(ctx, lens, H, D):
+    cu, codes, desc = _prepare(lens, H, D, seed=sum(lens) + D)
+    sm = np.float32(1.0 / math.sqrt(D))
+    ref = oracle.attn_full(*codes, *desc, cu, H, D, sm)
+    out = _run_gpu(ctx, cu, codes, desc, H, D, max(lens))
+    got = _gpu_bf16_to_f64(out)
+    assert not np.isnan(got).any()
+    assert_attn_close(got, ref, (lens, H, D))
+
+
+def test_c1_full_oracle(ctx):
+    """1024 tokens, 16 heads, head_dim 72, static scales: every output."""
+    w = synth.WORKLOADS["c1"]
+    q, k, v = w.qkv(0)
+    amax = [oracle.amax_bf16(x) for x in (q, k, v)]
+    desc = [oracle.descale_from_amax(np.float32(1.5) * np.float32(a)) for a in amax]
+    codes = [oracle.quantize_per_tensor(x, d).reshape(w.tokens, w.heads, w.head_dim)
+             for x, d in zip((q, k, v), desc)]
+    cu = synth.cu_seqlens(w.seg_lens)
+    ref = oracle.attn_full(*codes, *desc, cu, w.heads, w.head_dim, w.softmax_scale)
+    out = _run_gpu(ctx, cu, codes, desc, w.heads, w.head_dim, max(w.seg_lens))
+    e = assert_attn_close(_gpu_bf16_to_f64(out), ref, "c1")
+    print("c1 errors", e)
+
+
+@pytest.mark.parametrize("name", ["c2", "c3_2304", "c3_16384", "c4", "c5"])
+def test_workload_sampled_rows(ctx, name):
+    w = synth.WORKLOADS[name]
+    q, k, v = w.qkv(0)
+    amax = [oracle.amax_bf16(x) for x in (q, k, v)]
+    if w.mode == "static":
+        desc = [oracle.descale_from_amax(np.float32(1.5) * np.float32(a)) for a in amax]
+    else:
+        desc = list(oracle.Ring().update(amax))
+    codes = [oracle.quantize_per_tensor(x, d).reshape(w.tokens, w.heads, w.head_dim)
+             for x, d in zip((q, k, v), desc)]
+    cu = synth.cu_seqlens(w.seg_lens)
+    toks, hs = sample_pairs(cu, w.heads, per_seg=24, seed=len(name))
+    ref = oracle.attn_pairs(*codes, *desc, cu, w.heads, w.head_dim, w.softmax_scale, toks, hs)
+    out = _run_gpu(ctx, cu, codes, desc, w.heads, w.head_dim, max(w.seg_lens))
+    got = _gpu_bf16_to_f64(out)[toks, hs]
+    e = assert_attn_close(got, ref, name)
+    print(name, "errors", e)
+    # every row was written (no NaN left from the fill)
+    assert not torch.isnan(out.float()).any().item()
+
+
+def _code_step_distance(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """Distance in e4m3 grid steps between codes (sign-magnitude order)."""
+    def ordinal(c):
+        c = c.astype(np.int32)
+        mag = c & 0x7F
+        return np.where(c & 0x80, -mag, mag)
+    return np.abs(ordinal(a) - ordinal(b))
+
+
+def test_fp8_output_small_full(ctx):
+    lens, H, D = (200, 77), 2, 72
+    cu, codes, desc = _prepare(lens, H, D, seed=44)
+    sm = np.float32(1.0 / math.sqrt(D))
+    ref = oracle.attn_full(*codes, *desc, cu, H, D, sm)
+    out_scale = float(np.float32(np.abs(ref).max()) / np.float32(448.0))
+    want = oracle.fp8_output(ref, out_scale)
+    got = _run_gpu(ctx, cu, codes, desc, H, D, max(lens), output_scale=out_scale)
+    dist = _code_step_distance(got.cpu().numpy(), want)
+    assert dist.max() <= 1, dist.max()
+    deq = oracle.e4m3_decode(got.cpu().numpy()) * out_scale
+    cos = float(np.dot(deq.ravel(), ref.ravel()) / (np.linalg.norm(deq) * np.linalg.norm(ref)))
+    assert cos >= 0.999
+
+
+def test_fp8_output_c4_sampled(ctx):
+    """3 x 14400 tokens, static scales, fused FP8 output.  output_scale is
+    the amax of the oracle's sampled rows / 448 (the full amax needs the full
+    fp64 attention); larger values saturate on both sides alike."""
+    w = synth.WORKLOADS["c4"]
+    q, k, v = w.qkv(0)
+    amax = [oracle.amax_bf16(x) for x in (q, k, v)]
+    desc = [oracle.descale_from_amax(np.float32(1.5) * np.float32(a)) for a in amax]
+    codes = [oracle.quantize_per_tensor(x, d).reshape(w.tokens, w.heads, w.head_dim)
+             for x, d in zip((q, k, v), desc)]
+    cu = synth.cu_seqlens(w.seg_lens)
+    toks, hs = sample_pairs(cu, w.heads, per_seg=24, seed=4)
+    ref = oracle.attn_pairs(*codes, *desc, cu, w.heads, w.head_dim, w.softmax_scale, toks, hs)
+    out_scale = float(np.float32(np.abs(ref).max()) / np.float32(448.0))
+    want = oracle.fp8_output(ref, out_scale)
+    got = _run_gpu(ctx, cu, codes, desc, w.heads, w.head_dim, max(w.seg_lens),
+                   output_scale=out_scale)
+    g = got.cpu().numpy()[toks, hs]
+    assert _code_step_distance(g, want).max() <= 1
+
+
+def test_bad_cu_seqlens_reports_einval(ctx):
+    H, D = 2, 72
+    cu, codes, desc = _prepare((64, 64), H, D, seed=3)
+    bad = np.array([0, 100, 60], dtype=np.int32)  # non-monotone
+    q8, k8, v8 = (_dev(c) for c in codes)
+    d = torch.ones(1, dtype=torch.float32, device="cuda")
+    out = torch.zeros((128, H, D), dtype=torch.bfloat16, device="cuda")
+    fv.fp8_varlen_attn_fwd(q8, k8, v8, d, d, d, _dev(bad), 128, 0.1, out, ctx=ctx)
+    st, site = ctx.check()
+    assert st == fv.EINVAL and site == 100
+    # a segment longer than max_seqlen is rejected too
+    fv.fp8_varlen_attn_fwd(q8, k8, v8, d, d, d, _dev(cu), 32, 0.1, out, ctx=ctx)
+    st, site = ctx.check()
+    assert st == fv.EINVAL
+    # and the context is still usable
+    out2 = _run_gpu(ctx, cu, codes, desc, H, D, 64)
+    assert not torch.isnan(out2.float()).any().item()
+
+
+def test_end_to_end_dynamic_pipeline(ctx):
+    """amax ring -> quantize -> attention on the device, 3 forwards, against
+    the oracle's ring + quantizer + attention on the same BF16 inputs."""
+    lens, H, D = (333, 190), 4, 72
+    cu = synth.cu_seqlens(lens)
+    T = int(cu[-1])
+    layer = fv.FP8EncoderAttention(H, D, ctx=ctx)
+    ring_o = oracle.Ring()
+    for f in range(3):
+        bf = [synth.bf16_tensor(synth.stream_key(77, f, t), T, H * D) for t in range(3)]
+        desc = ring_o.update([oracle.amax_bf16(x) for x in bf])
+        codes = [oracle.quantize_per_tensor(x, d).reshape(T, H, D) for x, d in zip(bf, desc)]
+        ref = oracle.attn_full(*codes, *desc, cu, H, D, np.float32(1.0 / math.sqrt(D)))
+        dev = [_dev(x.view(np.int16), None).view(torch.bfloat16).reshape(T, H, D) for x in bf]
+        out = layer(*dev, _dev(cu), max(lens))
+        st, site = ctx.check()
+        assert st == fv.OK
+        assert (layer.descale.cpu().numpy().view(np.uint32) ==
+                np.asarray(desc, np.float32).view(np.uint32)).all()
+        assert_attn_close(_gpu_bf16_to_f64(out), ref, f"forward {f}")

@@ -1,0 +1,157 @@
+"""GPU parity of the HBM-bound kernels against the oracle, bit for bit:
+amax + 16-slot ring descales, per-tensor e4m3 quantization, and the
+per-token-group quantizer, on the workloads' shapes and edge cases."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+fv = pytest.importorskip("fp8_quantized_vit_b200")
+
+
+def _dev_bf16(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _host_u8(t: torch.Tensor) -> np.ndarray:
+    return t.view(torch.uint8).cpu().numpy()
+
+
+def _f32_bits(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float32).view(np.uint32)
+
+
+@pytest.fixture(scope="module")
+def ctx():
+    assert torch.cuda.is_available()
+    return fv.Context()
+
+
+def _check_ok(ctx):
+    st, site = ctx.check()
+    assert st == fv.OK, (fv.status_string(st), site)
+
+
+def test_ring_descales_bit_exact_over_20_forwards(ctx):
+    """Dynamic scaling over the 20 forwards of the 8192-token, head_dim-128
+    workload: the ring wraps after 16; every forward's descales and the ring
+    contents must equal the oracle's bit for bit."""
+    w = synth.WORKLOADS["c2"]
+    ring_d = fv.new_ring()
+    desc_d = torch.zeros(3, dtype=torch.float32, device="cuda")
+    ring_o = oracle.Ring()
+    for f in range(20):
+        q, k, v = w.qkv(f)
+        amax = [oracle.amax_bf16(x) for x in (q, k, v)]
+        want = ring_o.update(amax)
+        fv.fp8_amax_ring_update(_dev_bf16(q), _dev_bf16(k), _dev_bf16(v), ring_d, desc_d, ctx=ctx)
+        got = desc_d.cpu().numpy()
+        assert (_f32_bits(got) == _f32_bits(want)).all(), (f, got, want)
+        r = ring_d.cpu().numpy()
+        assert (_f32_bits(r[:48].reshape(3, 16)) == _f32_bits(ring_o.hist)).all(), f
+        assert r[48:49].view(np.int32)[0] == ring_o.pos[0]
+    _check_ok(ctx)
+
+
+@pytest.mark.parametrize("n", [0, 1, 7, 8, 9, 8 * 1000 + 5, 1 << 20])
+def test_amax_ring_ragged_sizes(ctx, n):
+    rng = np.random.default_rng(n)
+    bits = [np.ascontiguousarray(synth.bf16_tensor(synth.stream_key(n, 0, t), 1, max(n, 1))[0, :n])
+            for t in range(3)]
+    # put the largest magnitude at the very end so the tail path matters
+    if n:
+        for t in range(3):
+            bits[t][-1] = np.uint16(0xC2F0 + t)  # about -120 with a sign bit
+    ring_d = fv.new_ring()
+    desc_d = torch.zeros(3, dtype=torch.float32, device="cuda")
+    dev = [_dev_bf16(b) if n else torch.empty(8, dtype=torch.bfloat16, device="cuda") for b in bits]
+    fv.lib().fp8_amax_ring_update(ctx.handle, dev[0].data_ptr(), dev[1].data_ptr(),
+                                  dev[2].data_ptr(), n, ring_d.data_ptr(), desc_d.data_ptr(),
+                                  fv._stream())
+    ring_o = oracle.Ring()
+    want = ring_o.update([oracle.amax_bf16(b) for b in bits])
+    assert (_f32_bits(desc_d.cpu().numpy()) == _f32_bits(want)).all()
+    _check_ok(ctx)
+
+
+def test_ring_read_amax(ctx):
+    ring_d = fv.new_ring()
+    desc_d = torch.zeros(3, dtype=torch.float32, device="cuda")
+    seq = [(1.0, 2.0, 3.0), (5.0, 0.5, 0.25), (2.0, 2.0, 2.0)]
+    for a in seq:
+        x = [torch.full((64,), v, dtype=torch.bfloat16, device="cuda") for v in a]
+        fv.fp8_amax_ring_update(*x, ring_d, desc_d, ctx=ctx)
+    assert fv.fp8_ring_read_amax(ring_d) == [5.0, 2.0, 3.0]
+
+
+def _quant_case(ctx, q, k, v, desc):
+    n = q.size
+    dq, dk, dv = (_dev_bf16(x) for x in (q, k, v))
+    d = torch.tensor(desc, dtype=torch.float32, device="cuda")
+    outs = [torch.empty(max(n, 8), dtype=torch.uint8, device="cuda") for _ in range(3)]
+    fv.lib().fp8_quantize_qkv_per_tensor(ctx.handle, dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                         n, d.data_ptr(), outs[0].data_ptr(),
+                                         outs[1].data_ptr(), outs[2].data_ptr(), fv._stream())
+    _check_ok(ctx)
+    for x, o, s in zip((q, k, v), outs, desc):
+        want = oracle.quantize_per_tensor(x.ravel(), s)
+        got = _host_u8(o)[:n]
+        assert (got == want).all(), (np.nonzero(got != want)[0][:5])
+
+
+@pytest.mark.parametrize("name", ["c1", "c2", "c4", "c5"])
+def test_quantize_per_tensor_bit_exact(ctx, name):
+    """Static (margin 1.5) and dynamic descales on every workload's tensors."""
+    w = synth.WORKLOADS[name]
+    q, k, v = w.qkv(0)
+    amax = [oracle.amax_bf16(x) for x in (q, k, v)]
+    static = [oracle.descale_from_amax(np.float32(1.5) * np.float32(a)) for a in amax]
+    _quant_case(ctx, q, k, v, static)
+    if name in ("c1", "c2"):
+        tight = [oracle.descale_from_amax(a) for a in amax]  # amax maps onto exactly 448
+        _quant_case(ctx, q, k, v, tight)
+
+
+@pytest.mark.parametrize("n", [1, 7, 8, 9, 4097])
+def test_quantize_ragged_and_special_values(ctx, n):
+    rng = np.random.default_rng(n)
+    base = synth.bf16_tensor(synth.stream_key(5, n, 0), 1, max(n, 1))[0, :n].copy()
+    specials = np.array([0x0000, 0x8000, 0x0001, 0x8001, 0x7F7F, 0xFF7F, 0x3F80, 0xBF80],
+                        dtype=np.uint16)  # +-0, +-tiny, +-max finite, +-1
+    base[: min(n, 8)] = specials[: min(n, 8)]
+    for desc in (1.0, 1e-10, 0.013671875, 3.0e-3):
+        _quant_case(ctx, base, base[::-1].copy(), base, [desc, desc, desc])
+
+
+@pytest.mark.parametrize("m,n", [(1, 2048), (37504, 2048), (726, 7168), (4192, 7168),
+                                 (8192, 2048), (97200, 1152), (3, 128)])
+def test_group_quant_bit_exact(ctx, m, n):
+    """Shapes of the group quantizer page's table, and the attention outputs
+    of the 8192-token and 3x32400-token workloads."""
+    x = synth.bf16_tensor(synth.stream_key(m, n, 7), m, n)
+    want_q, want_s = oracle.group_quant(x, 128)
+    xd = _dev_bf16(x)
+    xq = torch.empty((m, n), dtype=torch.uint8, device="cuda")
+    sc = torch.empty((m, n // 128), dtype=torch.float32, device="cuda")
+    fv.per_token_group_quant_fp8(xd, 128, xq, sc, ctx=ctx)
+    _check_ok(ctx)
+    assert (_host_u8(xq) == want_q).all()
+    assert (_f32_bits(sc.cpu().numpy()) == _f32_bits(want_s)).all()
+
+
+@pytest.mark.parametrize("group", [16, 32, 64, 256])
+def test_group_quant_other_group_sizes(ctx, group):
+    m, n = 129, 1024
+    x = synth.bf16_tensor(synth.stream_key(group, 1, 2), m, n)
+    x[0, :group] = 0  # an all-zero group takes the 1e-10 floor
+    want_q, want_s = oracle.group_quant(x, group)
+    xq = torch.empty((m, n), dtype=torch.uint8, device="cuda")
+    sc = torch.empty((m, n // group), dtype=torch.float32, device="cuda")
+    fv.per_token_group_quant_fp8(_dev_bf16(x), group, xq, sc, ctx=ctx)
+    _check_ok(ctx)
+    assert (_host_u8(xq) == want_q).all()
+    assert (_f32_bits(sc.cpu().numpy()) == _f32_bits(want_s)).all()
