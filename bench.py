@@ -197,11 +197,13 @@ def run_reference(args):
     return 0
 
 
-def _config(w):
+def _config(w, n_fwd=None):
+    n_fwd = len(w.seeds) if n_fwd is None else n_fwd
+    gb = n_fwd * 3 * w.tokens * w.hd * 2 / 1e9
     return {"workload": w.name, "seq_lens": list(w.seg_lens), "heads": w.heads,
-            "head_dim": w.head_dim, "forwards": len(w.seeds),
+            "head_dim": w.head_dim, "forwards": n_fwd,
             "step": "amax ring + quantize q/k/v + attention (bf16 out) + group quant (128)",
-            "l2": "inputs rotate over 20 forwards (2.0 GB > 126 MB L2)",
+            "l2": f"inputs rotate over {n_fwd} forwards ({gb:.2f} GB; L2 is 126 MB)",
             "parallelism": "replicas"}
 
 
@@ -219,7 +221,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     w = synth.WORKLOADS[args.workload]
     T, H, D = w.tokens, w.heads, w.head_dim
-    n_fwd = len(w.seeds)
+    n_fwd = len(w.seeds) if args.forwards <= 0 else min(args.forwards, len(w.seeds))
     ctx = fv.Context(local)
     dev = torch.device("cuda", local)
 
@@ -336,7 +338,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3 (fp32 accumulate)",
-        "data": "synthetic", "config": _config(w),
+        "data": "synthetic", "config": _config(w, n_fwd),
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>",
                      "achieved": attn_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
                      "frac": attn_tflops / fp8_peak, "traffic": traffic,
@@ -371,6 +373,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--forwards", type=int, default=0,
+                    help="distinct input sets kept resident (0 = all of the workload's)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=1.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -61,3 +61,40 @@ def sample_pairs(cu: np.ndarray, heads: int, per_seg: int, seed: int):
             toks.append(a + int(r))
             hs.append(int((n + i) % heads) if n < heads else int(rng.integers(0, heads)))
     return np.array(toks, dtype=np.int64), np.array(hs, dtype=np.int32)
+
+
+def e4m3_half_step(y: np.ndarray) -> np.ndarray:
+    """Half the e4m3 grid spacing at |y| (y already divided by the scale)."""
+    a = np.minimum(np.abs(y), 448.0)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    step = np.where(a >= 2.0 ** -6, np.exp2(e - 3), 2.0 ** -9)
+    return 0.5 * step
+
+
+def fp8_output_errors(got_codes: np.ndarray, ref: np.ndarray, scale: float, decode) -> dict:
+    """FP8-output errors in value space: |deq(got) - o| beyond half an e4m3
+    step at o (the output format's own rounding; saturation at +-448*scale
+    counts as exact), the e4m3 grid distance to the oracle's codes, cosine."""
+    deq = decode(got_codes).astype(np.float64).ravel() * scale
+    o = ref.astype(np.float64).ravel()
+    oc = np.clip(o, -448.0 * scale, 448.0 * scale)
+    excess = np.maximum(0.0, np.abs(deq - oc) - e4m3_half_step(o / scale) * scale)
+    cos = float(np.dot(deq, o) / (np.linalg.norm(deq) * np.linalg.norm(o) + 1e-300))
+    return dict(max_excess=float(excess.max()), mean_excess=float(excess.mean()), cos=cos)
+
+
+def code_step_distance(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """Distance in e4m3 grid steps between codes (sign-magnitude order)."""
+    def ordinal(c):
+        c = c.astype(np.int32)
+        mag = c & 0x7F
+        return np.where(c & 0x80, -mag, mag)
+    return np.abs(ordinal(a) - ordinal(b))
+
+
+def assert_fp8_out_close(got_codes, ref, scale, decode, what=""):
+    e = fp8_output_errors(got_codes, ref, scale, decode)
+    assert e["max_excess"] <= ATTN_MAX_EXCESS, (what, e)
+    assert e["mean_excess"] <= ATTN_MEAN_ABS, (what, e)
+    assert e["cos"] >= ATTN_COS, (what, e)
+    return e

@@ -6,8 +6,10 @@ Small shapes (several tiles and ragged tails, 1..3 images, odd and even
 heads, head_dim 72 and 128) compare every output; the workload shapes
 compare sampled (token, head) rows the oracle computes one by one.
 Gate: max-abs 3e-2 measured as excess over the bf16 rounding of the exact
-result, mean-abs 3e-3, cosine >= 0.999.  FP8 output: every code within one
-e4m3 step of the oracle's code."""
+result, mean-abs 3e-3, cosine >= 0.999.  FP8 output: the same gate on the
+dequantised values, with the excess taken over half an e4m3 step (the output
+format's own rounding), and codes within one e4m3 step of the oracle's wherever
+|o| >= amax/16 (nearer zero the grid is finer than the kernel's absolute error)."""
 import math
 
 import numpy as np
@@ -16,7 +18,8 @@ import torch
 
 import oracle
 import synth
-from _helpers import (assert_attn_close, attn_errors, bf16_bits_to_f64, sample_pairs)
+from _helpers import (assert_attn_close, assert_fp8_out_close, bf16_bits_to_f64,
+                      code_step_distance, sample_pairs)
 
 pytestmark = pytest.mark.gpu
 
@@ -126,15 +129,6 @@ def test_workload_sampled_rows(ctx, name):
     assert not torch.isnan(out.float()).any().item()
 
 
-def _code_step_distance(a: np.ndarray, b: np.ndarray) -> np.ndarray:
-    """Distance in e4m3 grid steps between codes (sign-magnitude order)."""
-    def ordinal(c):
-        c = c.astype(np.int32)
-        mag = c & 0x7F
-        return np.where(c & 0x80, -mag, mag)
-    return np.abs(ordinal(a) - ordinal(b))
-
-
 def test_fp8_output_small_full(ctx):
     lens, H, D = (200, 77), 2, 72
     cu, codes, desc = _prepare(lens, H, D, seed=44)
@@ -142,12 +136,13 @@ def test_fp8_output_small_full(ctx):
     ref = oracle.attn_full(*codes, *desc, cu, H, D, sm)
     out_scale = float(np.float32(np.abs(ref).max()) / np.float32(448.0))
     want = oracle.fp8_output(ref, out_scale)
-    got = _run_gpu(ctx, cu, codes, desc, H, D, max(lens), output_scale=out_scale)
-    dist = _code_step_distance(got.cpu().numpy(), want)
-    assert dist.max() <= 1, dist.max()
-    deq = oracle.e4m3_decode(got.cpu().numpy()) * out_scale
-    cos = float(np.dot(deq.ravel(), ref.ravel()) / (np.linalg.norm(deq) * np.linalg.norm(ref)))
-    assert cos >= 0.999
+    got = _run_gpu(ctx, cu, codes, desc, H, D, max(lens), output_scale=out_scale).cpu().numpy()
+    e = assert_fp8_out_close(got, ref, out_scale, oracle.e4m3_decode, "fp8 out")
+    dist = code_step_distance(got, want)
+    print("fp8 out", e, "codes within one step:", float((dist <= 1).mean()))
+    # away from zero (|o| >= 1/16 of the amax) the codes agree to one step
+    big = np.abs(ref) >= np.abs(ref).max() / 16
+    assert dist[big].max() <= 1
 
 
 def test_fp8_output_c4_sampled(ctx):
@@ -168,7 +163,9 @@ def test_fp8_output_c4_sampled(ctx):
     got = _run_gpu(ctx, cu, codes, desc, w.heads, w.head_dim, max(w.seg_lens),
                    output_scale=out_scale)
     g = got.cpu().numpy()[toks, hs]
-    assert _code_step_distance(g, want).max() <= 1
+    assert_fp8_out_close(g, ref, out_scale, oracle.e4m3_decode, "c4 fp8 out")
+    big = np.abs(ref) >= np.abs(ref).max() / 16
+    assert code_step_distance(g, want)[big].max() <= 1
 
 
 def test_bad_cu_seqlens_reports_einval(ctx):
