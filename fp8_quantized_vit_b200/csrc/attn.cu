@@ -34,6 +34,10 @@ constexpr uint32_t kTmemO = 128;  // O accumulator columns [128, 128 + NPV)
 constexpr int kBox = 32;          // bytes per TMA box row (one SW32 atom row)
 constexpr int kTileBytes = kBox * 128;  // one [128 rows x 32 B] box
 constexpr uint64_t kTimeoutNs = 2000000000ull;
+// P is stored as 2^(x - m_ref + kPLog2); a tile max up to kSlackLog2 above the
+// reference max keeps P <= 2^(6 + 2.75) = 430 < 448 (e4m3 max).
+constexpr float kPLog2 = 6.0f;
+constexpr float kSlackLog2 = 2.75f;
 
 template <int D>
 struct Cfg;
@@ -106,18 +110,96 @@ __device__ __forceinline__ void tmem_ld8_sync(uint32_t taddr, uint32_t (&r)[8]) 
         : "memory");
 }
 
-// Quantize 4 probabilities (scaled to (0, 256]) into one hi word and one lo
-// word: hi = e4m3(p), lo = e4m3(p - hi); hi + lo carries ~8 mantissa bits.
+// ---- packed arithmetic used by the softmax --------------------------------
+
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+// f32 pair -> f16x2 (lo in bits 0..15)
+__device__ __forceinline__ uint32_t cvt_f16x2(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+// f16x2 -> two e4m3 codes (RNE, satfinite; bits 0..15 -> byte 0)
+__device__ __forceinline__ uint32_t e4m3x2_of_f16x2(uint32_t h) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(d) : "r"(h));
+    return d;
+}
+__device__ __forceinline__ uint32_t f16x2_of_e4m3x2(uint32_t e) {
+    uint32_t d;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"((uint16_t)e));
+    return d;
+}
+__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// 2^x on the FMA pipe for a pair of arguments (x >= -126 after the clamp).
+// Cody-Waite reduction x = n + f, n = rint(x) via the 1.5 * 2^23 magic add,
+// f in [-0.5, 0.5]; 2^f by a degree-3 polynomial fitted for minimal relative
+// error on [-0.5, 0.5] (fit_exp2.py: max relative error 7.5e-5); 2^n is
+// added into the exponent field with an integer add.  Used for a fixed share
+// of the elements so that the MUFU pipe (ex2.approx) is not the only source
+// of exponentials.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    x0 = fmaxf(x0, -126.0f);
+    x1 = fmaxf(x1, -126.0f);
+    const uint64_t t = fadd2(f2pack(x0, x1), f2pack(kMagic, kMagic));
+    float t0, t1;
+    f2unpack(t, t0, t1);
+    float n0, n1;
+    f2unpack(fadd2(t, f2pack(-kMagic, -kMagic)), n0, n1);
+    const uint64_t f = fadd2(f2pack(x0, x1), f2pack(-n0, -n1));
+    uint64_t p = ffma2(f, f2pack(0.0551716685295105f, 0.0551716685295105f),
+                       f2pack(0.2426111251115799f, 0.2426111251115799f));
+    p = ffma2(f, p, f2pack(0.6932609677314758f, 0.6932609677314758f));
+    p = ffma2(f, p, f2pack(0.9999280571937561f, 0.9999280571937561f));
+    float p0, p1;
+    f2unpack(p, p0, p1);
+    // the low bits of t hold n (two's complement); shift them into the exponent
+    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+// Split 4 probabilities into one hi word and one lo word of e4m3 codes:
+// hi = e4m3(p), lo = e4m3(p - hi), with p first rounded to f16 (11 bits) and
+// the residual formed exactly in f16.  hi + lo carries ~8 significant bits,
+// so the PV product on FP8 tensor cores loses no more than a BF16-width P.
 __device__ __forceinline__ void p_split4(float p0, float p1, float p2, float p3, uint32_t& hi,
                                          uint32_t& lo) {
-    const uint16_t h01 = f32x2_to_e4m3x2(p0, p1);
-    const uint16_t h23 = f32x2_to_e4m3x2(p2, p3);
-    const float2 b01 = e4m3x2_to_f32x2(h01);
-    const float2 b23 = e4m3x2_to_f32x2(h23);
-    const uint16_t l01 = f32x2_to_e4m3x2(p0 - b01.x, p1 - b01.y);
-    const uint16_t l23 = f32x2_to_e4m3x2(p2 - b23.x, p3 - b23.y);
-    hi = (uint32_t)h01 | ((uint32_t)h23 << 16);
-    lo = (uint32_t)l01 | ((uint32_t)l23 << 16);
+    const uint32_t h01 = cvt_f16x2(p0, p1);
+    const uint32_t h23 = cvt_f16x2(p2, p3);
+    const uint32_t e01 = e4m3x2_of_f16x2(h01);
+    const uint32_t e23 = e4m3x2_of_f16x2(h23);
+    const uint32_t l01 = e4m3x2_of_f16x2(hsub2(h01, f16x2_of_e4m3x2(e01)));
+    const uint32_t l23 = e4m3x2_of_f16x2(hsub2(h23, f16x2_of_e4m3x2(e23)));
+    hi = e01 | (e23 << 16);
+    lo = l01 | (l23 << 16);
 }
 
 template <int D>
@@ -308,63 +390,109 @@ __global__ void __launch_bounds__(kThreads, 2)
         fence_proxy_async_smem();
         mbar_arrive(b_q_ready);
 
-        float m_run = -INFINITY, l_run = 0.0f;
+        // Running state per row, in log2 units of the scaled score
+        // (x = s * scale_log2): m_ref is the reference max the exponentials
+        // are taken against, l_run the sum of the probabilities written to P.
+        // P = 2^(x - m_ref + kPLog2): values up to 2^(kPLog2 + kSlackLog2)
+        // stay inside e4m3 (max 448), so O and l are rescaled only when a
+        // tile's max exceeds m_ref by more than kSlackLog2 (both are scaled
+        // by the same factor, so the final o = O / l is unchanged).
+        float m_ref = -INFINITY, l_run = 0.0f;
         for (int j = 0; ok && j < n_kv; ++j) {
             ok = mbar_wait_bounded(b_s_full, j & 1, abort_flag, scr, SITE_ATTN_WAIT_S, kTimeoutNs);
             ok = __all_sync(0xFFFFFFFFu, ok);
             if (!ok) break;
             tc_fence_after();
             const int nvalid = min(kBN, seg_len - j * kBN);
+            const bool full = nvalid == kBN;
             // pass 1: row max over the valid keys
             float mx = -INFINITY;
+            if (full) {
+                float m2 = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < kBN / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32_sync(tS + 32 * c, r);
+                for (int c = 0; c < kBN / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32_sync(tS + 32 * c, r);
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (32 * c + i < nvalid) mx = fmaxf(mx, __uint_as_float(r[i]));
-            }
-            const float m_new = fmaxf(m_run, mx);
-            const bool need = (j > 0) && (m_new > m_run);
-            if (__any_sync(0xFFFFFFFFu, need)) {
-                ok = mbar_wait_bounded(b_o_ready, (j - 1) & 1, abort_flag, scr, SITE_ATTN_WAIT_O,
-                                       kTimeoutNs);
-                ok = __all_sync(0xFFFFFFFFu, ok);
-                if (!ok) break;
-                tc_fence_after();
-                const float alpha = need ? ex2_approx((m_run - m_new) * scale_log2) : 1.0f;
-#pragma unroll
-                for (int c = 0; c < C::NPV / 8; ++c) {
-                    uint32_t r[8];
-                    tmem_ld8_sync(tO + 8 * c, r);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                    tmem_st8(tO + 8 * c, r);
+                    for (int i = 0; i < 32; i += 4) {
+                        mx = fmax3(mx, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+                        m2 = fmax3(m2, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+                    }
                 }
-                tmem_wait_st();
-                l_run *= alpha;
+                mx = fmaxf(mx, m2);
+            } else {
+#pragma unroll
+                for (int c = 0; c < kBN / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32_sync(tS + 32 * c, r);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (32 * c + i < nvalid) mx = fmaxf(mx, __uint_as_float(r[i]));
+                }
             }
-            m_run = m_new;
-            // p = 2^(s*scale_log2 - m*scale_log2 + 8): probabilities scaled to (0, 256]
-            const float bias = m_new * scale_log2 - 8.0f;
+            const float mxc = mx * scale_log2;
+            if (j == 0) {
+                m_ref = mxc;  // the first PV initialises O, nothing to rescale
+            } else {
+                const bool need = mxc > m_ref + kSlackLog2;
+                if (__any_sync(0xFFFFFFFFu, need)) {
+                    ok = mbar_wait_bounded(b_o_ready, (j - 1) & 1, abort_flag, scr,
+                                           SITE_ATTN_WAIT_O, kTimeoutNs);
+                    ok = __all_sync(0xFFFFFFFFu, ok);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const float alpha = need ? ex2_approx(m_ref - mxc) : 1.0f;
+#pragma unroll
+                    for (int c = 0; c < C::NPV / 8; ++c) {
+                        uint32_t r[8];
+                        tmem_ld8_sync(tO + 8 * c, r);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                        tmem_st8(tO + 8 * c, r);
+                    }
+                    tmem_wait_st();
+                    l_run *= alpha;
+                    if (need) m_ref = mxc;
+                }
+            }
+            // pass 2: P = 2^(x - bias), bias = m_ref - kPLog2
+            const float bias = m_ref - kPLog2;
+            const uint64_t c2 = f2pack(scale_log2, scale_log2);
+            const uint64_t nb2 = f2pack(-bias, -bias);
+            uint64_t lacc0 = f2pack(0.0f, 0.0f), lacc1 = lacc0;
 #pragma unroll
             for (int c = 0; c < kBN / 32; ++c) {
                 uint32_t r[32];
                 tmem_ld32_sync(tS + 32 * c, r);
                 float p[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    p[i] = (32 * c + i < nvalid)
-                               ? ex2_approx(fmaf(__uint_as_float(r[i]), scale_log2, -bias))
-                               : 0.0f;
-                    l_run += p[i];
+                for (int i = 0; i < 32; i += 2) {
+                    float x0, x1;
+                    f2unpack(ffma2(f2pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), c2,
+                                   nb2),
+                             x0, x1);
+                    if (!full) {
+                        x0 = (32 * c + i < nvalid) ? x0 : -INFINITY;
+                        x1 = (32 * c + i + 1 < nvalid) ? x1 : -INFINITY;
+                    }
+                    p[i] = ex2_approx(x0);
+                    p[i + 1] = ex2_approx(x1);
+                    if (i & 2)
+                        lacc1 = fadd2(lacc1, f2pack(p[i], p[i + 1]));
+                    else
+                        lacc0 = fadd2(lacc0, f2pack(p[i], p[i + 1]));
                 }
                 uint32_t pk[16];
 #pragma unroll
                 for (int w = 0; w < 8; ++w)
                     p_split4(p[4 * w], p[4 * w + 1], p[4 * w + 2], p[4 * w + 3], pk[w], pk[8 + w]);
                 tmem_st16(tS + 16 * c, pk);
+            }
+            {
+                float a0, a1;
+                f2unpack(fadd2(lacc0, lacc1), a0, a1);
+                l_run += a0 + a1;
             }
             tmem_wait_st();
             tc_fence_before();

@@ -9,7 +9,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/fp8vit.h"
+#include "fp8vit.h"
 
 // Device scratch owned by a context (one cudaMalloc in fp8vit_create).
 struct fp8vit_scratch {

@@ -15,7 +15,7 @@
 #include <cstring>
 #include <string>
 
-#include "../../include/fp8vit.h"
+#include "fp8vit.h"
 
 namespace {
 
