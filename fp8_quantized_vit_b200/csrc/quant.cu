@@ -8,6 +8,8 @@
 // All three stream 16-byte vectors with grid-stride loops sized to the SM
 // count, and round with the hardware RNE-satfinite e4m3 conversion after an
 // IEEE fp32 division (x / scale, as the pages' definitions divide).
+#include <mutex>
+
 #include "fp8vit_internal.cuh"
 
 namespace {
@@ -264,3 +266,91 @@ fp8vit_status per_token_group_quant_fp8(fp8vit_ctx* ctx, const uint16_t* d_x, in
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of fp8_amax_ring_update.
+//
+// Some callers cannot allocate device memory at the point where they run the
+// path: a serving process that has already handed (nearly) all free HBM to
+// its own pool, code that must not pay cudaMalloc's implicit device-wide
+// synchronisation, or a plug-in that has no place to keep a library context
+// (fp8vit_create allocates).  For them this entry point takes its scratch
+// from a fixed array compiled into the library's device image instead.
+//
+// Scratch: sizeof(fp8vit_scratch) = 128 bytes (three running |x| maxima, an
+// arrival counter, status words), taken from a 256-byte array.  The amount
+// does not grow with n_elems, so any size the context entry point accepts is
+// accepted here; a scratch need above the array's capacity is rejected with
+// FP8VIT_EUNSUPPORTED.  Every GPU that loads the library holds the array
+// until the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 256;
+constexpr int kNoAllocMaxDevices = 64;
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_amax_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+struct NoAllocSetup {
+    std::mutex mu;
+    void* addr[kNoAllocMaxDevices] = {};
+    int num_sms[kNoAllocMaxDevices] = {};
+};
+
+NoAllocSetup& noalloc_setup() {
+    static NoAllocSetup s;
+    return s;
+}
+
+// Device address of the array on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+fp8vit_status noalloc_scratch(void** addr, int* num_sms) {
+    int dev = -1;
+    FP8VIT_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return FP8VIT_EUNSUPPORTED;
+    NoAllocSetup& s = noalloc_setup();
+    std::lock_guard<std::mutex> lock(s.mu);
+    if (!s.addr[dev]) {
+        void* p = nullptr;
+        FP8VIT_CUDA_TRY(cudaGetSymbolAddress(&p, g_amax_noalloc_scratch));
+        int sms = 0;
+        FP8VIT_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+        s.num_sms[dev] = sms;
+        s.addr[dev] = p;
+    }
+    *addr = s.addr[dev];
+    *num_sms = s.num_sms[dev];
+    return FP8VIT_OK;
+}
+
+}  // namespace
+
+extern "C" fp8vit_status fp8_amax_ring_update_noalloc(const uint16_t* d_q, const uint16_t* d_k,
+                                                      const uint16_t* d_v, int64_t n_elems,
+                                                      void* d_ring, float* d_descale3,
+                                                      void* stream) {
+    if (!d_q || !d_k || !d_v || !d_ring || !d_descale3 || n_elems < 0) return FP8VIT_EINVAL;
+    if (misaligned(d_q, 16) || misaligned(d_k, 16) || misaligned(d_v, 16) ||
+        misaligned(d_ring, 16) || misaligned(d_descale3, 4))
+        return FP8VIT_EINVAL;
+    if (sizeof(fp8vit_scratch) > kNoAllocScratchBytes) return FP8VIT_EUNSUPPORTED;
+    void* scratch = nullptr;
+    int num_sms = 0;
+    fp8vit_status st = noalloc_scratch(&scratch, &num_sms);
+    if (st != FP8VIT_OK) return st;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    // The array keeps whatever the previous call left; the kernel needs the
+    // maxima and the arrival counter at zero.
+    FP8VIT_CUDA_TRY(cudaMemsetAsync(scratch, 0, sizeof(fp8vit_scratch), cs));
+    const int grid = grid_for(n_elems >> 3, kAmaxThreads, 8, 4 * num_sms);
+    amax_ring_kernel<<<grid, kAmaxThreads, 0, cs>>>(
+        reinterpret_cast<const uint4*>(d_q), reinterpret_cast<const uint4*>(d_k),
+        reinterpret_cast<const uint4*>(d_v), n_elems, reinterpret_cast<fp8vit_ring*>(d_ring),
+        d_descale3, reinterpret_cast<fp8vit_scratch*>(scratch));
+    return cudaGetLastError() == cudaSuccess ? FP8VIT_OK : FP8VIT_ECUDA;
+}

@@ -100,6 +100,29 @@ fp8vit_status fp8_amax_ring_update(fp8vit_ctx* ctx, const uint16_t* d_q, const u
                                    const uint16_t* d_v, int64_t n_elems, void* d_ring,
                                    float* d_descale3, void* stream);
 
+/* Same computation and arguments as fp8_amax_ring_update, for callers that
+ * cannot allocate device memory where they run (for example a process whose
+ * memory pool already holds nearly all free HBM, code that must avoid
+ * cudaMalloc's device-wide synchronisation, or a caller with no place to keep
+ * a context, since fp8vit_create allocates).  The pages describe no such
+ * entry point; it has no counterpart there.
+ *   - Takes no context and allocates nothing: its 128 bytes of scratch come
+ *     from a 256-byte array built into the library's device image, which
+ *     every GPU that loads the library keeps until the process exits.  The
+ *     scratch need does not grow with n_elems; a need above the array's
+ *     capacity would be refused with FP8VIT_EUNSUPPORTED.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture on the device.
+ *   - Every call on a device shares the one array: each call clears it with
+ *     a 128-byte memset on `stream` before its kernel.  Calls whose work
+ *     overlaps on the GPU (different streams, no ordering) race on it and
+ *     give wrong maxima; order such calls, or use the context entry point.
+ * Returns FP8VIT_EINVAL for the same argument errors as fp8_amax_ring_update. */
+fp8vit_status fp8_amax_ring_update_noalloc(const uint16_t* d_q, const uint16_t* d_k,
+                                           const uint16_t* d_v, int64_t n_elems, void* d_ring,
+                                           float* d_descale3, void* stream);
+
 /* Host helper for the calibrate-once workflow (vLLM "FP8 ViT Encoder
  * Attention", "Calibrate-Once, Reuse Workflow"): synchronize `stream`, copy
  * the ring state to the host and return max_j hist[t][j] for t = q, k, v. */
