@@ -197,6 +197,50 @@ def run_reference(args):
     return 0
 
 
+def _quant_rooflines(fv, ctx, src, dev, hbm_gbs, reps=10):
+    """HBM roofline of the three quantizer kernels on 3 x 32400-token, 16-head,
+    head_dim-72 tensors ([97200, 1152] BF16 each, 224 MB): the resident BF16
+    inputs are tiled on the device to that size (same value distribution).
+    Each kernel reads more than the 126 MB L2, so its bytes come from HBM."""
+    import torch
+    n = 97200 * 1152
+    flat = [t.reshape(-1) for t in src]
+    big = [f.repeat((n + f.numel() - 1) // f.numel())[:n].contiguous() for f in flat]
+    ring = fv.new_ring(dev)
+    desc = torch.zeros(3, dtype=torch.float32, device=dev)
+    q8, k8, v8 = (torch.empty(n, dtype=torch.uint8, device=dev) for _ in range(3))
+    xq = torch.empty((97200, 1152), dtype=torch.uint8, device=dev)
+    xs = torch.empty((97200, 9), dtype=torch.float32, device=dev)
+    x2 = big[0].view(97200, 1152)
+    runs = {
+        "amax_ring_kernel": (lambda: fv.fp8_amax_ring_update(*big, ring, desc, ctx=ctx),
+                             3 * n * 2),
+        "quant3_kernel": (lambda: fv.fp8_quantize_qkv_per_tensor(*big, desc, q8, k8, v8,
+                                                                 ctx=ctx), 3 * n * 3),
+        "group_quant_kernel": (lambda: fv.per_token_group_quant_fp8(x2, 128, xq, xs, ctx=ctx),
+                               n * 3 + (n // 128) * 4),
+    }
+    out = {}
+    stream = torch.cuda.current_stream(dev)
+    for name, (fn, nbytes) in runs.items():
+        for _ in range(3):
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        for a, b in evs:
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[name] = {"bytes": nbytes, "ms": ms, "achieved_GBps": gbs, "peak_GBps": hbm_gbs,
+                     "frac": gbs / hbm_gbs}
+    del big, q8, k8, v8, xq, xs
+    return {"workload": "3x32400 tokens, 16 heads, head_dim 72 ([97200, 1152] per tensor)",
+            "bound": "hbm", "kernels": out}
+
+
 def _config(w, n_fwd=None):
     n_fwd = len(w.seeds) if n_fwd is None else n_fwd
     gb = n_fwd * 3 * w.tokens * w.hd * 2 / 1e9
@@ -332,6 +376,8 @@ def run_ours(args):
 
     peaks = _peaks()
     fp8_peak = 2.0 * peaks["bf16"]  # dense FP8 = 2 x dense BF16 (nominal ratio)
+    quant = None if args.no_quant_roofline else _quant_rooflines(fv, ctx, inputs[0], dev,
+                                                                 peaks["hbm"])
     traffic = _traffic(os.path.join(ROOT, "fp8_quantized_vit_b200", "csrc", "attn.cu"),
                        args.workload)
     line = {
@@ -348,6 +394,7 @@ def run_ours(args):
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": 4 * args.steps,
         "clocks": clk,
+        "quantizers": quant,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         codes, dsc = _oracle_inputs(w)
@@ -378,6 +425,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=1.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-quant-roofline", action="store_true")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

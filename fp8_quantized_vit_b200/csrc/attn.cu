@@ -110,6 +110,72 @@ __device__ __forceinline__ void tmem_ld8_sync(uint32_t taddr, uint32_t (&r)[8]) 
         : "memory");
 }
 
+// All 128 columns of this thread's lane, then wait.
+__device__ __forceinline__ void tmem_ld128_sync(uint32_t taddr, uint32_t (&r)[128]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x128.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,"
+        "%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,"
+        "%58,%59,%60,%61,%62,%63,%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,"
+        "%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,"
+        "%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,"
+        "%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%128];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]),
+          "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]),
+          "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]),
+          "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]),
+          "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]),
+          "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]),
+          "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]),
+          "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]),
+          "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]),
+          "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]),
+          "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]),
+          "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]),
+          "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]),
+          "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]),
+          "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]),
+          "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]),
+          "=r"(r[127])
+        : "r"(taddr)
+        : "memory");
+}
+
+// Issue a 32-column load without waiting; pair with tmem_wait_ld_dep(r).
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+// Wait for this thread's outstanding TMEM loads.  The registers are listed as
+// read-write operands so the compiler cannot move their uses above the wait.
+__device__ __forceinline__ void tmem_wait_ld_dep(uint32_t (&r)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]),
+                   "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                   "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]),
+                   "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
 // ---- packed arithmetic used by the softmax --------------------------------
 
 __device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
@@ -127,7 +193,7 @@ __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
 }
 __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
     uint64_t d;
-    asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -135,29 +201,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
 }
-// f32 pair -> f16x2 (lo in bits 0..15)
-__device__ __forceinline__ uint32_t cvt_f16x2(float lo, float hi) {
-    uint32_t d;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
-    return d;
-}
-// f16x2 -> two e4m3 codes (RNE, satfinite; bits 0..15 -> byte 0)
-__device__ __forceinline__ uint32_t e4m3x2_of_f16x2(uint32_t h) {
-    uint16_t d;
-    asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(d) : "r"(h));
-    return d;
-}
-__device__ __forceinline__ uint32_t f16x2_of_e4m3x2(uint32_t e) {
-    uint32_t d;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"((uint16_t)e));
-    return d;
-}
-__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-
 // 2^x on the FMA pipe for a pair of arguments (x >= -126 after the clamp).
 // Cody-Waite reduction x = n + f, n = rint(x) via the 1.5 * 2^23 magic add,
 // f in [-0.5, 0.5]; 2^f by a degree-3 polynomial fitted for minimal relative
@@ -186,20 +229,148 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float&
     y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
-// Split 4 probabilities into one hi word and one lo word of e4m3 codes:
-// hi = e4m3(p), lo = e4m3(p - hi), with p first rounded to f16 (11 bits) and
-// the residual formed exactly in f16.  hi + lo carries ~8 significant bits,
-// so the PV product on FP8 tensor cores loses no more than a BF16-width P.
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// Two 16-bit halves into one word (lo in bits 0..15).
+__device__ __forceinline__ uint32_t pack_h2(uint16_t lo, uint16_t hi) {
+    uint32_t d;
+    asm("mov.b32 %0, {%1, %2};" : "=r"(d) : "h"(lo), "h"(hi));
+    return d;
+}
+
+// Split 4 probabilities into one hi word and one lo word of e4m3 codes,
+// hi + lo ~= p with ~8 significant bits, so that the PV product on FP8
+// tensor cores keeps about a BF16-width P.  Veltkamp's splitting (Dekker,
+// "A floating-point technique for extending the available precision", 1971)
+// with factor 2^20 + 1 cuts each fp32 p into h (4 significant bits, exactly
+// an e4m3 value in the normal range) and the exact remainder p - h; the
+// remainder is then rounded to e4m3.  The split runs on the FMA pipe
+// (packed f32x2); only the two e4m3 conversions per pair use the ALU.
+// t = c - p is formed as fma(p, -1, c): written as a subtraction, the code
+// generator folds c - (c - p) back into p and the remainder vanishes.
 __device__ __forceinline__ void p_split4(float p0, float p1, float p2, float p3, uint32_t& hi,
                                          uint32_t& lo) {
-    const uint32_t h01 = cvt_f16x2(p0, p1);
-    const uint32_t h23 = cvt_f16x2(p2, p3);
-    const uint32_t e01 = e4m3x2_of_f16x2(h01);
-    const uint32_t e23 = e4m3x2_of_f16x2(h23);
-    const uint32_t l01 = e4m3x2_of_f16x2(hsub2(h01, f16x2_of_e4m3x2(e01)));
-    const uint32_t l23 = e4m3x2_of_f16x2(hsub2(h23, f16x2_of_e4m3x2(e23)));
-    hi = e01 | (e23 << 16);
-    lo = l01 | (l23 << 16);
+    const uint64_t k = f2pack(1048577.0f, 1048577.0f);
+    const uint64_t m1 = f2pack(-1.0f, -1.0f);
+    const uint64_t a = f2pack(p0, p1), b = f2pack(p2, p3);
+    const uint64_t ca = fmul2(a, k), cb = fmul2(b, k);
+    const uint64_t ha = fsub2(ca, ffma2(a, m1, ca)), hb = fsub2(cb, ffma2(b, m1, cb));
+    const uint64_t la = fsub2(a, ha), lb = fsub2(b, hb);
+    float h0, h1, h2, h3, l0, l1, l2, l3;
+    f2unpack(ha, h0, h1);
+    f2unpack(hb, h2, h3);
+    f2unpack(la, l0, l1);
+    f2unpack(lb, l2, l3);
+    hi = pack_h2(f32x2_to_e4m3x2(h0, h1), f32x2_to_e4m3x2(h2, h3));
+    lo = pack_h2(f32x2_to_e4m3x2(l0, l1), f32x2_to_e4m3x2(l2, l3));
+}
+
+#ifndef FP8VIT_POLY_EVERY
+#define FP8VIT_POLY_EVERY 0
+#endif
+
+// Row max of one S tile (128 keys of this thread's row; only the first
+// `nvalid` keys count when !FULL).
+template <bool FULL>
+__device__ __forceinline__ float tile_row_max(uint32_t tS, int nvalid) {
+    uint32_t r[128];
+    tmem_ld128_sync(tS, r);
+    {
+        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 128; i += 8) {
+            m0 = fmax3(m0, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+            m1 = fmax3(m1, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+            m2 = fmax3(m2, __uint_as_float(r[i + 4]), __uint_as_float(r[i + 5]));
+            m3 = fmax3(m3, __uint_as_float(r[i + 6]), __uint_as_float(r[i + 7]));
+        }
+        return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+    }
+}
+
+template <>
+__device__ __forceinline__ float tile_row_max<false>(uint32_t tS, int nvalid) {
+    float m = -INFINITY;
+#pragma unroll 1
+    for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32_sync(tS + 32 * c, r);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (32 * c + i < nvalid) m = fmaxf(m, __uint_as_float(r[i]));
+    }
+    return m;
+}
+
+// Probabilities of one 32-key chunk: p = 2^(s * c - bias), summed into the
+// two packed accumulators, split into 8 hi and 8 lo words of e4m3 codes.
+template <bool FULL>
+__device__ __forceinline__ void p_chunk(const uint32_t (&r)[32], int key0, int nvalid,
+                                        uint64_t c2, uint64_t nb2, uint64_t& l0, uint64_t& l1,
+                                        uint32_t (&pk)[16]) {
+    float p[32];
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+        float x0, x1;
+        f2unpack(ffma2(f2pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), c2, nb2), x0,
+                 x1);
+        if (!FULL) {
+            x0 = (key0 + i < nvalid) ? x0 : -INFINITY;
+            x1 = (key0 + i + 1 < nvalid) ? x1 : -INFINITY;
+            p[i] = ex2_approx(x0);
+            p[i + 1] = ex2_approx(x1);
+        } else if (FP8VIT_POLY_EVERY > 0 &&
+                   (i / 2) % (FP8VIT_POLY_EVERY > 0 ? FP8VIT_POLY_EVERY : 1) ==
+                       FP8VIT_POLY_EVERY - 1) {
+            exp2_poly2(x0, x1, p[i], p[i + 1]);
+        } else {
+            p[i] = ex2_approx(x0);
+            p[i + 1] = ex2_approx(x1);
+        }
+        if ((i / 2) & 1)
+            l1 = fadd2(l1, f2pack(p[i], p[i + 1]));
+        else
+            l0 = fadd2(l0, f2pack(p[i], p[i + 1]));
+    }
+#pragma unroll
+    for (int w = 0; w < 8; ++w)
+        p_split4(p[4 * w], p[4 * w + 1], p[4 * w + 2], p[4 * w + 3], pk[w], pk[8 + w]);
+}
+
+// P of one S tile written back over the consumed S columns: chunk c (keys
+// 32c..32c+31) goes to columns [16c, 16c+8) (hi) and [16c+8, 16c+16) (lo).
+// The load of chunk c+1 is in flight while chunk c is computed.
+template <bool FULL>
+__device__ __forceinline__ float tile_p(uint32_t tS, int nvalid, uint64_t c2, uint64_t nb2) {
+    uint32_t ra[32], rb[32], pk[16];
+    uint64_t l0 = f2pack(0.0f, 0.0f), l1 = l0;
+    tmem_ld32_async(tS, ra);
+    tmem_wait_ld_dep(ra);
+    tmem_ld32_async(tS + 32, rb);
+    p_chunk<FULL>(ra, 0, nvalid, c2, nb2, l0, l1, pk);
+    tmem_st16(tS, pk);
+    tmem_wait_ld_dep(rb);
+    tmem_ld32_async(tS + 64, ra);
+    p_chunk<FULL>(rb, 32, nvalid, c2, nb2, l0, l1, pk);
+    tmem_st16(tS + 16, pk);
+    tmem_wait_ld_dep(ra);
+    tmem_ld32_async(tS + 96, rb);
+    p_chunk<FULL>(ra, 64, nvalid, c2, nb2, l0, l1, pk);
+    tmem_st16(tS + 32, pk);
+    tmem_wait_ld_dep(rb);
+    p_chunk<FULL>(rb, 96, nvalid, c2, nb2, l0, l1, pk);
+    tmem_st16(tS + 48, pk);
+    float a0, a1;
+    f2unpack(fadd2(l0, l1), a0, a1);
+    return a0 + a1;
 }
 
 template <int D>
@@ -405,31 +576,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             tc_fence_after();
             const int nvalid = min(kBN, seg_len - j * kBN);
             const bool full = nvalid == kBN;
-            // pass 1: row max over the valid keys
-            float mx = -INFINITY;
-            if (full) {
-                float m2 = -INFINITY;
-#pragma unroll
-                for (int c = 0; c < kBN / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32_sync(tS + 32 * c, r);
-#pragma unroll
-                    for (int i = 0; i < 32; i += 4) {
-                        mx = fmax3(mx, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
-                        m2 = fmax3(m2, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
-                    }
-                }
-                mx = fmaxf(mx, m2);
-            } else {
-#pragma unroll
-                for (int c = 0; c < kBN / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32_sync(tS + 32 * c, r);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (32 * c + i < nvalid) mx = fmaxf(mx, __uint_as_float(r[i]));
-                }
-            }
+            const float mx = full ? tile_row_max<true>(tS, nvalid)
+                                  : tile_row_max<false>(tS, nvalid);
             const float mxc = mx * scale_log2;
             if (j == 0) {
                 m_ref = mxc;  // the first PV initialises O, nothing to rescale
@@ -460,40 +608,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const float bias = m_ref - kPLog2;
             const uint64_t c2 = f2pack(scale_log2, scale_log2);
             const uint64_t nb2 = f2pack(-bias, -bias);
-            uint64_t lacc0 = f2pack(0.0f, 0.0f), lacc1 = lacc0;
-#pragma unroll
-            for (int c = 0; c < kBN / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32_sync(tS + 32 * c, r);
-                float p[32];
-#pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    float x0, x1;
-                    f2unpack(ffma2(f2pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), c2,
-                                   nb2),
-                             x0, x1);
-                    if (!full) {
-                        x0 = (32 * c + i < nvalid) ? x0 : -INFINITY;
-                        x1 = (32 * c + i + 1 < nvalid) ? x1 : -INFINITY;
-                    }
-                    p[i] = ex2_approx(x0);
-                    p[i + 1] = ex2_approx(x1);
-                    if (i & 2)
-                        lacc1 = fadd2(lacc1, f2pack(p[i], p[i + 1]));
-                    else
-                        lacc0 = fadd2(lacc0, f2pack(p[i], p[i + 1]));
-                }
-                uint32_t pk[16];
-#pragma unroll
-                for (int w = 0; w < 8; ++w)
-                    p_split4(p[4 * w], p[4 * w + 1], p[4 * w + 2], p[4 * w + 3], pk[w], pk[8 + w]);
-                tmem_st16(tS + 16 * c, pk);
-            }
-            {
-                float a0, a1;
-                f2unpack(fadd2(lacc0, lacc1), a0, a1);
-                l_run += a0 + a1;
-            }
+            l_run += full ? tile_p<true>(tS, nvalid, c2, nb2) : tile_p<false>(tS, nvalid, c2, nb2);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(b_p_full);
