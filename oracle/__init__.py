@@ -37,35 +37,61 @@ def build(force: bool = False) -> str:
     return _LIB_PATH
 
 
+def _load_signatures(lib):
+    sig = {
+        "orc_e4m3_decode": (ctypes.c_double, [ctypes.c_uint8]),
+        "orc_e4m3_encode": (ctypes.c_uint8, [_F32]),
+        "orc_e4m3_encode_array": (None, [_P, _I64, _P]),
+        "orc_e4m3_decode_array": (None, [_P, _I64, _P]),
+        "orc_bf16_to_float": (_F32, [ctypes.c_uint16]),
+        "orc_double_to_bf16": (ctypes.c_uint16, [ctypes.c_double]),
+        "orc_amax_bf16": (_F32, [_P, _I64]),
+        "orc_descale_from_amax": (_F32, [_F32]),
+        "orc_ring_update": (None, [_P, _P, _P, _P]),
+        "orc_quantize_per_tensor": (None, [_P, _I64, _F32, _P]),
+        "orc_group_quant": (ctypes.c_int, [_P, _I64, _I64, _I32, _P, _P]),
+        "orc_attn_pairs": (ctypes.c_int, [_P, _P, _P, _F32, _F32, _F32, _P, _I32, _I32, _I32,
+                                          _F32, _P, _P, _I64, _P, _P]),
+        "orc_attn_full": (ctypes.c_int, [_P, _P, _P, _F32, _F32, _F32, _P, _I32, _I32, _I32,
+                                         _F32, _P]),
+        "orc_fp8_output": (None, [_P, _I64, _F32, _P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+
+
 def _load():
     global _lib
     if _lib is None:
         build()
         lib = ctypes.CDLL(_LIB_PATH)
-        sig = {
-            "orc_e4m3_decode": (ctypes.c_double, [ctypes.c_uint8]),
-            "orc_e4m3_encode": (ctypes.c_uint8, [_F32]),
-            "orc_e4m3_encode_array": (None, [_P, _I64, _P]),
-            "orc_e4m3_decode_array": (None, [_P, _I64, _P]),
-            "orc_bf16_to_float": (_F32, [ctypes.c_uint16]),
-            "orc_double_to_bf16": (ctypes.c_uint16, [ctypes.c_double]),
-            "orc_amax_bf16": (_F32, [_P, _I64]),
-            "orc_descale_from_amax": (_F32, [_F32]),
-            "orc_ring_update": (None, [_P, _P, _P, _P]),
-            "orc_quantize_per_tensor": (None, [_P, _I64, _F32, _P]),
-            "orc_group_quant": (ctypes.c_int, [_P, _I64, _I64, _I32, _P, _P]),
-            "orc_attn_pairs": (ctypes.c_int, [_P, _P, _P, _F32, _F32, _F32, _P, _I32, _I32, _I32,
-                                              _F32, _P, _P, _I64, _P, _P]),
-            "orc_attn_full": (ctypes.c_int, [_P, _P, _P, _F32, _F32, _F32, _P, _I32, _I32, _I32,
-                                             _F32, _P]),
-            "orc_fp8_output": (None, [_P, _I64, _F32, _P]),
-        }
-        for name, (res, args) in sig.items():
-            fn = getattr(lib, name)
-            fn.restype = res
-            fn.argtypes = args
+        _load_signatures(lib)
         _lib = lib
     return _lib
+
+
+class use_library:
+    """Context manager: route the wrappers below to another build of the
+    oracle (used by the tests that plant mistakes in a copy of oracle.c to
+    show the pins catch them)."""
+
+    def __init__(self, path: str):
+        self.path = path
+
+    def __enter__(self):
+        global _lib
+        self.saved = _load()
+        lib = ctypes.CDLL(self.path)
+        _load_signatures(lib)
+        _lib = lib
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.saved
+        return False
 
 
 def _c(a, dtype):
