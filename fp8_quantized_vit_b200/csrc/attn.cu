@@ -4,11 +4,13 @@
 // output_scale epilogue that writes e4m3).
 //
 // One CTA = one (image, head, 128-row query tile).  Warp roles:
-//   warp 0      TMA producer: Q once, then K/V tiles of 128 keys into an
+//   warp 0      TMA producer: Q once, then K/V tiles of 64 keys into an
 //               NS-stage shared-memory ring (SWIZZLE_32B, 32-byte boxes).
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer:
-//               S = Q K^T (kind::f8f6f4, K-major A and B) into TMEM,
-//               O += P V  (A = P from TMEM, B = V MN-major from smem).
+//               S = Q K^T (kind::f8f6f4, K-major A and B) into one of two
+//               TMEM S buffers, O += P V (A = P from TMEM, B = V MN-major
+//               from smem).  The next tile's S is computed while the softmax
+//               warps work on the current one.
 //   warps 2..5  softmax + epilogue, one query row per thread (TMEM lane):
 //               row max, exp2, row sum in registers; P written back to TMEM
 //               as two e4m3 terms (hi + lo) so that the PV product keeps
@@ -26,13 +28,14 @@
 namespace {
 
 constexpr int kBM = 128;          // query rows per CTA (MMA M)
-constexpr int kBN = 128;          // keys per KV tile
+constexpr int kBN = 64;           // keys per KV tile (QK MMA N, PV MMA K)
 constexpr int kThreads = 192;     // 6 warps
 constexpr int kTmemCols = 256;
-constexpr uint32_t kTmemS = 0;    // S columns [0,128); P hi/lo written over [0,64)
+constexpr uint32_t kTmemS = 0;    // S buffers: columns [0,64) and [64,128); P over [64b, 64b+32)
 constexpr uint32_t kTmemO = 128;  // O accumulator columns [128, 128 + NPV)
 constexpr int kBox = 32;          // bytes per TMA box row (one SW32 atom row)
-constexpr int kTileBytes = kBox * 128;  // one [128 rows x 32 B] box
+constexpr int kQTileBytes = kBox * kBM;   // one [128 rows x 32 B] Q box
+constexpr int kKVTileBytes = kBox * kBN;  // one [64 rows x 32 B] K or V box
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 // P is stored as 2^(x - m_ref + kPLog2); a tile max up to kSlackLog2 above the
 // reference max keeps P <= 2^(6 + 2.75) = 430 < 448 (e4m3 max).
@@ -46,36 +49,36 @@ struct Cfg<72> {
     static constexpr int KB = 3;    // 32-byte k-blocks of the QK contraction (96 bytes)
     static constexpr int VA = 3;    // 32-byte V column blocks loaded (96 bytes)
     static constexpr int NPV = 80;  // PV MMA N (covers head bytes [0,72) or [8,80))
-    static constexpr int NS = 3;    // K/V pipeline stages
+    static constexpr int NS = 5;    // K/V pipeline stages
 };
 template <>
 struct Cfg<128> {
     static constexpr int KB = 4;
     static constexpr int VA = 4;
     static constexpr int NPV = 128;
-    static constexpr int NS = 2;
+    static constexpr int NS = 4;
 };
 
 template <int D>
 struct Smem {
     static constexpr int Q = 0;
-    static constexpr int K = Q + Cfg<D>::KB * kTileBytes;
-    static constexpr int V = K + Cfg<D>::NS * Cfg<D>::KB * kTileBytes;
-    static constexpr int BAR = V + Cfg<D>::NS * Cfg<D>::VA * kTileBytes;
+    static constexpr int K = Q + Cfg<D>::KB * kQTileBytes;
+    static constexpr int V = K + Cfg<D>::NS * Cfg<D>::KB * kKVTileBytes;
+    static constexpr int BAR = V + Cfg<D>::NS * Cfg<D>::VA * kKVTileBytes;
     static constexpr int TOTAL = BAR + 256;
     static constexpr int ALLOC = TOTAL + 1024;  // slack for 1024-byte alignment
 };
 
 // Shared-memory matrix descriptors (tcgen05 "version 1" format), 32-byte
 // swizzle.  K-major: rows of 32 bytes, 8-row groups 256 bytes apart (SBO).
-// MN-major: 32-byte atoms along N, 4096 bytes apart (LBO); 8-key groups
-// 256 bytes apart (SBO).
+// MN-major (V): 32-byte atoms along N, one [64 keys x 32 B] box apart (LBO);
+// 8-key groups 256 bytes apart (SBO).
 __device__ __forceinline__ uint64_t desc_k_sw32(uint32_t addr) {
     return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(256 >> 4) << 32) |
            ((uint64_t)1 << 46) | ((uint64_t)6 << 61);
 }
 __device__ __forceinline__ uint64_t desc_mn_sw32(uint32_t addr) {
-    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)(kTileBytes >> 4) << 16) |
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)(kKVTileBytes >> 4) << 16) |
            ((uint64_t)(256 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)6 << 61);
 }
 
@@ -83,21 +86,6 @@ __device__ __forceinline__ uint64_t desc_mn_sw32(uint32_t addr) {
 __host__ __device__ constexpr uint32_t idesc_e4m3(int n, bool b_mn_major) {
     return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(n >> 3) << 17) |
            ((uint32_t)(128 >> 4) << 24);
-}
-
-__device__ __forceinline__ void tmem_ld32_sync(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-          "=r"(r[31])
-        : "r"(taddr)
-        : "memory");
 }
 
 __device__ __forceinline__ void tmem_ld8_sync(uint32_t taddr, uint32_t (&r)[8]) {
@@ -110,70 +98,14 @@ __device__ __forceinline__ void tmem_ld8_sync(uint32_t taddr, uint32_t (&r)[8]) 
         : "memory");
 }
 
-// All 128 columns of this thread's lane, then wait.
-__device__ __forceinline__ void tmem_ld128_sync(uint32_t taddr, uint32_t (&r)[128]) {
+// 64 consecutive columns of this thread's lane into a[0..31], b[0..31], then wait.
+__device__ __forceinline__ void tmem_ld64_sync(uint32_t taddr, uint32_t (&a)[32], uint32_t (&b)[32]) {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x128.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,"
-        "%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,"
-        "%58,%59,%60,%61,%62,%63,%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,"
-        "%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,"
-        "%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,"
-        "%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%128];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
         "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-          "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]),
-          "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]),
-          "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]),
-          "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]),
-          "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]),
-          "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]),
-          "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]),
-          "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]),
-          "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]),
-          "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]),
-          "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]),
-          "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]),
-          "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]),
-          "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]),
-          "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]),
-          "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]),
-          "=r"(r[127])
+        : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]), "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15]), "=r"(a[16]), "=r"(a[17]), "=r"(a[18]), "=r"(a[19]), "=r"(a[20]), "=r"(a[21]), "=r"(a[22]), "=r"(a[23]), "=r"(a[24]), "=r"(a[25]), "=r"(a[26]), "=r"(a[27]), "=r"(a[28]), "=r"(a[29]), "=r"(a[30]), "=r"(a[31]), "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7]), "=r"(b[8]), "=r"(b[9]), "=r"(b[10]), "=r"(b[11]), "=r"(b[12]), "=r"(b[13]), "=r"(b[14]), "=r"(b[15]), "=r"(b[16]), "=r"(b[17]), "=r"(b[18]), "=r"(b[19]), "=r"(b[20]), "=r"(b[21]), "=r"(b[22]), "=r"(b[23]), "=r"(b[24]), "=r"(b[25]), "=r"(b[26]), "=r"(b[27]), "=r"(b[28]), "=r"(b[29]), "=r"(b[30]), "=r"(b[31])
         : "r"(taddr)
         : "memory");
-}
-
-// Issue a 32-column load without waiting; pair with tmem_wait_ld_dep(r).
-__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-          "=r"(r[31])
-        : "r"(taddr)
-        : "memory");
-}
-
-// Wait for this thread's outstanding TMEM loads.  The registers are listed as
-// read-write operands so the compiler cannot move their uses above the wait.
-__device__ __forceinline__ void tmem_wait_ld_dep(uint32_t (&r)[32]) {
-    asm volatile("tcgen05.wait::ld.sync.aligned;"
-                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
-                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
-                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]),
-                   "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
-                   "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]),
-                   "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
-                 :
-                 : "memory");
 }
 
 // ---- packed arithmetic used by the softmax --------------------------------
@@ -277,35 +209,27 @@ __device__ __forceinline__ void p_split4(float p0, float p1, float p2, float p3,
 #define FP8VIT_POLY_EVERY 0
 #endif
 
-// Row max of one S tile (128 keys of this thread's row; only the first
-// `nvalid` keys count when !FULL).
+// Row max of one 64-key S tile held in registers (a = keys 0..31, b = keys
+// 32..63); only the first `nvalid` keys count when !FULL.
 template <bool FULL>
-__device__ __forceinline__ float tile_row_max(uint32_t tS, int nvalid) {
-    uint32_t r[128];
-    tmem_ld128_sync(tS, r);
-    {
+__device__ __forceinline__ float tile_row_max(const uint32_t (&a)[32], const uint32_t (&b)[32],
+                                              int nvalid) {
+    if (FULL) {
         float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 128; i += 8) {
-            m0 = fmax3(m0, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
-            m1 = fmax3(m1, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
-            m2 = fmax3(m2, __uint_as_float(r[i + 4]), __uint_as_float(r[i + 5]));
-            m3 = fmax3(m3, __uint_as_float(r[i + 6]), __uint_as_float(r[i + 7]));
+        for (int i = 0; i < 32; i += 4) {
+            m0 = fmax3(m0, __uint_as_float(a[i]), __uint_as_float(a[i + 1]));
+            m1 = fmax3(m1, __uint_as_float(a[i + 2]), __uint_as_float(a[i + 3]));
+            m2 = fmax3(m2, __uint_as_float(b[i]), __uint_as_float(b[i + 1]));
+            m3 = fmax3(m3, __uint_as_float(b[i + 2]), __uint_as_float(b[i + 3]));
         }
         return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
     }
-}
-
-template <>
-__device__ __forceinline__ float tile_row_max<false>(uint32_t tS, int nvalid) {
     float m = -INFINITY;
-#pragma unroll 1
-    for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32_sync(tS + 32 * c, r);
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-            if (32 * c + i < nvalid) m = fmaxf(m, __uint_as_float(r[i]));
+    for (int i = 0; i < 32; ++i) {
+        if (i < nvalid) m = fmaxf(m, __uint_as_float(a[i]));
+        if (32 + i < nvalid) m = fmaxf(m, __uint_as_float(b[i]));
     }
     return m;
 }
@@ -345,32 +269,21 @@ __device__ __forceinline__ void p_chunk(const uint32_t (&r)[32], int key0, int n
         p_split4(p[4 * w], p[4 * w + 1], p[4 * w + 2], p[4 * w + 3], pk[w], pk[8 + w]);
 }
 
-// P of one S tile written back over the consumed S columns: chunk c (keys
-// 32c..32c+31) goes to columns [16c, 16c+8) (hi) and [16c+8, 16c+16) (lo).
-// The load of chunk c+1 is in flight while chunk c is computed.
+// P of one 64-key tile written over the first 32 columns of its S buffer:
+// chunk c (keys 32c..32c+31) goes to columns [16c, 16c+8) (hi) and
+// [16c+8, 16c+16) (lo).  Returns the tile's probability sum.
 template <bool FULL>
-__device__ __forceinline__ float tile_p(uint32_t tS, int nvalid, uint64_t c2, uint64_t nb2) {
-    uint32_t ra[32], rb[32], pk[16];
+__device__ __forceinline__ float tile_p(const uint32_t (&a)[32], const uint32_t (&b)[32],
+                                        uint32_t tSb, int nvalid, uint64_t c2, uint64_t nb2) {
+    uint32_t pk[16];
     uint64_t l0 = f2pack(0.0f, 0.0f), l1 = l0;
-    tmem_ld32_async(tS, ra);
-    tmem_wait_ld_dep(ra);
-    tmem_ld32_async(tS + 32, rb);
-    p_chunk<FULL>(ra, 0, nvalid, c2, nb2, l0, l1, pk);
-    tmem_st16(tS, pk);
-    tmem_wait_ld_dep(rb);
-    tmem_ld32_async(tS + 64, ra);
-    p_chunk<FULL>(rb, 32, nvalid, c2, nb2, l0, l1, pk);
-    tmem_st16(tS + 16, pk);
-    tmem_wait_ld_dep(ra);
-    tmem_ld32_async(tS + 96, rb);
-    p_chunk<FULL>(ra, 64, nvalid, c2, nb2, l0, l1, pk);
-    tmem_st16(tS + 32, pk);
-    tmem_wait_ld_dep(rb);
-    p_chunk<FULL>(rb, 96, nvalid, c2, nb2, l0, l1, pk);
-    tmem_st16(tS + 48, pk);
-    float a0, a1;
-    f2unpack(fadd2(l0, l1), a0, a1);
-    return a0 + a1;
+    p_chunk<FULL>(a, 0, nvalid, c2, nb2, l0, l1, pk);
+    tmem_st16(tSb, pk);
+    p_chunk<FULL>(b, 32, nvalid, c2, nb2, l0, l1, pk);
+    tmem_st16(tSb + 16, pk);
+    float s0, s1;
+    f2unpack(fadd2(l0, l1), s0, s1);
+    return s0 + s1;
 }
 
 template <int D>
@@ -406,26 +319,32 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t sQ = smem_u32(sm + L::Q);
     const uint32_t sK = smem_u32(sm + L::K);
     const uint32_t sV = smem_u32(sm + L::V);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR);
-    const uint32_t bar0 = smem_u32(bars);
+    const uint32_t bar0 = smem_u32(sm + L::BAR);
     // barrier indices
+    // Barriers of per-tile events come in pairs indexed by the tile's parity
+    // (b = j & 1), so that a waiter is never more than one phase behind the
+    // phase it waits for: tile j's event is completion (j >> 1) of barrier b.
     const uint32_t b_q_full = bar0 + 8 * 0;
     const uint32_t b_q_ready = bar0 + 8 * 1;
-    const uint32_t b_s_full = bar0 + 8 * 2;
-    const uint32_t b_p_full = bar0 + 8 * 3;
-    const uint32_t b_o_ready = bar0 + 8 * 4;
-    auto b_k_full = [&](int s) { return bar0 + 8 * (5 + s); };
-    auto b_v_full = [&](int s) { return bar0 + 8 * (5 + NS + s); };
-    auto b_kv_empty = [&](int s) { return bar0 + 8 * (5 + 2 * NS + s); };
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::BAR + 8 * (5 + 3 * NS));
+    const uint32_t b_drain = bar0 + 8 * 2;
+    auto b_s_full = [&](int b) { return bar0 + 8 * (3 + b); };   // S(j) computed
+    auto b_p_full = [&](int b) { return bar0 + 8 * (5 + b); };   // P(j) written
+    auto b_o_ready = [&](int b) { return bar0 + 8 * (7 + b); };  // PV(j) complete
+    auto b_k_full = [&](int s) { return bar0 + 8 * (9 + s); };
+    auto b_v_full = [&](int s) { return bar0 + 8 * (9 + NS + s); };
+    auto b_kv_empty = [&](int s) { return bar0 + 8 * (9 + 2 * NS + s); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::BAR + 8 * (9 + 3 * NS));
     volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
 
     if (threadIdx.x == 0) {
         mbar_init(b_q_full, 1);
         mbar_init(b_q_ready, 128);
-        mbar_init(b_s_full, 1);
-        mbar_init(b_p_full, 128);
-        mbar_init(b_o_ready, 1);
+        mbar_init(b_drain, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(b_s_full(b), 1);
+            mbar_init(b_p_full(b), 128);
+            mbar_init(b_o_ready(b), 1);
+        }
         for (int s = 0; s < NS; ++s) {
             mbar_init(b_k_full(s), 1);
             mbar_init(b_v_full(s), 1);
@@ -453,9 +372,10 @@ __global__ void __launch_bounds__(kThreads, 2)
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
-            mbar_arrive_expect_tx(b_q_full, C::KB * kTileBytes);
+            mbar_arrive_expect_tx(b_q_full, C::KB * kQTileBytes);
             for (int kb = 0; kb < C::KB; ++kb)
-                tma_load_2d(sQ + kb * kTileBytes, &tm_q, x0 + kBox * kb, seg_start + q0, b_q_full);
+                tma_load_2d(sQ + kb * kQTileBytes, &tm_q, x0 + kBox * kb, seg_start + q0,
+                            b_q_full);
             int issued = 0;
             for (int j = 0; j < n_kv; ++j) {
                 const int s = j % NS;
@@ -464,13 +384,13 @@ __global__ void __launch_bounds__(kThreads, 2)
                                        SITE_ATTN_WAIT_EMPTY, kTimeoutNs))
                     break;
                 const int32_t row = seg_start + j * kBN;
-                mbar_arrive_expect_tx(b_k_full(s), C::KB * kTileBytes);
+                mbar_arrive_expect_tx(b_k_full(s), C::KB * kKVTileBytes);
                 for (int kb = 0; kb < C::KB; ++kb)
-                    tma_load_2d(sK + (s * C::KB + kb) * kTileBytes, &tm_k, x0 + kBox * kb, row,
+                    tma_load_2d(sK + (s * C::KB + kb) * kKVTileBytes, &tm_k, x0 + kBox * kb, row,
                                 b_k_full(s));
-                mbar_arrive_expect_tx(b_v_full(s), C::VA * kTileBytes);
+                mbar_arrive_expect_tx(b_v_full(s), C::VA * kKVTileBytes);
                 for (int a = 0; a < C::VA; ++a)
-                    tma_load_2d(sV + (s * C::VA + a) * kTileBytes, &tm_v, x0 + kBox * a, row,
+                    tma_load_2d(sV + (s * C::VA + a) * kKVTileBytes, &tm_v, x0 + kBox * a, row,
                                 b_v_full(s));
                 ++issued;
             }
@@ -486,53 +406,73 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
+        // S(j) = Q K_j^T goes to S buffer j & 1.  S(j+1) is issued before P(j)
+        // is waited for, so the tensor cores compute the next scores while
+        // the softmax warps work on the current ones; the buffer it reuses
+        // held P(j-1), so PV(j-1) must have completed first.
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_e4m3(kBN, false);
             constexpr uint32_t idesc_pv = idesc_e4m3(C::NPV, true);
-            const uint32_t tS = tmem + kTmemS, tO = tmem + kTmemO;
-            bool ok = mbar_wait_bounded(b_q_ready, 0, abort_flag, scr, SITE_ATTN_WAIT_QREADY,
-                                        kTimeoutNs);
-            int committed = 0;  // number of o_ready commits issued
-            for (int j = 0; ok && j < n_kv; ++j) {
+            const uint32_t tO = tmem + kTmemO;
+            auto issue_qk = [&](int j) {
                 const int s = j % NS;
-                const uint32_t ph = (j / NS) & 1;
-                if (!mbar_wait_bounded(b_k_full(s), ph, abort_flag, scr, SITE_ATTN_WAIT_K,
-                                       kTimeoutNs))
-                    break;
-                // S may be overwritten only after PV of the previous tile has
-                // read P out of it.
-                if (j > 0 && !mbar_wait_bounded(b_o_ready, (j - 1) & 1, abort_flag, scr,
-                                                SITE_ATTN_WAIT_O, kTimeoutNs))
-                    break;
-                tc_fence_after();
+                const uint32_t tSb = tmem + kTmemS + 64 * (j & 1);
 #pragma unroll
                 for (int kb = 0; kb < C::KB; ++kb)
-                    umma_f8_ss(tS, desc_k_sw32(sQ + kb * kTileBytes),
-                               desc_k_sw32(sK + (s * C::KB + kb) * kTileBytes), idesc_qk,
+                    umma_f8_ss(tSb, desc_k_sw32(sQ + kb * kQTileBytes),
+                               desc_k_sw32(sK + (s * C::KB + kb) * kKVTileBytes), idesc_qk,
                                kb > 0 ? 1u : 0u);
-                umma_commit(b_s_full);
-                if (!mbar_wait_bounded(b_v_full(s), ph, abort_flag, scr, SITE_ATTN_WAIT_V,
-                                       kTimeoutNs))
+                umma_commit(b_s_full(j & 1));
+            };
+            bool ok = mbar_wait_bounded(b_q_ready, 0, abort_flag, scr, SITE_ATTN_WAIT_QREADY,
+                                        kTimeoutNs);
+            bool issued_any = false;
+            if (ok) {
+                ok = mbar_wait_bounded(b_k_full(0), 0, abort_flag, scr, SITE_ATTN_WAIT_K,
+                                       kTimeoutNs);
+                if (ok) {
+                    tc_fence_after();
+                    issue_qk(0);
+                    issued_any = true;
+                }
+            }
+            for (int j = 0; ok && j < n_kv; ++j) {
+                if (j + 1 < n_kv) {
+                    const int s1 = (j + 1) % NS;
+                    if (!mbar_wait_bounded(b_k_full(s1), ((j + 1) / NS) & 1, abort_flag, scr,
+                                           SITE_ATTN_WAIT_K, kTimeoutNs))
+                        break;
+                    if (j >= 1 && !mbar_wait_bounded(b_o_ready((j - 1) & 1), ((j - 1) >> 1) & 1,
+                                                     abort_flag, scr, SITE_ATTN_WAIT_O,
+                                                     kTimeoutNs))
+                        break;
+                    tc_fence_after();
+                    issue_qk(j + 1);
+                }
+                const int s = j % NS;
+                if (!mbar_wait_bounded(b_v_full(s), (j / NS) & 1, abort_flag, scr,
+                                       SITE_ATTN_WAIT_V, kTimeoutNs))
                     break;
-                if (!mbar_wait_bounded(b_p_full, j & 1, abort_flag, scr, SITE_ATTN_WAIT_P,
-                                       kTimeoutNs))
+                if (!mbar_wait_bounded(b_p_full(j & 1), (j >> 1) & 1, abort_flag, scr,
+                                       SITE_ATTN_WAIT_P, kTimeoutNs))
                     break;
                 tc_fence_after();
-                const uint32_t vbase = sV + s * C::VA * kTileBytes;
+                const uint32_t tPb = tmem + kTmemS + 64 * (j & 1);
+                const uint32_t vbase = sV + s * C::VA * kKVTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < kBN / 32; ++kk) {
                     const uint64_t bdesc = desc_mn_sw32(vbase + kk * 32 * kBox);
-                    umma_f8_ts(tO, tS + 16 * kk, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-                    umma_f8_ts(tO, tS + 16 * kk + 8, bdesc, idesc_pv, 1u);
+                    umma_f8_ts(tO, tPb + 16 * kk, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_f8_ts(tO, tPb + 16 * kk + 8, bdesc, idesc_pv, 1u);
                 }
-                umma_commit(b_o_ready);
+                umma_commit(b_o_ready(j & 1));
                 umma_commit(b_kv_empty(s));
-                ++committed;
             }
-            // Never leave MMAs in flight: wait for the last commit.
-            if (committed > 0)
-                mbar_wait_bounded(b_o_ready, (committed - 1) & 1, abort_flag, scr,
-                                  SITE_ATTN_DRAIN, kTimeoutNs);
+            // Never leave MMAs in flight: one more commit tracks all of them.
+            if (issued_any) {
+                umma_commit(b_drain);
+                mbar_wait_bounded(b_drain, 0, abort_flag, scr, SITE_ATTN_DRAIN, kTimeoutNs);
+            }
         }
     } else {
         // ---------------- softmax + epilogue (warps 2..5) ----------------
@@ -551,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             // kb at kb*4096 + r*32, 16-byte chunk c stored at chunk c ^ ((r>>2)&1).
             uint8_t* q = sm + L::Q;
             const int sw = (row >> 2) & 1;
-            uint8_t* kb2 = q + 2 * kTileBytes + row * kBox;
+            uint8_t* kb2 = q + 2 * kQTileBytes + row * kBox;
             *reinterpret_cast<uint4*>(kb2 + ((1 ^ sw) << 4)) = make_uint4(0, 0, 0, 0);
             if (col_off == 0)
                 *reinterpret_cast<uint2*>(kb2 + ((0 ^ sw) << 4) + 8) = make_uint2(0, 0);
@@ -570,22 +510,27 @@ __global__ void __launch_bounds__(kThreads, 2)
         // by the same factor, so the final o = O / l is unchanged).
         float m_ref = -INFINITY, l_run = 0.0f;
         for (int j = 0; ok && j < n_kv; ++j) {
-            ok = mbar_wait_bounded(b_s_full, j & 1, abort_flag, scr, SITE_ATTN_WAIT_S, kTimeoutNs);
+            const int b = j & 1;
+            ok = mbar_wait_bounded(b_s_full(b), (j >> 1) & 1, abort_flag, scr, SITE_ATTN_WAIT_S,
+                                   kTimeoutNs);
             ok = __all_sync(0xFFFFFFFFu, ok);
             if (!ok) break;
             tc_fence_after();
+            const uint32_t tSb = tS + 64 * b;
             const int nvalid = min(kBN, seg_len - j * kBN);
             const bool full = nvalid == kBN;
-            const float mx = full ? tile_row_max<true>(tS, nvalid)
-                                  : tile_row_max<false>(tS, nvalid);
+            uint32_t ra[32], rb[32];
+            tmem_ld64_sync(tSb, ra, rb);
+            const float mx =
+                full ? tile_row_max<true>(ra, rb, nvalid) : tile_row_max<false>(ra, rb, nvalid);
             const float mxc = mx * scale_log2;
             if (j == 0) {
                 m_ref = mxc;  // the first PV initialises O, nothing to rescale
             } else {
                 const bool need = mxc > m_ref + kSlackLog2;
                 if (__any_sync(0xFFFFFFFFu, need)) {
-                    ok = mbar_wait_bounded(b_o_ready, (j - 1) & 1, abort_flag, scr,
-                                           SITE_ATTN_WAIT_O, kTimeoutNs);
+                    ok = mbar_wait_bounded(b_o_ready((j - 1) & 1), ((j - 1) >> 1) & 1,
+                                           abort_flag, scr, SITE_ATTN_WAIT_O, kTimeoutNs);
                     ok = __all_sync(0xFFFFFFFFu, ok);
                     if (!ok) break;
                     tc_fence_after();
@@ -604,19 +549,21 @@ __global__ void __launch_bounds__(kThreads, 2)
                     if (need) m_ref = mxc;
                 }
             }
-            // pass 2: P = 2^(x - bias), bias = m_ref - kPLog2
+            // P = 2^(x - bias), bias = m_ref - kPLog2
             const float bias = m_ref - kPLog2;
             const uint64_t c2 = f2pack(scale_log2, scale_log2);
             const uint64_t nb2 = f2pack(-bias, -bias);
-            l_run += full ? tile_p<true>(tS, nvalid, c2, nb2) : tile_p<false>(tS, nvalid, c2, nb2);
+            l_run += full ? tile_p<true>(ra, rb, tSb, nvalid, c2, nb2)
+                          : tile_p<false>(ra, rb, tSb, nvalid, c2, nb2);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(b_p_full);
+            mbar_arrive(b_p_full(b));
         }
         // epilogue
         if (ok) {
-            ok = mbar_wait_bounded(b_o_ready, (n_kv - 1) & 1, abort_flag, scr, SITE_ATTN_WAIT_O,
-                                   kTimeoutNs);
+            // PV(n_kv - 1)'s commit tracks every earlier MMA of the issuer too.
+            ok = mbar_wait_bounded(b_o_ready((n_kv - 1) & 1), ((n_kv - 1) >> 1) & 1, abort_flag,
+                                   scr, SITE_ATTN_WAIT_O, kTimeoutNs);
             ok = __all_sync(0xFFFFFFFFu, ok);
         }
         if (ok) {
@@ -663,12 +610,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 }
 
-bool encode_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_bytes) {
+bool encode_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_bytes,
+                int box_rows) {
     fp8vit_encode_tiled_fn enc = fp8vit_get_encode_tiled();
     if (!enc) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-    const cuuint32_t box[2] = {(cuuint32_t)kBox, (cuuint32_t)kBM};
+    const cuuint32_t box[2] = {(cuuint32_t)kBox, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
@@ -683,8 +631,8 @@ fp8vit_status launch(fp8vit_ctx* ctx, const uint8_t* q8, const uint8_t* k8, cons
                      void* out, int32_t out_fp8, const float* out_scale, cudaStream_t st) {
     CUtensorMap mq, mk, mv;
     const int64_t row_bytes = (int64_t)H * D;
-    if (!encode_map(&mq, q8, T, row_bytes) || !encode_map(&mk, k8, T, row_bytes) ||
-        !encode_map(&mv, v8, T, row_bytes))
+    if (!encode_map(&mq, q8, T, row_bytes, kBM) || !encode_map(&mk, k8, T, row_bytes, kBN) ||
+        !encode_map(&mv, v8, T, row_bytes, kBN))
         return FP8VIT_ECUDA;
     static bool attr_set[2] = {false, false};  // per template instance (one device set-up)
     auto kern = attn_fwd_kernel<D>;
