@@ -6,11 +6,12 @@ the current CUDA stream.  The library must be built (``__graft_entry__.build``
 or ``python -m fp8_quantized_vit_b200._build``); there is no fallback.
 
 Entry points (same names as the C ABI):
-  fp8_amax_ring_update, fp8_quantize_qkv_per_tensor, fp8_varlen_attn_fwd,
-  per_token_group_quant_fp8, fp8_static_scales_load, fp8_static_scales_save,
-  fp8_descale_from_amax, fp8_ring_read_amax, ring_init
+  fp8_amax_ring_update, fp8_amax3, fp8_ring_push, fp8_quantize_qkv_per_tensor,
+  fp8_varlen_attn_fwd, per_token_group_quant_fp8, fp8_static_scales_load,
+  fp8_static_scales_save, fp8_descale_from_amax, fp8_ring_read_amax, ring_init
 and ``FP8EncoderAttention``, which chains them for one attention layer
-(dynamic ring or static scales, BF16 or FP8 output, optional group quant).
+(dynamic ring or static scales, BF16 or FP8 output; with a process group, the
+images of one batch split across GPUs, see ``sharding``).
 """
 from __future__ import annotations
 
@@ -37,6 +38,8 @@ _SIGNATURES = {
     "fp8vit_ring_init": (_I32, [_P, _P]),
     "fp8_amax_ring_update": (_I32, [_P, _P, _P, _P, _I64, _P, _P, _P]),
     "fp8_ring_read_amax": (_I32, [_P, _P, _P]),
+    "fp8_amax3": (_I32, [_P, _P, _P, _P, _I64, _P, _P]),
+    "fp8_ring_push": (_I32, [_P, _P, _P, _P]),
     "fp8_quantize_qkv_per_tensor": (_I32, [_P, _P, _P, _P, _I64, _P, _P, _P, _P, _P]),
     "fp8_varlen_attn_fwd": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I64, _I32, _I32,
                                    _F32, _P, _I32, _P, _P]),
@@ -170,6 +173,26 @@ def fp8_amax_ring_update(q, k, v, ring, descale3, ctx=None, stream=None):
     return descale3
 
 
+def fp8_amax3(q, k, v, amax3, ctx=None, stream=None):
+    """amax3[t] = max |x_t| of q, k, v (no ring update)."""
+    n = q.numel()
+    if k.numel() != n or v.numel() != n:
+        raise ValueError("q, k, v must have the same number of elements")
+    _check(lib().fp8_amax3(_ctx(ctx), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+                           _ptr(v, torch.bfloat16, "v"), n, _ptr(amax3, torch.float32, "amax3"),
+                           _stream(stream)), "fp8_amax3")
+    return amax3
+
+
+def fp8_ring_push(amax3, ring, descale3, stream=None):
+    """One forward of the ring rule for the device amax values amax3."""
+    _check(lib().fp8_ring_push(_ptr(amax3, torch.float32, "amax3"),
+                               _ptr(ring, torch.float32, "ring"),
+                               _ptr(descale3, torch.float32, "descale3"), _stream(stream)),
+           "fp8_ring_push")
+    return descale3
+
+
 def fp8_ring_read_amax(ring, stream=None) -> list[float]:
     out = (ctypes.c_float * 3)()
     _check(lib().fp8_ring_read_amax(_ptr(ring, torch.float32, "ring"), out, _stream(stream)),
@@ -261,13 +284,16 @@ class FP8EncoderAttention:
     """
 
     def __init__(self, num_heads: int, head_dim: int, softmax_scale: float | None = None,
-                 static_amax=None, margin: float = 1.5, device=None, ctx: Context | None = None):
+                 static_amax=None, margin: float = 1.5, device=None, ctx: Context | None = None,
+                 process_group=None):
         self.H, self.D = num_heads, head_dim
         self.softmax_scale = (float(torch.tensor(head_dim ** -0.5, dtype=torch.float32))
                               if softmax_scale is None else softmax_scale)
         self.device = torch.device(device or "cuda")
         self.ctx = ctx or default_context()
         self.descale = torch.zeros(3, dtype=torch.float32, device=self.device)
+        self.process_group = process_group
+        self._amax3 = torch.zeros(3, dtype=torch.float32, device=self.device)
         self.ring = None
         if static_amax is None:
             self.ring = new_ring(self.device)
@@ -307,7 +333,14 @@ class FP8EncoderAttention:
         Returns the attention output (BF16, or e4m3 codes if output_scale)."""
         T = q.shape[0]
         b = self._buffers(T, output_scale is not None)
-        if self.ring is not None:
+        if self.ring is not None and self.process_group is not None:
+            # this rank holds some of the batch's images: agree on the
+            # per-tensor amax with the other ranks before the ring update
+            from .sharding import allreduce_amax3
+            fp8_amax3(q, k, v, self._amax3, ctx=self.ctx)
+            allreduce_amax3(self._amax3, self.process_group)
+            fp8_ring_push(self._amax3, self.ring, self.descale)
+        elif self.ring is not None:
             fp8_amax_ring_update(q, k, v, self.ring, self.descale, ctx=self.ctx)
         fp8_quantize_qkv_per_tensor(q, k, v, self.descale, b["q8"], b["k8"], b["v8"],
                                     ctx=self.ctx)

@@ -14,7 +14,7 @@
 
 namespace {
 
-constexpr int kAmaxThreads = 512;
+constexpr int kAmaxThreads = 256;
 constexpr int kQuantThreads = 256;
 constexpr int kGroupThreads = 256;
 
@@ -32,39 +32,42 @@ __device__ __forceinline__ uint32_t absmax_vec(uint32_t acc, const uint4& x) {
     return absmax2(acc, x.w);
 }
 
-__global__ void __launch_bounds__(kAmaxThreads) amax_ring_kernel(
-    const uint4* __restrict__ q, const uint4* __restrict__ k, const uint4* __restrict__ v,
-    int64_t n_elems, fp8vit_ring* __restrict__ ring, float* __restrict__ descale3,
-    fp8vit_scratch* __restrict__ scr) {
+// |x| max of one tensor over this thread's grid-stride share, four 16-byte
+// loads in flight per thread.
+__device__ __forceinline__ uint32_t amax_share(const uint4* __restrict__ p, int64_t n_elems) {
     const int64_t nvec = n_elems >> 3;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const uint4* src[3] = {q, k, v};
-    uint32_t m[3];
-#pragma unroll
-    for (int t = 0; t < 3; ++t) {
-        const uint4* p = src[t];
-        uint32_t a0 = 0, a1 = 0;
-        int64_t i = i0;
-        for (; i + 3 * stride < nvec; i += 4 * stride) {
-            uint4 x0 = __ldcs(p + i);
-            uint4 x1 = __ldcs(p + i + stride);
-            uint4 x2 = __ldcs(p + i + 2 * stride);
-            uint4 x3 = __ldcs(p + i + 3 * stride);
-            a0 = absmax_vec(a0, x0);
-            a1 = absmax_vec(a1, x1);
-            a0 = absmax_vec(a0, x2);
-            a1 = absmax_vec(a1, x3);
-        }
-        for (; i < nvec; i += stride) a0 = absmax_vec(a0, __ldcs(p + i));
-        const int tail = (int)(n_elems & 7);
-        if (blockIdx.x == 0 && (int)threadIdx.x < tail) {
-            const uint16_t* ps = reinterpret_cast<const uint16_t*>(p);
-            a0 = absmax2(a0, ps[(nvec << 3) + threadIdx.x]);
-        }
-        a0 = __vmaxu2(a0, a1);
-        m[t] = max(a0 & 0xFFFFu, a0 >> 16);
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    uint32_t a0 = 0, a1 = 0;
+    for (; i + 3 * stride < nvec; i += 4 * stride) {
+        const uint4 x0 = __ldcs(p + i), x1 = __ldcs(p + i + stride);
+        const uint4 x2 = __ldcs(p + i + 2 * stride), x3 = __ldcs(p + i + 3 * stride);
+        a0 = absmax_vec(absmax_vec(a0, x0), x2);
+        a1 = absmax_vec(absmax_vec(a1, x1), x3);
     }
+    for (; i < nvec; i += stride) a0 = absmax_vec(a0, __ldcs(p + i));
+    const int tail = (int)(n_elems & 7);
+    if (blockIdx.x == 0 && (int)threadIdx.x < tail)
+        a0 = absmax2(a0, reinterpret_cast<const uint16_t*>(p)[(nvec << 3) + threadIdx.x]);
+    a0 = __vmaxu2(a0, a1);
+    return max(a0 & 0xFFFFu, a0 >> 16);
+}
+
+// Four CTAs (1024 threads) per SM with four loads in flight per thread:
+// 64 KB of loads in flight per SM.
+__device__ __forceinline__ void ring_rule(fp8vit_ring* ring, const float (&amax)[3],
+                                       float* descale3);
+
+// ring == nullptr: write the three amaxes (fp32) to out3 instead of running
+// the ring rule (the sharded path all-reduces them first).
+__global__ void __launch_bounds__(kAmaxThreads, 4) amax_ring_kernel(
+    const uint4* __restrict__ q, const uint4* __restrict__ k, const uint4* __restrict__ v,
+    int64_t n_elems, fp8vit_ring* __restrict__ ring, float* __restrict__ out3,
+    fp8vit_scratch* __restrict__ scr) {
+    uint32_t m[3];
+    m[0] = amax_share(q, n_elems);
+    m[1] = amax_share(k, n_elems);
+    m[2] = amax_share(v, n_elems);
     __shared__ uint32_t red[3][kAmaxThreads / 32];
     __shared__ int is_last;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -96,92 +99,136 @@ __global__ void __launch_bounds__(kAmaxThreads) amax_ring_kernel(
 #pragma unroll
     for (int t = 0; t < 3; ++t) amax[t] = bf16_bits_to_f32(atomicExch(&scr->amax_bits[t], 0u));
     atomicExch(&scr->arrivals, 0u);
-    int32_t p = ring->pos;
-    p = ((p % 16) + 16) % 16;
+    if (ring == nullptr) {
 #pragma unroll
-    for (int t = 0; t < 3; ++t) ring->hist[t][p] = amax[t];
-    ring->pos = (p + 1) & 15;
-#pragma unroll
-    for (int t = 0; t < 3; ++t) {
-        float mx = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) mx = ring->hist[t][j] > mx ? ring->hist[t][j] : mx;
-        float d = __fdiv_rn(mx, 448.0f);
-        descale3[t] = d > 1e-10f ? d : 1e-10f;
+        for (int t = 0; t < 3; ++t) out3[t] = amax[t];
+        return;
     }
+    ring_rule(ring, amax, out3);
 }
 
-// 8 bf16 (one 16-byte vector) / scale -> 8 e4m3 codes (8 bytes).
-__device__ __forceinline__ uint2 quant8(const uint4& x, float s) {
+// The 16-slot ring rule for one forward: write the amaxes at pos, advance
+// pos, descale = max(max over the slots / 448, 1e-10) (fp32 division).
+__device__ __forceinline__ void ring_rule(fp8vit_ring* ring, const float (&amax)[3],
+                                       float* descale3) {
+    int32_t p = ring->pos;
+    p = ((p % 16) + 16) % 16;
+#pragma unroll 1
+    for (int t = 0; t < 3; ++t) {
+        ring->hist[t][p] = amax[t];
+        float mx = 0.0f;
+#pragma unroll 1
+        for (int j = 0; j < 16; ++j) mx = ring->hist[t][j] > mx ? ring->hist[t][j] : mx;
+        const float d = __fdiv_rn(mx, 448.0f);
+        descale3[t] = d > 1e-10f ? d : 1e-10f;
+    }
+    ring->pos = (p + 1) & 15;
+}
+
+__global__ void ring_push_kernel(const float* __restrict__ amax3, fp8vit_ring* __restrict__ ring,
+                                 float* __restrict__ descale3) {
+    const float a[3] = {amax3[0], amax3[1], amax3[2]};
+    ring_rule(ring, a, descale3);
+}
+
+// x / s rounded to nearest fp32, given r = RN(1/s) (s > 0, finite).
+// Markstein's correction (IBM J. Res. Dev. 34(1), 1990): with an exactly
+// rounded reciprocal, q0 = RN(x r) is within one ulp of x / s, the
+// remainder x - s q0 is exact in one FMA, and RN(q0 + rem r) is the
+// correctly rounded quotient -- the IEEE division the quantizers are defined
+// with, without a divide per element.  Quotients of magnitude >= 1024
+// saturate to +-448 in e4m3 whatever their last bits, so they skip the
+// correction (which would turn an overflowed q0 into NaN); the sign of a
+// zero quotient is the sign of x.  Checked bit for bit against IEEE division
+// on every finite BF16 value at 96 scales.
+__device__ __forceinline__ float div_by_scale(float x, float s, float r) {
+    const float q0 = __fmul_rn(x, r);
+    const float rem = __fmaf_rn(-q0, s, x);
+    const float q1 = __fmaf_rn(rem, r, q0);
+    return copysignf(fabsf(q0) < 1024.0f ? q1 : q0, x);
+}
+
+// 8 bf16 (one 16-byte vector) / scale -> 8 e4m3 codes (8 bytes); r = RN(1/s).
+__device__ __forceinline__ uint2 quant8(const uint4& x, float s, float r) {
     uint32_t w[4] = {x.x, x.y, x.z, x.w};
     uint32_t c[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        float lo = __fdiv_rn(__uint_as_float(w[i] << 16), s);
-        float hi = __fdiv_rn(__uint_as_float(w[i] & 0xFFFF0000u), s);
+        float lo = div_by_scale(__uint_as_float(w[i] << 16), s, r);
+        float hi = div_by_scale(__uint_as_float(w[i] & 0xFFFF0000u), s, r);
         c[i] = f32x2_to_e4m3x2(lo, hi);
     }
     return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
-__global__ void __launch_bounds__(kQuantThreads) quant3_kernel(
-    const uint4* __restrict__ q, const uint4* __restrict__ k, const uint4* __restrict__ v,
-    int64_t n_elems, const float* __restrict__ descale3, uint2* __restrict__ q8,
-    uint2* __restrict__ k8, uint2* __restrict__ v8) {
+// One tensor's grid-stride share: four 16-byte loads in flight per thread.
+__device__ __forceinline__ void quant_share(const uint4* __restrict__ p, uint2* __restrict__ o,
+                                            int64_t n_elems, float s) {
+    const float r = __frcp_rn(s);
     const int64_t nvec = n_elems >> 3;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const uint4* src[3] = {q, k, v};
-    uint2* dst[3] = {q8, k8, v8};
-#pragma unroll
-    for (int t = 0; t < 3; ++t) {
-        const float s = descale3[t];
-        const uint4* p = src[t];
-        uint2* o = dst[t];
-        int64_t i = i0;
-        for (; i + stride < nvec; i += 2 * stride) {
-            uint4 x0 = __ldcs(p + i);
-            uint4 x1 = __ldcs(p + i + stride);
-            __stcs(o + i, quant8(x0, s));
-            __stcs(o + i + stride, quant8(x1, s));
-        }
-        if (i < nvec) __stcs(o + i, quant8(__ldcs(p + i), s));
-        const int tail = (int)(n_elems & 7);
-        if (blockIdx.x == 0 && (int)threadIdx.x < tail) {
-            const uint16_t* ps = reinterpret_cast<const uint16_t*>(p);
-            uint8_t* os = reinterpret_cast<uint8_t*>(o);
-            const int64_t e = (nvec << 3) + threadIdx.x;
-            float y = __fdiv_rn(bf16_bits_to_f32(ps[e]), s);
-            os[e] = (uint8_t)(f32x2_to_e4m3x2(y, 0.0f) & 0xFF);
-        }
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (; i + 3 * stride < nvec; i += 4 * stride) {
+        const uint4 x0 = __ldcs(p + i), x1 = __ldcs(p + i + stride);
+        const uint4 x2 = __ldcs(p + i + 2 * stride), x3 = __ldcs(p + i + 3 * stride);
+        __stcs(o + i, quant8(x0, s, r));
+        __stcs(o + i + stride, quant8(x1, s, r));
+        __stcs(o + i + 2 * stride, quant8(x2, s, r));
+        __stcs(o + i + 3 * stride, quant8(x3, s, r));
+    }
+    for (; i < nvec; i += stride) __stcs(o + i, quant8(__ldcs(p + i), s, r));
+    const int tail = (int)(n_elems & 7);
+    if (blockIdx.x == 0 && (int)threadIdx.x < tail) {
+        const int64_t e = (nvec << 3) + threadIdx.x;
+        const float y = div_by_scale(bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(p)[e]), s, r);
+        reinterpret_cast<uint8_t*>(o)[e] = (uint8_t)(f32x2_to_e4m3x2(y, 0.0f) & 0xFF);
     }
 }
 
+__global__ void __launch_bounds__(kQuantThreads, 4) quant3_kernel(
+    const uint4* __restrict__ q, const uint4* __restrict__ k, const uint4* __restrict__ v,
+    int64_t n_elems, const float* __restrict__ descale3, uint2* __restrict__ q8,
+    uint2* __restrict__ k8, uint2* __restrict__ v8) {
+    quant_share(q, q8, n_elems, descale3[0]);
+    quant_share(k, k8, n_elems, descale3[1]);
+    quant_share(v, v8, n_elems, descale3[2]);
+}
+
 // LPG = lanes per group = group / 8; each lane owns one 16-byte vector of
-// its group; a warp covers 32 / LPG groups per iteration.
+// its group; a warp covers 32 / LPG groups per step and keeps kUnroll steps
+// (kUnroll loads per lane) in flight.
 template <int LPG>
 __global__ void __launch_bounds__(kGroupThreads) group_quant_kernel(
     const uint4* __restrict__ x, int64_t total_groups, uint2* __restrict__ xq,
     float* __restrict__ scales) {
     constexpr int kGPW = 32 / LPG;
+    constexpr int kUnroll = 4;
     const int lane = threadIdx.x & 31;
     const int sub = lane / LPG, gl = lane % LPG;
     const int64_t warp_id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t g0 = warp_id * kGPW; g0 < total_groups; g0 += nwarps * kGPW) {
-        const int64_t g = g0 + sub;
-        const bool valid = g < total_groups;
-        uint4 xv = valid ? __ldcs(x + g * LPG + gl) : make_uint4(0, 0, 0, 0);
-        uint32_t a = absmax_vec(0u, xv);
-        a = max(a & 0xFFFFu, a >> 16);
+    for (int64_t g0 = warp_id * kGPW * kUnroll; g0 < total_groups;
+         g0 += nwarps * kGPW * kUnroll) {
+        uint4 xv[kUnroll];
 #pragma unroll
-        for (int off = LPG / 2; off > 0; off >>= 1)
-            a = max(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
-        float s = __fdiv_rn(bf16_bits_to_f32(a), 448.0f);
-        s = s > 1e-10f ? s : 1e-10f;
-        if (valid) {
-            __stcs(xq + g * LPG + gl, quant8(xv, s));
-            if (gl == 0) scales[g] = s;
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t g = g0 + u * kGPW + sub;
+            xv[u] = g < total_groups ? __ldcs(x + g * LPG + gl) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t g = g0 + u * kGPW + sub;
+            uint32_t a = absmax_vec(0u, xv[u]);
+            a = max(a & 0xFFFFu, a >> 16);
+#pragma unroll
+            for (int off = LPG / 2; off > 0; off >>= 1)
+                a = max(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+            float sc = __fdiv_rn(bf16_bits_to_f32(a), 448.0f);
+            sc = sc > 1e-10f ? sc : 1e-10f;
+            if (g < total_groups) {
+                __stcs(xq + g * LPG + gl, quant8(xv[u], sc, __frcp_rn(sc)));
+                if (gl == 0) scales[g] = sc;
+            }
         }
     }
 }
@@ -214,6 +261,29 @@ fp8vit_status fp8_amax_ring_update(fp8vit_ctx* ctx, const uint16_t* d_q, const u
         reinterpret_cast<const uint4*>(d_q), reinterpret_cast<const uint4*>(d_k),
         reinterpret_cast<const uint4*>(d_v), n_elems, reinterpret_cast<fp8vit_ring*>(d_ring),
         d_descale3, ctx->d_scratch);
+    return cudaGetLastError() == cudaSuccess ? FP8VIT_OK : FP8VIT_ECUDA;
+}
+
+fp8vit_status fp8_amax3(fp8vit_ctx* ctx, const uint16_t* d_q, const uint16_t* d_k,
+                        const uint16_t* d_v, int64_t n_elems, float* d_amax3, void* stream) {
+    if (!ctx || !d_q || !d_k || !d_v || !d_amax3 || n_elems < 0) return FP8VIT_EINVAL;
+    if (misaligned(d_q, 16) || misaligned(d_k, 16) || misaligned(d_v, 16) ||
+        misaligned(d_amax3, 4))
+        return FP8VIT_EINVAL;
+    const int grid = grid_for(n_elems >> 3, kAmaxThreads, 8, 4 * ctx->num_sms);
+    amax_ring_kernel<<<grid, kAmaxThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const uint4*>(d_q), reinterpret_cast<const uint4*>(d_k),
+        reinterpret_cast<const uint4*>(d_v), n_elems, nullptr, d_amax3, ctx->d_scratch);
+    return cudaGetLastError() == cudaSuccess ? FP8VIT_OK : FP8VIT_ECUDA;
+}
+
+fp8vit_status fp8_ring_push(const float* d_amax3, void* d_ring, float* d_descale3,
+                            void* stream) {
+    if (!d_amax3 || !d_ring || !d_descale3) return FP8VIT_EINVAL;
+    if (misaligned(d_ring, 16) || misaligned(d_amax3, 4) || misaligned(d_descale3, 4))
+        return FP8VIT_EINVAL;
+    ring_push_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        d_amax3, reinterpret_cast<fp8vit_ring*>(d_ring), d_descale3);
     return cudaGetLastError() == cudaSuccess ? FP8VIT_OK : FP8VIT_ECUDA;
 }
 

@@ -100,6 +100,21 @@ fp8vit_status fp8_amax_ring_update(fp8vit_ctx* ctx, const uint16_t* d_q, const u
                                    const uint16_t* d_v, int64_t n_elems, void* d_ring,
                                    float* d_descale3, void* stream);
 
+/* The two halves of fp8_amax_ring_update, for a packed batch split across
+ * GPUs (each GPU holds some of the images): every rank runs fp8_amax3 on its
+ * share, the ranks all-reduce the three values with max (e.g. NCCL), and each
+ * runs fp8_ring_push with the result, so all ranks quantize with the same
+ * per-tensor descales.  fp8_amax3 followed by fp8_ring_push on one GPU gives
+ * bit for bit what fp8_amax_ring_update gives.
+ *   fp8_amax3: d_amax3[t] = max |x_t| over n_elems BF16 elements (fp32,
+ *     exact), t = q, k, v.  Same argument rules as fp8_amax_ring_update.
+ *   fp8_ring_push: the ring rule of fp8_amax_ring_update applied to the
+ *     three device values d_amax3 (one thread; writes d_ring and d_descale3). */
+fp8vit_status fp8_amax3(fp8vit_ctx* ctx, const uint16_t* d_q, const uint16_t* d_k,
+                        const uint16_t* d_v, int64_t n_elems, float* d_amax3, void* stream);
+fp8vit_status fp8_ring_push(const float* d_amax3, void* d_ring, float* d_descale3,
+                            void* stream);
+
 /* Same computation and arguments as fp8_amax_ring_update, for callers that
  * cannot allocate device memory where they run (for example a process whose
  * memory pool already holds nearly all free HBM, code that must avoid

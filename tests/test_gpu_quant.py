@@ -155,3 +155,48 @@ def test_group_quant_other_group_sizes(ctx, group):
     _check_ok(ctx)
     assert (_host_u8(xq) == want_q).all()
     assert (_f32_bits(sc.cpu().numpy()) == _f32_bits(want_s)).all()
+
+
+def test_amax3_then_ring_push_equals_fused_update(ctx):
+    """The split path used when one batch is spread over several GPUs
+    (amax, all-reduce, ring push) gives the fused update's bits on one GPU."""
+    w = synth.WORKLOADS["c2"]
+    ring_a, ring_b = fv.new_ring(), fv.new_ring()
+    da = torch.zeros(3, dtype=torch.float32, device="cuda")
+    db = torch.zeros(3, dtype=torch.float32, device="cuda")
+    amax3 = torch.zeros(3, dtype=torch.float32, device="cuda")
+    for f in range(18):
+        x = [synth.bf16_tensor(synth.stream_key(700 + f, f, t), 512, 2048) for t in range(3)]
+        dev = [_dev_bf16(a) for a in x]
+        fv.fp8_amax_ring_update(*dev, ring_a, da, ctx=ctx)
+        fv.fp8_amax3(*dev, amax3, ctx=ctx)
+        assert (_f32_bits(amax3.cpu().numpy()) ==
+                _f32_bits([oracle.amax_bf16(a) for a in x])).all()
+        fv.fp8_ring_push(amax3, ring_b, db)
+        assert (_f32_bits(da.cpu().numpy()) == _f32_bits(db.cpu().numpy())).all(), f
+        assert (_f32_bits(ring_a.cpu().numpy()) == _f32_bits(ring_b.cpu().numpy())).all(), f
+    _check_ok(ctx)
+
+
+def _descale_set(n_random: int = 80):
+    """Descales that stress the division: the 1e-10 floor, powers of two,
+    fp32 values with all-ones mantissas, 448-related values, random ones."""
+    f = [1e-10, 2.0 ** -30, 2.0 ** -9, 2.0 ** -1, 1.0, 2.0, 2.0 ** 20,
+         np.nextafter(np.float32(1.0), np.float32(0)), np.nextafter(np.float32(2.0), np.float32(0)),
+         np.float32(1.0) / np.float32(448.0), np.float32(1.5) / np.float32(448.0),
+         np.float32(3.0) / np.float32(7.0), np.float32(0.1), np.float32(1e-3), 0.013671875,
+         np.float32(123.456)]
+    rng = np.random.default_rng(2025)
+    amax = np.exp(rng.uniform(np.log(1e-4), np.log(1e4), n_random)).astype(np.float32)
+    f += list(amax / np.float32(448.0))
+    return [float(np.float32(v)) for v in f]
+
+
+def test_quantize_every_bf16_value(ctx):
+    """Every finite BF16 value through the per-tensor quantizer at 96
+    descales, bit for bit against the oracle's IEEE fp32 division."""
+    allb = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    x = allb[(allb & 0x7F80) != 0x7F80]          # drop inf and NaN patterns
+    x = np.concatenate([x, x[: (-x.size) % 8]])   # multiple of 8
+    for d in _descale_set():
+        _quant_case(ctx, x, x[::-1].copy(), x, [d, d, d])
