@@ -385,7 +385,7 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3 (fp32 accumulate)",
         "data": "synthetic", "config": _config(w, n_fwd),
-        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>",
+        "roofline": {"bound": "tensor", "kernel": f"attn_fwd_kernel<{D}>",
                      "achieved": attn_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
                      "frac": attn_tflops / fp8_peak, "traffic": traffic,
                      "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16']} x 2 (fp8/bf16)",

@@ -161,48 +161,46 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float&
     y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
-__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-// Two 16-bit halves into one word (lo in bits 0..15).
-__device__ __forceinline__ uint32_t pack_h2(uint16_t lo, uint16_t hi) {
+// f32 pair -> f16x2 (lo in bits 0..15)
+__device__ __forceinline__ uint32_t cvt_f16x2(float lo, float hi) {
     uint32_t d;
-    asm("mov.b32 %0, {%1, %2};" : "=r"(d) : "h"(lo), "h"(hi));
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+// f16x2 -> two e4m3 codes in bits 0..15 (RNE, satfinite; bits 0..15 of the
+// source -> byte 0), returned zero-extended
+__device__ __forceinline__ uint32_t e4m3x2_of_f16x2(uint32_t h) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(d) : "r"(h));
+    return d;
+}
+// two e4m3 codes (bits 0..15) -> f16x2 (exact)
+__device__ __forceinline__ uint32_t f16x2_of_e4m3x2(uint32_t e) {
+    uint32_t d;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"((uint16_t)e));
+    return d;
+}
+__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
 }
 
 // Split 4 probabilities into one hi word and one lo word of e4m3 codes,
 // hi + lo ~= p with ~8 significant bits, so that the PV product on FP8
-// tensor cores keeps about a BF16-width P.  Veltkamp's splitting (Dekker,
-// "A floating-point technique for extending the available precision", 1971)
-// with factor 2^20 + 1 cuts each fp32 p into h (4 significant bits, exactly
-// an e4m3 value in the normal range) and the exact remainder p - h; the
-// remainder is then rounded to e4m3.  The split runs on the FMA pipe
-// (packed f32x2); only the two e4m3 conversions per pair use the ALU.
-// t = c - p is formed as fma(p, -1, c): written as a subtraction, the code
-// generator folds c - (c - p) back into p and the remainder vanishes.
+// tensor cores keeps about a BF16-width P.  p is rounded to f16 (11 bits);
+// hi = e4m3(p16); the residual p16 - hi is exact in f16 (both share the
+// exponent range of p16); lo = e4m3(residual).  Five conversions/subtracts
+// per pair.  The words are combined from zero-extended halves with shifts
+// (packing two 16-bit asm results with mov.b32 {a, b} was miscompiled here).
 __device__ __forceinline__ void p_split4(float p0, float p1, float p2, float p3, uint32_t& hi,
                                          uint32_t& lo) {
-    const uint64_t k = f2pack(1048577.0f, 1048577.0f);
-    const uint64_t m1 = f2pack(-1.0f, -1.0f);
-    const uint64_t a = f2pack(p0, p1), b = f2pack(p2, p3);
-    const uint64_t ca = fmul2(a, k), cb = fmul2(b, k);
-    const uint64_t ha = fsub2(ca, ffma2(a, m1, ca)), hb = fsub2(cb, ffma2(b, m1, cb));
-    const uint64_t la = fsub2(a, ha), lb = fsub2(b, hb);
-    float h0, h1, h2, h3, l0, l1, l2, l3;
-    f2unpack(ha, h0, h1);
-    f2unpack(hb, h2, h3);
-    f2unpack(la, l0, l1);
-    f2unpack(lb, l2, l3);
-    hi = pack_h2(f32x2_to_e4m3x2(h0, h1), f32x2_to_e4m3x2(h2, h3));
-    lo = pack_h2(f32x2_to_e4m3x2(l0, l1), f32x2_to_e4m3x2(l2, l3));
+    const uint32_t h01 = cvt_f16x2(p0, p1), h23 = cvt_f16x2(p2, p3);
+    const uint32_t e01 = e4m3x2_of_f16x2(h01), e23 = e4m3x2_of_f16x2(h23);
+    const uint32_t l01 = e4m3x2_of_f16x2(hsub2(h01, f16x2_of_e4m3x2(e01)));
+    const uint32_t l23 = e4m3x2_of_f16x2(hsub2(h23, f16x2_of_e4m3x2(e23)));
+    hi = e01 | (e23 << 16);
+    lo = l01 | (l23 << 16);
 }
 
 #ifndef FP8VIT_POLY_EVERY
