@@ -7,15 +7,18 @@
 //   warp 0      TMA producer: Q once, then K/V tiles of 64 keys into an
 //               NS-stage shared-memory ring (SWIZZLE_32B, 32-byte boxes).
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer:
-//               S = Q K^T (kind::f8f6f4, K-major A and B) into one of two
-//               TMEM S buffers, O += P V (A = P from TMEM, B = V MN-major
-//               from smem).  The next tile's S is computed while the softmax
-//               warps work on the current one.
+//               S = Q K^T (kind::f8f6f4, K-major A and B) into the TMEM S
+//               buffer, O += P V (A = P from TMEM, B = V MN-major from
+//               smem).  S(j+1) is issued as soon as the softmax warps have
+//               copied S(j) into registers, so it is computed while they
+//               work on tile j; P has two TMEM slots of its own, so the next
+//               QK never waits for the previous PV.
 //   warps 2..5  softmax + epilogue, one query row per thread (TMEM lane):
-//               row max, exp2, row sum in registers; P written back to TMEM
-//               as two e4m3 terms (hi + lo) so that the PV product keeps
-//               ~8 mantissa bits while running on FP8 tensor cores; O is
-//               rescaled in TMEM when the row max rises.
+//               row max, exp2, row sum in registers; P written to its TMEM
+//               slot as two e4m3 terms (hi + lo) so that the PV product
+//               keeps ~8 mantissa bits while running on FP8 tensor cores; O
+//               is rescaled in TMEM when the row max rises (after P is
+//               written, when the previous PV has long completed).
 // head_dim 72 is padded inside the kernel: the QK contraction runs over 96
 // bytes starting at the head's offset rounded down to 16 bytes (TMA needs a
 // 16-byte aligned x coordinate); bytes of the window outside the head are
@@ -31,7 +34,8 @@ constexpr int kBM = 128;          // query rows per CTA (MMA M)
 constexpr int kBN = 64;           // keys per KV tile (QK MMA N, PV MMA K)
 constexpr int kThreads = 192;     // 6 warps
 constexpr int kTmemCols = 256;
-constexpr uint32_t kTmemS = 0;    // S buffers: columns [0,64) and [64,128); P over [64b, 64b+32)
+constexpr uint32_t kTmemS = 0;    // S buffer: columns [0, 64)
+constexpr uint32_t kTmemP = 64;   // P slots: columns [64 + 32b, 96 + 32b), b = tile parity
 constexpr uint32_t kTmemO = 128;  // O accumulator columns [128, 128 + NPV)
 constexpr int kBox = 32;          // bytes per TMA box row (one SW32 atom row)
 constexpr int kQTileBytes = kBox * kBM;   // one [128 rows x 32 B] Q box
@@ -106,6 +110,49 @@ __device__ __forceinline__ void tmem_ld64_sync(uint32_t taddr, uint32_t (&a)[32]
         : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]), "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15]), "=r"(a[16]), "=r"(a[17]), "=r"(a[18]), "=r"(a[19]), "=r"(a[20]), "=r"(a[21]), "=r"(a[22]), "=r"(a[23]), "=r"(a[24]), "=r"(a[25]), "=r"(a[26]), "=r"(a[27]), "=r"(a[28]), "=r"(a[29]), "=r"(a[30]), "=r"(a[31]), "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7]), "=r"(b[8]), "=r"(b[9]), "=r"(b[10]), "=r"(b[11]), "=r"(b[12]), "=r"(b[13]), "=r"(b[14]), "=r"(b[15]), "=r"(b[16]), "=r"(b[17]), "=r"(b[18]), "=r"(b[19]), "=r"(b[20]), "=r"(b[21]), "=r"(b[22]), "=r"(b[23]), "=r"(b[24]), "=r"(b[25]), "=r"(b[26]), "=r"(b[27]), "=r"(b[28]), "=r"(b[29]), "=r"(b[30]), "=r"(b[31])
         : "r"(taddr)
         : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+        "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+// O *= alpha over columns [0, NPV) of this thread's lane, in 32-column steps
+// (one load wait per step); NPV = 80 ends with two 8-column pieces.
+template <int NPV>
+__device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
+#pragma unroll
+    for (int c = 0; c + 32 <= NPV; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(tO + c, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+        tmem_st32(tO + c, r);
+    }
+    if constexpr (NPV % 32 != 0) {
+        static_assert(NPV % 32 == 16, "O tail is one 16-column piece");
+        constexpr int c = NPV - 16;
+        uint32_t r[8], s[8];
+        tmem_ld8(tO + c, r);
+        tmem_ld8(tO + c + 8, s);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            s[i] = __float_as_uint(__uint_as_float(s[i]) * alpha);
+        }
+        tmem_st8(tO + c, r);
+        tmem_st8(tO + c + 8, s);
+    }
 }
 
 // ---- packed arithmetic used by the softmax --------------------------------
@@ -267,9 +314,9 @@ __device__ __forceinline__ void p_chunk(const uint32_t (&r)[32], int key0, int n
         p_split4(p[4 * w], p[4 * w + 1], p[4 * w + 2], p[4 * w + 3], pk[w], pk[8 + w]);
 }
 
-// P of one 64-key tile written over the first 32 columns of its S buffer:
-// chunk c (keys 32c..32c+31) goes to columns [16c, 16c+8) (hi) and
-// [16c+8, 16c+16) (lo).  Returns the tile's probability sum.
+// P of one 64-key tile written to a 32-column P slot: chunk c (keys
+// 32c..32c+31) goes to columns [16c, 16c+8) (hi) and [16c+8, 16c+16) (lo).
+// Returns the tile's probability sum.
 template <bool FULL>
 __device__ __forceinline__ float tile_p(const uint32_t (&a)[32], const uint32_t (&b)[32],
                                         uint32_t tSb, int nvalid, uint64_t c2, uint64_t nb2) {
@@ -319,33 +366,37 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t sV = smem_u32(sm + L::V);
     const uint32_t bar0 = smem_u32(sm + L::BAR);
     // barrier indices
-    // Barriers of per-tile events come in pairs indexed by the tile's parity
-    // (b = j & 1), so that a waiter is never more than one phase behind the
-    // phase it waits for: tile j's event is completion (j >> 1) of barrier b.
+    // s_full / s_free complete once per tile (phase j & 1): S(j+1) is only
+    // issued after s_free(j), which the softmax warps arrive on after
+    // waiting for s_full(j), so neither can run two phases ahead of its
+    // waiter.  P and PV events come in pairs indexed by the tile's parity
+    // (b = j & 1), tile j's event being completion (j >> 1) of barrier b:
+    // a waiter for tile j - 1 or j - 2 can never see that barrier two
+    // phases ahead, because PV(j) needs P(j), which the waiter writes later.
     const uint32_t b_q_full = bar0 + 8 * 0;
     const uint32_t b_q_ready = bar0 + 8 * 1;
     const uint32_t b_drain = bar0 + 8 * 2;
-    auto b_s_full = [&](int b) { return bar0 + 8 * (3 + b); };   // S(j) computed
+    const uint32_t b_s_full = bar0 + 8 * 3;                      // S(j) computed
+    const uint32_t b_s_free = bar0 + 8 * 4;                      // S(j) copied to registers
     auto b_p_full = [&](int b) { return bar0 + 8 * (5 + b); };   // P(j) written
     auto b_o_ready = [&](int b) { return bar0 + 8 * (7 + b); };  // PV(j) complete
-    auto b_k_full = [&](int s) { return bar0 + 8 * (9 + s); };
-    auto b_v_full = [&](int s) { return bar0 + 8 * (9 + NS + s); };
-    auto b_kv_empty = [&](int s) { return bar0 + 8 * (9 + 2 * NS + s); };
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::BAR + 8 * (9 + 3 * NS));
+    auto b_kv_full = [&](int s) { return bar0 + 8 * (9 + s); };  // K and V of a stage landed
+    auto b_kv_empty = [&](int s) { return bar0 + 8 * (9 + NS + s); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::BAR + 8 * (9 + 2 * NS));
     volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
 
     if (threadIdx.x == 0) {
         mbar_init(b_q_full, 1);
         mbar_init(b_q_ready, 128);
         mbar_init(b_drain, 1);
+        mbar_init(b_s_full, 1);
+        mbar_init(b_s_free, 128);
         for (int b = 0; b < 2; ++b) {
-            mbar_init(b_s_full(b), 1);
             mbar_init(b_p_full(b), 128);
             mbar_init(b_o_ready(b), 1);
         }
         for (int s = 0; s < NS; ++s) {
-            mbar_init(b_k_full(s), 1);
-            mbar_init(b_v_full(s), 1);
+            mbar_init(b_kv_full(s), 1);
             mbar_init(b_kv_empty(s), 1);
         }
         *abort_flag = 0;
@@ -382,51 +433,48 @@ __global__ void __launch_bounds__(kThreads, 2)
                                        SITE_ATTN_WAIT_EMPTY, kTimeoutNs))
                     break;
                 const int32_t row = seg_start + j * kBN;
-                mbar_arrive_expect_tx(b_k_full(s), C::KB * kKVTileBytes);
+                mbar_arrive_expect_tx(b_kv_full(s), (C::KB + C::VA) * kKVTileBytes);
                 for (int kb = 0; kb < C::KB; ++kb)
                     tma_load_2d(sK + (s * C::KB + kb) * kKVTileBytes, &tm_k, x0 + kBox * kb, row,
-                                b_k_full(s));
-                mbar_arrive_expect_tx(b_v_full(s), C::VA * kKVTileBytes);
+                                b_kv_full(s));
                 for (int a = 0; a < C::VA; ++a)
                     tma_load_2d(sV + (s * C::VA + a) * kKVTileBytes, &tm_v, x0 + kBox * a, row,
-                                b_v_full(s));
+                                b_kv_full(s));
                 ++issued;
             }
             // Drain: every issued copy must land before the CTA may exit.
             mbar_wait_bounded(b_q_full, 0, abort_flag, scr, SITE_ATTN_DRAIN, kTimeoutNs);
             for (int j = issued - 1; j >= 0 && j >= issued - NS; --j) {
                 const int s = j % NS;
-                mbar_wait_bounded(b_k_full(s), (j / NS) & 1, abort_flag, scr, SITE_ATTN_DRAIN,
-                                  kTimeoutNs);
-                mbar_wait_bounded(b_v_full(s), (j / NS) & 1, abort_flag, scr, SITE_ATTN_DRAIN,
+                mbar_wait_bounded(b_kv_full(s), (j / NS) & 1, abort_flag, scr, SITE_ATTN_DRAIN,
                                   kTimeoutNs);
             }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
-        // S(j) = Q K_j^T goes to S buffer j & 1.  S(j+1) is issued before P(j)
-        // is waited for, so the tensor cores compute the next scores while
-        // the softmax warps work on the current ones; the buffer it reuses
-        // held P(j-1), so PV(j-1) must have completed first.
+        // S(j) = Q K_j^T goes to the S buffer.  S(j+1) is issued as soon as
+        // the softmax warps have copied S(j) into registers (s_free), before
+        // P(j) is waited for, so the tensor cores compute the next scores
+        // while the softmax warps work on the current ones.
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_e4m3(kBN, false);
             constexpr uint32_t idesc_pv = idesc_e4m3(C::NPV, true);
             const uint32_t tO = tmem + kTmemO;
             auto issue_qk = [&](int j) {
                 const int s = j % NS;
-                const uint32_t tSb = tmem + kTmemS + 64 * (j & 1);
+                const uint32_t tSb = tmem + kTmemS;
 #pragma unroll
                 for (int kb = 0; kb < C::KB; ++kb)
                     umma_f8_ss(tSb, desc_k_sw32(sQ + kb * kQTileBytes),
                                desc_k_sw32(sK + (s * C::KB + kb) * kKVTileBytes), idesc_qk,
                                kb > 0 ? 1u : 0u);
-                umma_commit(b_s_full(j & 1));
+                umma_commit(b_s_full);
             };
             bool ok = mbar_wait_bounded(b_q_ready, 0, abort_flag, scr, SITE_ATTN_WAIT_QREADY,
                                         kTimeoutNs);
             bool issued_any = false;
             if (ok) {
-                ok = mbar_wait_bounded(b_k_full(0), 0, abort_flag, scr, SITE_ATTN_WAIT_K,
+                ok = mbar_wait_bounded(b_kv_full(0), 0, abort_flag, scr, SITE_ATTN_WAIT_K,
                                        kTimeoutNs);
                 if (ok) {
                     tc_fence_after();
@@ -437,25 +485,22 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int j = 0; ok && j < n_kv; ++j) {
                 if (j + 1 < n_kv) {
                     const int s1 = (j + 1) % NS;
-                    if (!mbar_wait_bounded(b_k_full(s1), ((j + 1) / NS) & 1, abort_flag, scr,
+                    if (!mbar_wait_bounded(b_kv_full(s1), ((j + 1) / NS) & 1, abort_flag, scr,
                                            SITE_ATTN_WAIT_K, kTimeoutNs))
                         break;
-                    if (j >= 1 && !mbar_wait_bounded(b_o_ready((j - 1) & 1), ((j - 1) >> 1) & 1,
-                                                     abort_flag, scr, SITE_ATTN_WAIT_O,
-                                                     kTimeoutNs))
+                    if (!mbar_wait_bounded(b_s_free, j & 1, abort_flag, scr, SITE_ATTN_WAIT_SFREE,
+                                           kTimeoutNs))
                         break;
                     tc_fence_after();
                     issue_qk(j + 1);
                 }
+                // V(j) landed with K(j), which QK(j) waited for.
                 const int s = j % NS;
-                if (!mbar_wait_bounded(b_v_full(s), (j / NS) & 1, abort_flag, scr,
-                                       SITE_ATTN_WAIT_V, kTimeoutNs))
-                    break;
                 if (!mbar_wait_bounded(b_p_full(j & 1), (j >> 1) & 1, abort_flag, scr,
                                        SITE_ATTN_WAIT_P, kTimeoutNs))
                     break;
                 tc_fence_after();
-                const uint32_t tPb = tmem + kTmemS + 64 * (j & 1);
+                const uint32_t tPb = tmem + kTmemP + 32 * (j & 1);
                 const uint32_t vbase = sV + s * C::VA * kKVTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < kBN / 32; ++kk) {
@@ -477,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;  // query row in the tile == TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-        const uint32_t tS = lane_base + kTmemS, tO = lane_base + kTmemO;
+        const uint32_t tS = lane_base + kTmemS, tP = lane_base + kTmemP, tO = lane_base + kTmemO;
         const float dq = *dq_p, dk = *dk_p, dv = *dv_p;
         const float scale_log2 = sm_scale * dq * dk * 1.4426950408889634f;
 
@@ -507,52 +552,47 @@ __global__ void __launch_bounds__(kThreads, 2)
         // tile's max exceeds m_ref by more than kSlackLog2 (both are scaled
         // by the same factor, so the final o = O / l is unchanged).
         float m_ref = -INFINITY, l_run = 0.0f;
+        const uint32_t tSb = tS;
         for (int j = 0; ok && j < n_kv; ++j) {
             const int b = j & 1;
-            ok = mbar_wait_bounded(b_s_full(b), (j >> 1) & 1, abort_flag, scr, SITE_ATTN_WAIT_S,
-                                   kTimeoutNs);
+            ok = mbar_wait_bounded(b_s_full, j & 1, abort_flag, scr, SITE_ATTN_WAIT_S, kTimeoutNs);
             ok = __all_sync(0xFFFFFFFFu, ok);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t tSb = tS + 64 * b;
             const int nvalid = min(kBN, seg_len - j * kBN);
             const bool full = nvalid == kBN;
             uint32_t ra[32], rb[32];
             tmem_ld64_sync(tSb, ra, rb);
+            tc_fence_before();
+            mbar_arrive(b_s_free);  // the S buffer may take S(j+1) now
             const float mx =
                 full ? tile_row_max<true>(ra, rb, nvalid) : tile_row_max<false>(ra, rb, nvalid);
             const float mxc = mx * scale_log2;
-            if (j == 0) {
-                m_ref = mxc;  // the first PV initialises O, nothing to rescale
-            } else {
-                const bool need = mxc > m_ref + kSlackLog2;
-                if (__any_sync(0xFFFFFFFFu, need)) {
-                    ok = mbar_wait_bounded(b_o_ready((j - 1) & 1), ((j - 1) >> 1) & 1,
-                                           abort_flag, scr, SITE_ATTN_WAIT_O, kTimeoutNs);
-                    ok = __all_sync(0xFFFFFFFFu, ok);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const float alpha = need ? ex2_approx(m_ref - mxc) : 1.0f;
-#pragma unroll
-                    for (int c = 0; c < C::NPV / 8; ++c) {
-                        uint32_t r[8];
-                        tmem_ld8_sync(tO + 8 * c, r);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                        tmem_st8(tO + 8 * c, r);
-                    }
-                    tmem_wait_st();
-                    l_run *= alpha;
-                    if (need) m_ref = mxc;
-                }
-            }
+            // j == 0 sets the reference; the first PV initialises O.
+            const bool need = j == 0 || mxc > m_ref + kSlackLog2;
+            const bool rescale = j > 0 && __any_sync(0xFFFFFFFFu, need);
+            const float alpha = (j > 0 && need) ? ex2_approx(m_ref - mxc) : 1.0f;
+            if (need) m_ref = mxc;
+            // P slot b held P(j - 2).  PV(j - 2) was issued before QK(j), and
+            // the commit that completed s_full(j) tracks every earlier MMA of
+            // the issuer, so PV(j - 2) has completed: the slot is free.
             // P = 2^(x - bias), bias = m_ref - kPLog2
             const float bias = m_ref - kPLog2;
             const uint64_t c2 = f2pack(scale_log2, scale_log2);
             const uint64_t nb2 = f2pack(-bias, -bias);
-            l_run += full ? tile_p<true>(ra, rb, tSb, nvalid, c2, nb2)
-                          : tile_p<false>(ra, rb, tSb, nvalid, c2, nb2);
+            const uint32_t tPb = tP + 32 * b;
+            const float tile_sum = full ? tile_p<true>(ra, rb, tPb, nvalid, c2, nb2)
+                                        : tile_p<false>(ra, rb, tPb, nvalid, c2, nb2);
+            l_run = l_run * alpha + tile_sum;
+            if (rescale) {
+                // O holds PV(0..j-1): wait for PV(j - 1), then scale it.
+                ok = mbar_wait_bounded(b_o_ready((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag,
+                                       scr, SITE_ATTN_WAIT_O, kTimeoutNs);
+                ok = __all_sync(0xFFFFFFFFu, ok);
+                if (!ok) break;
+                tc_fence_after();
+                rescale_o<C::NPV>(tO, alpha);
+            }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(b_p_full(b));

@@ -52,6 +52,7 @@ enum : int32_t {
     SITE_ATTN_WAIT_EMPTY = 116,
     SITE_ATTN_WAIT_QREADY = 117,
     SITE_ATTN_DRAIN = 118,
+    SITE_ATTN_WAIT_SFREE = 119,
 };
 
 __device__ __forceinline__ void fp8vit_report(fp8vit_scratch* s, int32_t status, int32_t site) {
