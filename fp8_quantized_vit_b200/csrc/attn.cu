@@ -155,6 +155,14 @@ __device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
     }
 }
 
+// One arrival per warp: every lane's prior memory and tcgen05 operations
+// (each lane has executed its own fences) are ordered before lane 0's arrive
+// by the warp barrier.
+__device__ __forceinline__ void warp_arrive(uint32_t bar, int lane) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar);
+}
+
 // ---- packed arithmetic used by the softmax --------------------------------
 
 __device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
@@ -180,34 +188,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
 }
-// 2^x on the FMA pipe for a pair of arguments (x >= -126 after the clamp).
-// Cody-Waite reduction x = n + f, n = rint(x) via the 1.5 * 2^23 magic add,
-// f in [-0.5, 0.5]; 2^f by a degree-3 polynomial fitted for minimal relative
-// error on [-0.5, 0.5] (fit_exp2.py: max relative error 7.5e-5); 2^n is
-// added into the exponent field with an integer add.  Used for a fixed share
-// of the elements so that the MUFU pipe (ex2.approx) is not the only source
-// of exponentials.
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
-    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-    x0 = fmaxf(x0, -126.0f);
-    x1 = fmaxf(x1, -126.0f);
-    const uint64_t t = fadd2(f2pack(x0, x1), f2pack(kMagic, kMagic));
-    float t0, t1;
-    f2unpack(t, t0, t1);
-    float n0, n1;
-    f2unpack(fadd2(t, f2pack(-kMagic, -kMagic)), n0, n1);
-    const uint64_t f = fadd2(f2pack(x0, x1), f2pack(-n0, -n1));
-    uint64_t p = ffma2(f, f2pack(0.0551716685295105f, 0.0551716685295105f),
-                       f2pack(0.2426111251115799f, 0.2426111251115799f));
-    p = ffma2(f, p, f2pack(0.6932609677314758f, 0.6932609677314758f));
-    p = ffma2(f, p, f2pack(0.9999280571937561f, 0.9999280571937561f));
-    float p0, p1;
-    f2unpack(p, p0, p1);
-    // the low bits of t hold n (two's complement); shift them into the exponent
-    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
-
 // f32 pair -> f16x2 (lo in bits 0..15)
 __device__ __forceinline__ uint32_t cvt_f16x2(float lo, float hi) {
     uint32_t d;
@@ -250,60 +230,33 @@ __device__ __forceinline__ void p_split4(float p0, float p1, float p2, float p3,
     lo = l01 | (l23 << 16);
 }
 
-#ifndef FP8VIT_POLY_EVERY
-#define FP8VIT_POLY_EVERY 0
-#endif
-
 // Row max of one 64-key S tile held in registers (a = keys 0..31, b = keys
-// 32..63); only the first `nvalid` keys count when !FULL.
-template <bool FULL>
-__device__ __forceinline__ float tile_row_max(const uint32_t (&a)[32], const uint32_t (&b)[32],
-                                              int nvalid) {
-    if (FULL) {
-        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+// 32..63); keys past the segment end already hold -inf.
+__device__ __forceinline__ float tile_row_max(const uint32_t (&a)[32], const uint32_t (&b)[32]) {
+    float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-            m0 = fmax3(m0, __uint_as_float(a[i]), __uint_as_float(a[i + 1]));
-            m1 = fmax3(m1, __uint_as_float(a[i + 2]), __uint_as_float(a[i + 3]));
-            m2 = fmax3(m2, __uint_as_float(b[i]), __uint_as_float(b[i + 1]));
-            m3 = fmax3(m3, __uint_as_float(b[i + 2]), __uint_as_float(b[i + 3]));
-        }
-        return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+    for (int i = 0; i < 32; i += 4) {
+        m0 = fmax3(m0, __uint_as_float(a[i]), __uint_as_float(a[i + 1]));
+        m1 = fmax3(m1, __uint_as_float(a[i + 2]), __uint_as_float(a[i + 3]));
+        m2 = fmax3(m2, __uint_as_float(b[i]), __uint_as_float(b[i + 1]));
+        m3 = fmax3(m3, __uint_as_float(b[i + 2]), __uint_as_float(b[i + 3]));
     }
-    float m = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        if (i < nvalid) m = fmaxf(m, __uint_as_float(a[i]));
-        if (32 + i < nvalid) m = fmaxf(m, __uint_as_float(b[i]));
-    }
-    return m;
+    return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
 }
 
-// Probabilities of one 32-key chunk: p = 2^(s * c - bias), summed into the
-// two packed accumulators, split into 8 hi and 8 lo words of e4m3 codes.
-template <bool FULL>
-__device__ __forceinline__ void p_chunk(const uint32_t (&r)[32], int key0, int nvalid,
-                                        uint64_t c2, uint64_t nb2, uint64_t& l0, uint64_t& l1,
-                                        uint32_t (&pk)[16]) {
+// Probabilities of one 32-key chunk: p = 2^(s * c - bias) (a score of -inf
+// gives 0), summed into the two packed accumulators, split into 8 hi and 8
+// lo words of e4m3 codes.
+__device__ __forceinline__ void p_chunk(const uint32_t (&r)[32], uint64_t c2, uint64_t nb2,
+                                        uint64_t& l0, uint64_t& l1, uint32_t (&pk)[16]) {
     float p[32];
 #pragma unroll
     for (int i = 0; i < 32; i += 2) {
         float x0, x1;
         f2unpack(ffma2(f2pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), c2, nb2), x0,
                  x1);
-        if (!FULL) {
-            x0 = (key0 + i < nvalid) ? x0 : -INFINITY;
-            x1 = (key0 + i + 1 < nvalid) ? x1 : -INFINITY;
-            p[i] = ex2_approx(x0);
-            p[i + 1] = ex2_approx(x1);
-        } else if (FP8VIT_POLY_EVERY > 0 &&
-                   (i / 2) % (FP8VIT_POLY_EVERY > 0 ? FP8VIT_POLY_EVERY : 1) ==
-                       FP8VIT_POLY_EVERY - 1) {
-            exp2_poly2(x0, x1, p[i], p[i + 1]);
-        } else {
-            p[i] = ex2_approx(x0);
-            p[i + 1] = ex2_approx(x1);
-        }
+        p[i] = ex2_approx(x0);
+        p[i + 1] = ex2_approx(x1);
         if ((i / 2) & 1)
             l1 = fadd2(l1, f2pack(p[i], p[i + 1]));
         else
@@ -317,15 +270,14 @@ __device__ __forceinline__ void p_chunk(const uint32_t (&r)[32], int key0, int n
 // P of one 64-key tile written to a 32-column P slot: chunk c (keys
 // 32c..32c+31) goes to columns [16c, 16c+8) (hi) and [16c+8, 16c+16) (lo).
 // Returns the tile's probability sum.
-template <bool FULL>
 __device__ __forceinline__ float tile_p(const uint32_t (&a)[32], const uint32_t (&b)[32],
-                                        uint32_t tSb, int nvalid, uint64_t c2, uint64_t nb2) {
+                                        uint32_t tPb, uint64_t c2, uint64_t nb2) {
     uint32_t pk[16];
     uint64_t l0 = f2pack(0.0f, 0.0f), l1 = l0;
-    p_chunk<FULL>(a, 0, nvalid, c2, nb2, l0, l1, pk);
-    tmem_st16(tSb, pk);
-    p_chunk<FULL>(b, 32, nvalid, c2, nb2, l0, l1, pk);
-    tmem_st16(tSb + 16, pk);
+    p_chunk(a, c2, nb2, l0, l1, pk);
+    tmem_st16(tPb, pk);
+    p_chunk(b, c2, nb2, l0, l1, pk);
+    tmem_st16(tPb + 16, pk);
     float s0, s1;
     f2unpack(fadd2(l0, l1), s0, s1);
     return s0 + s1;
@@ -387,12 +339,12 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     if (threadIdx.x == 0) {
         mbar_init(b_q_full, 1);
-        mbar_init(b_q_ready, 128);
+        mbar_init(b_q_ready, 4);  // one elected arrival per softmax warp
         mbar_init(b_drain, 1);
         mbar_init(b_s_full, 1);
-        mbar_init(b_s_free, 128);
+        mbar_init(b_s_free, 4);
         for (int b = 0; b < 2; ++b) {
-            mbar_init(b_p_full(b), 128);
+            mbar_init(b_p_full(b), 4);
             mbar_init(b_o_ready(b), 1);
         }
         for (int s = 0; s < NS; ++s) {
@@ -542,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 *reinterpret_cast<uint2*>(q + row * kBox + ((0 ^ sw) << 4)) = make_uint2(0, 0);
         }
         fence_proxy_async_smem();
-        mbar_arrive(b_q_ready);
+        warp_arrive(b_q_ready, lane);
 
         // Running state per row, in log2 units of the scaled score
         // (x = s * scale_log2): m_ref is the reference max the exponentials
@@ -564,9 +516,16 @@ __global__ void __launch_bounds__(kThreads, 2)
             uint32_t ra[32], rb[32];
             tmem_ld64_sync(tSb, ra, rb);
             tc_fence_before();
-            mbar_arrive(b_s_free);  // the S buffer may take S(j+1) now
-            const float mx =
-                full ? tile_row_max<true>(ra, rb, nvalid) : tile_row_max<false>(ra, rb, nvalid);
+            warp_arrive(b_s_free, lane);  // the S buffer may take S(j+1) now
+            if (!full) {
+                // keys past the segment end score -inf: one code path below
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    ra[i] = i < nvalid ? ra[i] : 0xFF800000u;
+                    rb[i] = 32 + i < nvalid ? rb[i] : 0xFF800000u;
+                }
+            }
+            const float mx = tile_row_max(ra, rb);
             const float mxc = mx * scale_log2;
             // j == 0 sets the reference; the first PV initialises O.
             const bool need = j == 0 || mxc > m_ref + kSlackLog2;
@@ -581,8 +540,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const uint64_t c2 = f2pack(scale_log2, scale_log2);
             const uint64_t nb2 = f2pack(-bias, -bias);
             const uint32_t tPb = tP + 32 * b;
-            const float tile_sum = full ? tile_p<true>(ra, rb, tPb, nvalid, c2, nb2)
-                                        : tile_p<false>(ra, rb, tPb, nvalid, c2, nb2);
+            const float tile_sum = tile_p(ra, rb, tPb, c2, nb2);
             l_run = l_run * alpha + tile_sum;
             if (rescale) {
                 // O holds PV(0..j-1): wait for PV(j - 1), then scale it.
@@ -595,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(b_p_full(b));
+            warp_arrive(b_p_full(b), lane);
         }
         // epilogue
         if (ok) {
