@@ -283,7 +283,9 @@ __device__ __forceinline__ float tile_p(const uint32_t (&a)[32], const uint32_t 
     return s0 + s1;
 }
 
-template <int D>
+// FP8OUT selects the epilogue at compile time (e4m3 through output_scale, or
+// bf16), so each instance carries one epilogue only.
+template <int D, bool FP8OUT>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ dq_p,
@@ -568,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const float inv = __fdiv_rn(dv, l_run);
             const int64_t tok = (int64_t)seg_start + q0 + row;
             const int64_t off = (tok * num_heads + h) * D;
-            const float oscale = out_fp8 ? *out_scale_p : 1.0f;
+            const float oscale = FP8OUT ? *out_scale_p : 1.0f;
 #pragma unroll
             for (int c = 0; c < D / 8; ++c) {
                 uint32_t r[8];
@@ -577,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
                 for (int i = 0; i < 8; ++i) o[i] = __uint_as_float(r[i]) * inv;
                 if (!valid) continue;
-                if (out_fp8) {
+                if constexpr (FP8OUT) {
                     uint32_t w0 = (uint32_t)f32x2_to_e4m3x2(__fdiv_rn(o[0], oscale), __fdiv_rn(o[1], oscale)) |
                                   ((uint32_t)f32x2_to_e4m3x2(__fdiv_rn(o[2], oscale), __fdiv_rn(o[3], oscale)) << 16);
                     uint32_t w1 = (uint32_t)f32x2_to_e4m3x2(__fdiv_rn(o[4], oscale), __fdiv_rn(o[5], oscale)) |
@@ -630,13 +632,13 @@ fp8vit_status launch(fp8vit_ctx* ctx, const uint8_t* q8, const uint8_t* k8, cons
     if (!encode_map(&mq, q8, T, row_bytes, kBM) || !encode_map(&mk, k8, T, row_bytes, kBN) ||
         !encode_map(&mv, v8, T, row_bytes, kBN))
         return FP8VIT_ECUDA;
-    static bool attr_set[2] = {false, false};  // per template instance (one device set-up)
-    auto kern = attn_fwd_kernel<D>;
-    if (!attr_set[D == 128]) {
+    static bool attr_set[2] = {false, false};  // per output type (one device set-up)
+    auto kern = out_fp8 ? attn_fwd_kernel<D, true> : attn_fwd_kernel<D, false>;
+    if (!attr_set[out_fp8 ? 1 : 0]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Smem<D>::ALLOC) != cudaSuccess)
             return FP8VIT_ECUDA;
-        attr_set[D == 128] = true;
+        attr_set[out_fp8 ? 1 : 0] = true;
     }
     dim3 grid((unsigned)((max_seqlen + kBM - 1) / kBM), (unsigned)H, (unsigned)num_seqs);
     kern<<<grid, kThreads, Smem<D>::ALLOC, st>>>(mq, mk, mv, dq, dk, dv, cu, max_seqlen, T, H,
