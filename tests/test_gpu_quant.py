@@ -200,3 +200,30 @@ def test_quantize_every_bf16_value(ctx):
     x = np.concatenate([x, x[: (-x.size) % 8]])   # multiple of 8
     for d in _descale_set():
         _quant_case(ctx, x, x[::-1].copy(), x, [d, d, d])
+
+
+@pytest.mark.parametrize("group", [16, 32, 64, 128, 256])
+def test_group_quant_every_bf16_value(ctx, group):
+    """Every finite BF16 value (both zeros, subnormals, the largest finite)
+    through the group quantizer, shuffled into rows so that groups mix
+    magnitudes, bit for bit against the oracle's IEEE division."""
+    allb = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    x = allb[(allb & 0x7F80) != 0x7F80]
+    rng = np.random.default_rng(group)
+    x = rng.permutation(x)
+    n = 1024
+    x = np.concatenate([x, np.full((-x.size) % n, 0x8000, dtype=np.uint16)]).reshape(-1, n)
+    # a few groups of zeros only, of -0 only, and one value among zeros
+    x[0, :group] = 0
+    x[1, :group] = 0x8000
+    x[2, :group] = 0x8000
+    x[2, group // 2] = 0x0001
+    want_q, want_s = oracle.group_quant(x, group)
+    xq = torch.empty(x.shape, dtype=torch.uint8, device="cuda")
+    sc = torch.empty((x.shape[0], n // group), dtype=torch.float32, device="cuda")
+    fv.per_token_group_quant_fp8(_dev_bf16(x), group, xq, sc, ctx=ctx)
+    _check_ok(ctx)
+    got = _host_u8(xq)
+    bad = np.nonzero(got != want_q)
+    assert bad[0].size == 0, (bad[0][:5], bad[1][:5], got[bad][:5], want_q[bad][:5])
+    assert (_f32_bits(sc.cpu().numpy()) == _f32_bits(want_s)).all()
