@@ -342,7 +342,13 @@ fp8vit_status fp8_quantize_qkv_per_tensor(fp8vit_ctx* ctx, const uint16_t* d_q,
         misaligned(d_q8, 8) || misaligned(d_k8, 8) || misaligned(d_v8, 8) ||
         misaligned(d_descale3, 4))
         return FP8VIT_EINVAL;
-    const int grid = grid_for(n_elems >> 3, kQuantThreads, 4, 8 * ctx->num_sms);
+    // one resident wave of grid-stride blocks (see per_token_group_quant_fp8)
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant3_kernel, kQuantThreads, 0) !=
+            cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    const int grid = grid_for(n_elems >> 3, kQuantThreads, 4, per_sm * ctx->num_sms);
     quant3_kernel<<<grid, kQuantThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
         reinterpret_cast<const uint4*>(d_q), reinterpret_cast<const uint4*>(d_k),
         reinterpret_cast<const uint4*>(d_v), n_elems, d_descale3, reinterpret_cast<uint2*>(d_q8),
@@ -365,8 +371,20 @@ fp8vit_status per_token_group_quant_fp8(fp8vit_ctx* ctx, const uint16_t* d_x, in
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int lpg = group / 8;
     const int64_t gpw = 32 / (lpg > 0 ? lpg : 1);
+    // One resident wave: every block streams an equal grid-stride share, so a
+    // grid larger than what fits at once would leave a partial second wave.
+    int per_sm = 0;
+    const void* kfn = group == 16    ? (const void*)group_quant_kernel<2>
+                      : group == 32  ? (const void*)group_quant_kernel<4>
+                      : group == 64  ? (const void*)group_quant_kernel<8>
+                      : group == 128 ? (const void*)group_quant_kernel<16>
+                                     : (const void*)group_quant_kernel<32>;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kfn, kGroupThreads, 0) !=
+            cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
     const int grid = grid_for((total_groups + gpw - 1) / gpw * 32, kGroupThreads, 4,
-                              8 * ctx->num_sms);
+                              per_sm * ctx->num_sms);
     const uint4* x = reinterpret_cast<const uint4*>(d_x);
     uint2* xq = reinterpret_cast<uint2*>(d_xq);
     switch (group) {
