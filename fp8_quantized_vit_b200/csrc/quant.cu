@@ -282,6 +282,28 @@ inline bool misaligned(const void* p, uintptr_t a) {
     return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0;
 }
 
+// Resident blocks per SM of a kernel, queried once per kernel (later calls,
+// e.g. inside a CUDA-graph capture, make no CUDA API call).
+inline int resident_blocks(const void* kfn, int threads) {
+    static std::mutex mu;
+    static const void* keys[16];
+    static int vals[16];
+    static int n = 0;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n; ++i)
+        if (keys[i] == kfn) return vals[i];
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kfn, threads, 0) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    if (n < 16) {
+        keys[n] = kfn;
+        vals[n] = per_sm;
+        ++n;
+    }
+    return per_sm;
+}
+
 inline int grid_for(int64_t work_items, int threads, int per_thread, int max_blocks) {
     int64_t b = (work_items + (int64_t)threads * per_thread - 1) / ((int64_t)threads * per_thread);
     if (b < 1) b = 1;
@@ -343,11 +365,7 @@ fp8vit_status fp8_quantize_qkv_per_tensor(fp8vit_ctx* ctx, const uint16_t* d_q,
         misaligned(d_descale3, 4))
         return FP8VIT_EINVAL;
     // one resident wave of grid-stride blocks (see per_token_group_quant_fp8)
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant3_kernel, kQuantThreads, 0) !=
-            cudaSuccess ||
-        per_sm < 1)
-        per_sm = 1;
+    const int per_sm = resident_blocks((const void*)quant3_kernel, kQuantThreads);
     const int grid = grid_for(n_elems >> 3, kQuantThreads, 4, per_sm * ctx->num_sms);
     quant3_kernel<<<grid, kQuantThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
         reinterpret_cast<const uint4*>(d_q), reinterpret_cast<const uint4*>(d_k),
@@ -373,16 +391,12 @@ fp8vit_status per_token_group_quant_fp8(fp8vit_ctx* ctx, const uint16_t* d_x, in
     const int64_t gpw = 32 / (lpg > 0 ? lpg : 1);
     // One resident wave: every block streams an equal grid-stride share, so a
     // grid larger than what fits at once would leave a partial second wave.
-    int per_sm = 0;
     const void* kfn = group == 16    ? (const void*)group_quant_kernel<2>
                       : group == 32  ? (const void*)group_quant_kernel<4>
                       : group == 64  ? (const void*)group_quant_kernel<8>
                       : group == 128 ? (const void*)group_quant_kernel<16>
                                      : (const void*)group_quant_kernel<32>;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kfn, kGroupThreads, 0) !=
-            cudaSuccess ||
-        per_sm < 1)
-        per_sm = 1;
+    const int per_sm = resident_blocks(kfn, kGroupThreads);
     const int grid = grid_for((total_groups + gpw - 1) / gpw * 32, kGroupThreads, 4,
                               per_sm * ctx->num_sms);
     const uint4* x = reinterpret_cast<const uint4*>(d_x);
