@@ -197,6 +197,33 @@ def run_reference(args):
     return 0
 
 
+def _sdpa_comparator(w, inputs, dev, reps=10):
+    """torch's BF16 scaled_dot_product_attention on the same BF16 inputs of a
+    single-image workload: a library comparator for context, not the metric."""
+    import torch
+    import torch.nn.functional as F
+    if len(w.seg_lens) != 1:
+        return None
+    T, H, D = w.tokens, w.heads, w.head_dim
+    q, k, v = (x.view(1, T, H, D).transpose(1, 2) for x in inputs[0])
+    try:
+        for _ in range(2):
+            F.scaled_dot_product_attention(q, k, v, scale=w.softmax_scale)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            F.scaled_dot_product_attention(q, k, v, scale=w.softmax_scale)
+        e1.record()
+        torch.cuda.synchronize()
+    except Exception as exc:  # no fused BF16 kernel for this shape
+        return {"unavailable": str(exc).splitlines()[0][:120]}
+    ms = e0.elapsed_time(e1) / reps
+    return {"impl": "torch.nn.functional.scaled_dot_product_attention, bf16",
+            "ms": ms, "tflops": w.attn_flops() / (ms * 1e-3) / 1e12}
+
+
 def _quant_rooflines(fv, ctx, src, dev, hbm_gbs, reps=10):
     """HBM roofline of the three quantizer kernels on 3 x 32400-token, 16-head,
     head_dim-72 tensors ([97200, 1152] BF16 each, 224 MB): the resident BF16
@@ -429,6 +456,8 @@ def run_ours(args):
         "clocks": clk,
         "quantizers": quant,
     }
+    if args.compare_sdpa:
+        line["comparator"] = _sdpa_comparator(w, inputs, dev)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         codes, dsc = _oracle_inputs(w)
         f, sec, rows = _oracle_rows_time(w, codes, dsc, args.cpu_seconds, seed=7)
@@ -459,6 +488,8 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=1.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-quant-roofline", action="store_true")
+    ap.add_argument("--compare-sdpa", action="store_true",
+                    help="also time torch BF16 SDPA on the same inputs (single-image workloads)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
