@@ -26,6 +26,8 @@
 // runs with N = 80 and the epilogue picks the head's 72 columns.
 #include <math.h>
 
+#include <atomic>
+
 #include "fp8vit_internal.cuh"
 
 namespace {
@@ -632,13 +634,18 @@ fp8vit_status launch(fp8vit_ctx* ctx, const uint8_t* q8, const uint8_t* k8, cons
     if (!encode_map(&mq, q8, T, row_bytes, kBM) || !encode_map(&mk, k8, T, row_bytes, kBN) ||
         !encode_map(&mv, v8, T, row_bytes, kBN))
         return FP8VIT_ECUDA;
-    static bool attr_set[2] = {false, false};  // per output type (one device set-up)
+    // The dynamic shared-memory limit is a per-device setting of each kernel
+    // instance: raise it once per (device, output type).
+    static std::atomic<uint64_t> attr_set[2];
     auto kern = out_fp8 ? attn_fwd_kernel<D, true> : attn_fwd_kernel<D, false>;
-    if (!attr_set[out_fp8 ? 1 : 0]) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FP8VIT_ECUDA;
+    const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
+    if (!bit || !(attr_set[out_fp8 ? 1 : 0].load() & bit)) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Smem<D>::ALLOC) != cudaSuccess)
             return FP8VIT_ECUDA;
-        attr_set[out_fp8 ? 1 : 0] = true;
+        attr_set[out_fp8 ? 1 : 0].fetch_or(bit);
     }
     dim3 grid((unsigned)((max_seqlen + kBM - 1) / kBM), (unsigned)H, (unsigned)num_seqs);
     kern<<<grid, kThreads, Smem<D>::ALLOC, st>>>(mq, mk, mv, dq, dk, dv, cu, max_seqlen, T, H,
