@@ -4,15 +4,20 @@
 // output_scale epilogue that writes e4m3).
 //
 // One CTA = one (image, head, 128-row query tile).  Warp roles:
-//   warp 0      TMA producer: Q once, then K/V tiles of 64 keys into an
-//               NS-stage shared-memory ring (SWIZZLE_32B, 32-byte boxes).
+//   warp 0      TMA producer: Q once, then K/V tiles of BN keys (64 at
+//               head_dim 128, 96 at head_dim 72) into an NS-stage
+//               shared-memory ring (SWIZZLE_32B, 32-byte boxes).
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer:
 //               S = Q K^T (kind::f8f6f4, K-major A and B) into the TMEM S
 //               buffer, O += P V (A = P from TMEM, B = V MN-major from
 //               smem).  S(j+1) is issued as soon as the softmax warps have
 //               copied S(j) into registers, so it is computed while they
-//               work on tile j; P has two TMEM slots of its own, so the next
-//               QK never waits for the previous PV.
+//               work on tile j; P has TMEM columns of its own, so the next
+//               QK never waits for the previous PV.  TMEM (256 columns, two
+//               CTAs per SM): head_dim 128 has S 64 + two P slots of 32 + O
+//               128; head_dim 72 has S 96 + one P slot of 48 + O 80, and its
+//               softmax computes P(j) in registers and stores it once PV(j-1)
+//               has read the slot.
 //   warps 2..5  softmax + epilogue, one query row per thread (TMEM lane):
 //               row max, exp2, row sum in registers; P written to its TMEM
 //               slot as two e4m3 terms (hi + lo) so that the PV product
@@ -33,15 +38,10 @@
 namespace {
 
 constexpr int kBM = 128;          // query rows per CTA (MMA M)
-constexpr int kBN = 64;           // keys per KV tile (QK MMA N, PV MMA K)
 constexpr int kThreads = 192;     // 6 warps
 constexpr int kTmemCols = 256;
-constexpr uint32_t kTmemS = 0;    // S buffer: columns [0, 64)
-constexpr uint32_t kTmemP = 64;   // P slots: columns [64 + 32b, 96 + 32b), b = tile parity
-constexpr uint32_t kTmemO = 128;  // O accumulator columns [128, 128 + NPV)
 constexpr int kBox = 32;          // bytes per TMA box row (one SW32 atom row)
 constexpr int kQTileBytes = kBox * kBM;   // one [128 rows x 32 B] Q box
-constexpr int kKVTileBytes = kBox * kBN;  // one [64 rows x 32 B] K or V box
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 // P is stored as 2^(x - m_ref + kPLog2); a tile max up to kSlackLog2 above the
 // reference max keeps P <= 2^(6 + 2.75) = 430 < 448 (e4m3 max).
@@ -56,6 +56,10 @@ struct Cfg<72> {
     static constexpr int VA = 3;    // 32-byte V column blocks loaded (96 bytes)
     static constexpr int NPV = 80;  // PV MMA N (covers head bytes [0,72) or [8,80))
     static constexpr int NS = 5;    // K/V pipeline stages
+    static constexpr int BN = 96;   // keys per KV tile (QK MMA N, PV MMA K)
+    static constexpr int PSLOTS = 1;
+    // TMEM columns: S [0, 96), one P slot [96, 144), O [144, 224)
+    static constexpr uint32_t TS = 0, TP = 96, TO = 144;
 };
 template <>
 struct Cfg<128> {
@@ -63,14 +67,19 @@ struct Cfg<128> {
     static constexpr int VA = 4;
     static constexpr int NPV = 128;
     static constexpr int NS = 4;
+    static constexpr int BN = 64;
+    static constexpr int PSLOTS = 2;
+    // TMEM columns: S [0, 64), P slots [64 + 32b, 96 + 32b), O [128, 256)
+    static constexpr uint32_t TS = 0, TP = 64, TO = 128;
 };
 
 template <int D>
 struct Smem {
     static constexpr int Q = 0;
     static constexpr int K = Q + Cfg<D>::KB * kQTileBytes;
-    static constexpr int V = K + Cfg<D>::NS * Cfg<D>::KB * kKVTileBytes;
-    static constexpr int BAR = V + Cfg<D>::NS * Cfg<D>::VA * kKVTileBytes;
+    static constexpr int KVT = kBox * Cfg<D>::BN;  // one [BN rows x 32 B] K or V box
+    static constexpr int V = K + Cfg<D>::NS * Cfg<D>::KB * KVT;
+    static constexpr int BAR = V + Cfg<D>::NS * Cfg<D>::VA * KVT;
     static constexpr int TOTAL = BAR + 256;
     static constexpr int ALLOC = TOTAL + 1024;  // slack for 1024-byte alignment
 };
@@ -83,8 +92,9 @@ __device__ __forceinline__ uint64_t desc_k_sw32(uint32_t addr) {
     return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(256 >> 4) << 32) |
            ((uint64_t)1 << 46) | ((uint64_t)6 << 61);
 }
+template <int KVT>
 __device__ __forceinline__ uint64_t desc_mn_sw32(uint32_t addr) {
-    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)(kKVTileBytes >> 4) << 16) |
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)(KVT >> 4) << 16) |
            ((uint64_t)(256 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)6 << 61);
 }
 
@@ -232,18 +242,25 @@ __device__ __forceinline__ void p_split4(float p0, float p1, float p2, float p3,
     lo = l01 | (l23 << 16);
 }
 
-// Row max of one 64-key S tile held in registers (a = keys 0..31, b = keys
-// 32..63); keys past the segment end already hold -inf.
-__device__ __forceinline__ float tile_row_max(const uint32_t (&a)[32], const uint32_t (&b)[32]) {
-    float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+// Row max of one S tile of NCH 32-key chunks held in registers; keys past the
+// segment end already hold -inf.
+template <int NCH>
+__device__ __forceinline__ float tile_row_max(const uint32_t (&r)[NCH][32]) {
+    float m[NCH];
 #pragma unroll
-    for (int i = 0; i < 32; i += 4) {
-        m0 = fmax3(m0, __uint_as_float(a[i]), __uint_as_float(a[i + 1]));
-        m1 = fmax3(m1, __uint_as_float(a[i + 2]), __uint_as_float(a[i + 3]));
-        m2 = fmax3(m2, __uint_as_float(b[i]), __uint_as_float(b[i + 1]));
-        m3 = fmax3(m3, __uint_as_float(b[i + 2]), __uint_as_float(b[i + 3]));
+    for (int c = 0; c < NCH; ++c) {
+        float a = -INFINITY, b = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+            a = fmax3(a, __uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1]));
+            b = fmax3(b, __uint_as_float(r[c][i + 2]), __uint_as_float(r[c][i + 3]));
+        }
+        m[c] = fmaxf(a, b);
     }
-    return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+    float mx = m[0];
+#pragma unroll
+    for (int c = 1; c < NCH; ++c) mx = fmaxf(mx, m[c]);
+    return mx;
 }
 
 // Probabilities of one 32-key chunk: p = 2^(s * c - bias) (a score of -inf
@@ -312,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     const int q0 = qt * kBM;
     if (q0 >= seg_len) return;
-    const int n_kv = (seg_len + kBN - 1) / kBN;
+    const int n_kv = (seg_len + C::BN - 1) / C::BN;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
@@ -388,13 +405,13 @@ __global__ void __launch_bounds__(kThreads, 2)
                     !mbar_wait_bounded(b_kv_empty(s), ((j / NS) - 1) & 1, abort_flag, scr,
                                        SITE_ATTN_WAIT_EMPTY, kTimeoutNs))
                     break;
-                const int32_t row = seg_start + j * kBN;
-                mbar_arrive_expect_tx(b_kv_full(s), (C::KB + C::VA) * kKVTileBytes);
+                const int32_t row = seg_start + j * C::BN;
+                mbar_arrive_expect_tx(b_kv_full(s), (C::KB + C::VA) * L::KVT);
                 for (int kb = 0; kb < C::KB; ++kb)
-                    tma_load_2d(sK + (s * C::KB + kb) * kKVTileBytes, &tm_k, x0 + kBox * kb, row,
+                    tma_load_2d(sK + (s * C::KB + kb) * L::KVT, &tm_k, x0 + kBox * kb, row,
                                 b_kv_full(s));
                 for (int a = 0; a < C::VA; ++a)
-                    tma_load_2d(sV + (s * C::VA + a) * kKVTileBytes, &tm_v, x0 + kBox * a, row,
+                    tma_load_2d(sV + (s * C::VA + a) * L::KVT, &tm_v, x0 + kBox * a, row,
                                 b_kv_full(s));
                 ++issued;
             }
@@ -413,16 +430,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         // P(j) is waited for, so the tensor cores compute the next scores
         // while the softmax warps work on the current ones.
         if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_e4m3(kBN, false);
+            constexpr uint32_t idesc_qk = idesc_e4m3(C::BN, false);
             constexpr uint32_t idesc_pv = idesc_e4m3(C::NPV, true);
-            const uint32_t tO = tmem + kTmemO;
+            const uint32_t tO = tmem + C::TO;
             auto issue_qk = [&](int j) {
                 const int s = j % NS;
-                const uint32_t tSb = tmem + kTmemS;
+                const uint32_t tSb = tmem + C::TS;
 #pragma unroll
                 for (int kb = 0; kb < C::KB; ++kb)
                     umma_f8_ss(tSb, desc_k_sw32(sQ + kb * kQTileBytes),
-                               desc_k_sw32(sK + (s * C::KB + kb) * kKVTileBytes), idesc_qk,
+                               desc_k_sw32(sK + (s * C::KB + kb) * L::KVT), idesc_qk,
                                kb > 0 ? 1u : 0u);
                 umma_commit(b_s_full);
             };
@@ -456,11 +473,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                                        SITE_ATTN_WAIT_P, kTimeoutNs))
                     break;
                 tc_fence_after();
-                const uint32_t tPb = tmem + kTmemP + 32 * (j & 1);
-                const uint32_t vbase = sV + s * C::VA * kKVTileBytes;
+                const uint32_t tPb = tmem + C::TP + (C::PSLOTS == 2 ? 32 * (j & 1) : 0);
+                const uint32_t vbase = sV + s * C::VA * L::KVT;
 #pragma unroll
-                for (int kk = 0; kk < kBN / 32; ++kk) {
-                    const uint64_t bdesc = desc_mn_sw32(vbase + kk * 32 * kBox);
+                for (int kk = 0; kk < C::BN / 32; ++kk) {
+                    const uint64_t bdesc = desc_mn_sw32<L::KVT>(vbase + kk * 32 * kBox);
                     umma_f8_ts(tO, tPb + 16 * kk, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
                     umma_f8_ts(tO, tPb + 16 * kk + 8, bdesc, idesc_pv, 1u);
                 }
@@ -478,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;  // query row in the tile == TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-        const uint32_t tS = lane_base + kTmemS, tP = lane_base + kTmemP, tO = lane_base + kTmemO;
+        const uint32_t tS = lane_base + C::TS, tP = lane_base + C::TP, tO = lane_base + C::TO;
         const float dq = *dq_p, dk = *dk_p, dv = *dv_p;
         const float scale_log2 = sm_scale * dq * dk * 1.4426950408889634f;
 
@@ -508,52 +525,77 @@ __global__ void __launch_bounds__(kThreads, 2)
         // tile's max exceeds m_ref by more than kSlackLog2 (both are scaled
         // by the same factor, so the final o = O / l is unchanged).
         float m_ref = -INFINITY, l_run = 0.0f;
-        const uint32_t tSb = tS;
+        constexpr int NCH = C::BN / 32;
         for (int j = 0; ok && j < n_kv; ++j) {
             const int b = j & 1;
             ok = mbar_wait_bounded(b_s_full, j & 1, abort_flag, scr, SITE_ATTN_WAIT_S, kTimeoutNs);
             ok = __all_sync(0xFFFFFFFFu, ok);
             if (!ok) break;
             tc_fence_after();
-            const int nvalid = min(kBN, seg_len - j * kBN);
-            const bool full = nvalid == kBN;
-            uint32_t ra[32], rb[32];
-            tmem_ld64_sync(tSb, ra, rb);
+            const int nvalid = min(C::BN, seg_len - j * C::BN);
+            uint32_t r[NCH][32];
+            if constexpr (NCH == 2) {
+                tmem_ld64_sync(tS, r[0], r[1]);
+            } else {
+#pragma unroll
+                for (int c = 0; c < NCH; ++c) tmem_ld32(tS + 32 * c, r[c]);
+                tmem_wait_ld();
+            }
             tc_fence_before();
             warp_arrive(b_s_free, lane);  // the S buffer may take S(j+1) now
-            if (!full) {
+            if (nvalid < C::BN) {
                 // keys past the segment end score -inf: one code path below
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    ra[i] = i < nvalid ? ra[i] : 0xFF800000u;
-                    rb[i] = 32 + i < nvalid ? rb[i] : 0xFF800000u;
-                }
+                for (int c = 0; c < NCH; ++c)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        r[c][i] = 32 * c + i < nvalid ? r[c][i] : 0xFF800000u;
             }
-            const float mx = tile_row_max(ra, rb);
+            const float mx = tile_row_max<NCH>(r);
             const float mxc = mx * scale_log2;
             // j == 0 sets the reference; the first PV initialises O.
             const bool need = j == 0 || mxc > m_ref + kSlackLog2;
             const bool rescale = j > 0 && __any_sync(0xFFFFFFFFu, need);
             const float alpha = (j > 0 && need) ? ex2_approx(m_ref - mxc) : 1.0f;
             if (need) m_ref = mxc;
-            // P slot b held P(j - 2).  PV(j - 2) was issued before QK(j), and
-            // the commit that completed s_full(j) tracks every earlier MMA of
-            // the issuer, so PV(j - 2) has completed: the slot is free.
             // P = 2^(x - bias), bias = m_ref - kPLog2
             const float bias = m_ref - kPLog2;
             const uint64_t c2 = f2pack(scale_log2, scale_log2);
             const uint64_t nb2 = f2pack(-bias, -bias);
-            const uint32_t tPb = tP + 32 * b;
-            const float tile_sum = tile_p(ra, rb, tPb, c2, nb2);
-            l_run = l_run * alpha + tile_sum;
-            if (rescale) {
-                // O holds PV(0..j-1): wait for PV(j - 1), then scale it.
-                ok = mbar_wait_bounded(b_o_ready((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag,
-                                       scr, SITE_ATTN_WAIT_O, kTimeoutNs);
-                ok = __all_sync(0xFFFFFFFFu, ok);
-                if (!ok) break;
-                tc_fence_after();
-                rescale_o<C::NPV>(tO, alpha);
+            if constexpr (C::PSLOTS == 2) {
+                // P slot b held P(j - 2).  PV(j - 2) was issued before QK(j),
+                // and the commit that completed s_full(j) tracks every earlier
+                // MMA of the issuer, so PV(j - 2) has completed: the slot is free.
+                l_run = l_run * alpha + tile_p(r[0], r[1], tP + 32 * b, c2, nb2);
+                if (rescale) {
+                    // O holds PV(0..j-1): wait for PV(j - 1), then scale it.
+                    ok = mbar_wait_bounded(b_o_ready((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag,
+                                           scr, SITE_ATTN_WAIT_O, kTimeoutNs);
+                    ok = __all_sync(0xFFFFFFFFu, ok);
+                    if (!ok) break;
+                    tc_fence_after();
+                    rescale_o<C::NPV>(tO, alpha);
+                }
+            } else {
+                // One P slot: P(j) is computed in registers, then stored once
+                // PV(j - 1) has read P(j - 1) (and completed O for a rescale).
+                uint64_t l0 = f2pack(0.0f, 0.0f), l1 = l0;
+                uint32_t pk[NCH][16];
+#pragma unroll
+                for (int c = 0; c < NCH; ++c) p_chunk(r[c], c2, nb2, l0, l1, pk[c]);
+                float s0, s1;
+                f2unpack(fadd2(l0, l1), s0, s1);
+                l_run = l_run * alpha + (s0 + s1);
+                if (j > 0) {
+                    ok = mbar_wait_bounded(b_o_ready((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag,
+                                           scr, SITE_ATTN_WAIT_O, kTimeoutNs);
+                    ok = __all_sync(0xFFFFFFFFu, ok);
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+#pragma unroll
+                for (int c = 0; c < NCH; ++c) tmem_st16(tP + 16 * c, pk[c]);
+                if (rescale) rescale_o<C::NPV>(tO, alpha);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -631,8 +673,9 @@ fp8vit_status launch(fp8vit_ctx* ctx, const uint8_t* q8, const uint8_t* k8, cons
                      void* out, int32_t out_fp8, const float* out_scale, cudaStream_t st) {
     CUtensorMap mq, mk, mv;
     const int64_t row_bytes = (int64_t)H * D;
-    if (!encode_map(&mq, q8, T, row_bytes, kBM) || !encode_map(&mk, k8, T, row_bytes, kBN) ||
-        !encode_map(&mv, v8, T, row_bytes, kBN))
+    if (!encode_map(&mq, q8, T, row_bytes, kBM) ||
+        !encode_map(&mk, k8, T, row_bytes, Cfg<D>::BN) ||
+        !encode_map(&mv, v8, T, row_bytes, Cfg<D>::BN))
         return FP8VIT_ECUDA;
     // The dynamic shared-memory limit is a per-device setting of each kernel
     // instance: raise it once per (device, output type).

@@ -78,6 +78,7 @@ def _gpu_bf16_to_f64(out: torch.Tensor) -> np.ndarray:
 SMALL = [
     ((1,), 2, 72), ((2,), 2, 128), ((127,), 2, 72), ((128,), 2, 128), ((129,), 4, 72),
     ((300, 1, 77), 2, 72), ((256, 129), 2, 128), ((5, 0, 200), 2, 72), ((513,), 2, 128),
+    ((96, 192, 97), 2, 72), ((64, 65, 191), 2, 128),
 ]
 
 
