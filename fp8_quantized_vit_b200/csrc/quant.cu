@@ -267,7 +267,11 @@ __global__ void __launch_bounds__(kGroupThreads) group_quant_kernel(
 #pragma unroll
             for (int off = LPG / 2; off > 0; off >>= 1)
                 a = max(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
-            float sc = __fdiv_rn(bf16_bits_to_f32(a), 448.0f);
+            // amax / 448 in IEEE fp32: Markstein with RN(1/448), exact for
+            // every non-negative bf16 amax
+            const float af = bf16_bits_to_f32(a);
+            const float q0 = __fmul_rn(af, 1.0f / 448.0f);
+            float sc = __fmaf_rn(__fmaf_rn(-448.0f, q0, af), 1.0f / 448.0f, q0);
             sc = sc > 1e-10f ? sc : 1e-10f;
             if (g < total_groups) {
                 const float nr = -__frcp_rn(sc);

@@ -202,6 +202,36 @@ def test_quantize_every_bf16_value(ctx):
         _quant_case(ctx, x, x[::-1].copy(), x, [d, d, d])
 
 
+def test_group_quant_every_amax(ctx):
+    """Each of the 32640 non-negative finite BF16 values (zero included) is
+    the amax of one 128-element group, so the scale amax / 448 and its
+    reciprocal are exercised at every value they can take; the other 127
+    elements of the group are random BF16 values of magnitude <= the amax,
+    either sign.  Bit for bit against the oracle's IEEE division."""
+    group = 128
+    amax_bits = np.arange(0, 0x7F80, dtype=np.uint32)
+    g = amax_bits.size
+    rng = np.random.default_rng(2024)
+    mag = (rng.random((g, group)) * (amax_bits[:, None] + 1)).astype(np.uint32)
+    mag = np.minimum(mag, amax_bits[:, None])
+    mag[:, 0] = amax_bits
+    sign = rng.integers(0, 2, size=(g, group), dtype=np.uint32) << 15
+    x = (mag | sign).astype(np.uint16)
+    # the amax element at a random position of its group
+    perm = rng.permuted(np.tile(np.arange(group), (g, 1)), axis=1)
+    x = np.take_along_axis(x, perm, axis=1)
+    x = x.reshape(-1, 8 * group)  # 8 groups per row
+    want_q, want_s = oracle.group_quant(x, group)
+    xq = torch.empty(x.shape, dtype=torch.uint8, device="cuda")
+    sc = torch.empty((x.shape[0], 8), dtype=torch.float32, device="cuda")
+    fv.per_token_group_quant_fp8(_dev_bf16(x), group, xq, sc, ctx=ctx)
+    _check_ok(ctx)
+    got = _host_u8(xq)
+    bad = np.nonzero(got != want_q)
+    assert bad[0].size == 0, (bad[0][:5], bad[1][:5], got[bad][:5], want_q[bad][:5])
+    assert (_f32_bits(sc.cpu().numpy()) == _f32_bits(want_s)).all()
+
+
 @pytest.mark.parametrize("group", [16, 32, 64, 128, 256])
 def test_group_quant_every_bf16_value(ctx, group):
     """Every finite BF16 value (both zeros, subnormals, the largest finite)
