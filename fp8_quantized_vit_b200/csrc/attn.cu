@@ -225,23 +225,6 @@ __device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
     return d;
 }
 
-// Split 4 probabilities into one hi word and one lo word of e4m3 codes,
-// hi + lo ~= p with ~8 significant bits, so that the PV product on FP8
-// tensor cores keeps about a BF16-width P.  p is rounded to f16 (11 bits);
-// hi = e4m3(p16); the residual p16 - hi is exact in f16 (both share the
-// exponent range of p16); lo = e4m3(residual).  Five conversions/subtracts
-// per pair.  The words are combined from zero-extended halves with shifts
-// (packing two 16-bit asm results with mov.b32 {a, b} was miscompiled here).
-__device__ __forceinline__ void p_split4(float p0, float p1, float p2, float p3, uint32_t& hi,
-                                         uint32_t& lo) {
-    const uint32_t h01 = cvt_f16x2(p0, p1), h23 = cvt_f16x2(p2, p3);
-    const uint32_t e01 = e4m3x2_of_f16x2(h01), e23 = e4m3x2_of_f16x2(h23);
-    const uint32_t l01 = e4m3x2_of_f16x2(hsub2(h01, f16x2_of_e4m3x2(e01)));
-    const uint32_t l23 = e4m3x2_of_f16x2(hsub2(h23, f16x2_of_e4m3x2(e23)));
-    hi = e01 | (e23 << 16);
-    lo = l01 | (l23 << 16);
-}
-
 // Row max of one S tile of NCH 32-key chunks held in registers; keys past the
 // segment end already hold -inf.
 template <int NCH>
@@ -264,26 +247,47 @@ __device__ __forceinline__ float tile_row_max(const uint32_t (&r)[NCH][32]) {
 }
 
 // Probabilities of one 32-key chunk: p = 2^(s * c - bias) (a score of -inf
-// gives 0), summed into the two packed accumulators, split into 8 hi and 8
-// lo words of e4m3 codes.
+// gives 0), summed into the two packed accumulators, then split into 8 hi and
+// 8 lo words of e4m3 codes with hi + lo ~= p to ~8 significant bits, so that
+// the PV product on FP8 tensor cores keeps about a BF16-width P: p is rounded
+// to f16 (11 bits); hi = e4m3(p16); the residual p16 - hi is exact in f16
+// (both share the exponent range of p16); lo = e4m3(residual).  Five
+// conversions/subtracts per pair, written stage by stage over the chunk.  The
+// words are combined from zero-extended halves with shifts (packing two
+// 16-bit asm results with mov.b32 {a, b} was miscompiled here).
 __device__ __forceinline__ void p_chunk(const uint32_t (&r)[32], uint64_t c2, uint64_t nb2,
                                         uint64_t& l0, uint64_t& l1, uint32_t (&pk)[16]) {
     float p[32];
+    uint64_t x[16];
 #pragma unroll
-    for (int i = 0; i < 32; i += 2) {
+    for (int i = 0; i < 16; ++i)
+        x[i] = ffma2(f2pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), c2, nb2);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
         float x0, x1;
-        f2unpack(ffma2(f2pack(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), c2, nb2), x0,
-                 x1);
-        p[i] = ex2_approx(x0);
-        p[i + 1] = ex2_approx(x1);
-        if ((i / 2) & 1)
-            l1 = fadd2(l1, f2pack(p[i], p[i + 1]));
-        else
-            l0 = fadd2(l0, f2pack(p[i], p[i + 1]));
+        f2unpack(x[i], x0, x1);
+        p[2 * i] = ex2_approx(x0);
+        p[2 * i + 1] = ex2_approx(x1);
     }
 #pragma unroll
-    for (int w = 0; w < 8; ++w)
-        p_split4(p[4 * w], p[4 * w + 1], p[4 * w + 2], p[4 * w + 3], pk[w], pk[8 + w]);
+    for (int i = 0; i < 16; i += 2) {
+        l0 = fadd2(l0, f2pack(p[2 * i], p[2 * i + 1]));
+        l1 = fadd2(l1, f2pack(p[2 * i + 2], p[2 * i + 3]));
+    }
+    uint32_t h[16], e[16], d[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) h[i] = cvt_f16x2(p[2 * i], p[2 * i + 1]);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) e[i] = e4m3x2_of_f16x2(h[i]);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) d[i] = hsub2(h[i], f16x2_of_e4m3x2(e[i]));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) d[i] = e4m3x2_of_f16x2(d[i]);
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+        pk[w] = e[2 * w] | (e[2 * w + 1] << 16);
+        pk[8 + w] = d[2 * w] | (d[2 * w + 1] << 16);
+    }
 }
 
 // P of one 64-key tile written to a 32-column P slot: chunk c (keys
