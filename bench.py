@@ -294,6 +294,8 @@ def run_ours(args):
     T, H, D = w.tokens, w.heads, w.head_dim
     n_fwd = len(w.seeds) if args.forwards <= 0 else min(args.forwards, len(w.seeds))
     ctx = fv.Context(local)
+    if args.p_terms != 2:
+        ctx.set_attn_p_terms(args.p_terms)
     dev = torch.device("cuda", local)
 
     # inputs: all forwards resident in HBM
@@ -442,7 +444,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3 (fp32 accumulate)",
-        "data": "synthetic", "config": _config(w, n_fwd),
+        "data": "synthetic", "config": dict(_config(w, n_fwd), p_terms=args.p_terms),
         "roofline": {"bound": "tensor", "kernel": f"attn_fwd_kernel<{D}>",
                      "achieved": attn_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
                      "frac": attn_tflops / fp8_peak, "traffic": traffic,
@@ -488,6 +490,9 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=1.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-quant-roofline", action="store_true")
+    ap.add_argument("--p-terms", type=int, choices=[1, 2], default=2,
+                    help="e4m3 terms of P in the PV product (2: hi + lo, the default that meets "
+                         "the attention tolerance; 1: a single term, faster, less accurate)")
     ap.add_argument("--compare-sdpa", action="store_true",
                     help="also time torch BF16 SDPA on the same inputs (single-image workloads)")
     args = ap.parse_args()

@@ -34,6 +34,7 @@ _SIGNATURES = {
     "fp8vit_destroy": (_I32, [_P]),
     "fp8vit_check": (_I32, [_P, _P, ctypes.POINTER(_I32)]),
     "fp8vit_status_string": (ctypes.c_char_p, [_I32]),
+    "fp8vit_set_attn_p_terms": (_I32, [_P, _I32]),
     "fp8vit_version": (_I32, []),
     "fp8vit_ring_init": (_I32, [_P, _P]),
     "fp8_amax_ring_update": (_I32, [_P, _P, _P, _P, _I64, _P, _P, _P]),
@@ -121,6 +122,12 @@ class Context:
         site = _I32(0)
         st = lib().fp8vit_check(self.handle, _stream(stream), ctypes.byref(site))
         return st, site.value
+
+    def set_attn_p_terms(self, terms: int):
+        """P of the attention's PV product as 2 e4m3 terms (hi + lo, the
+        default, meets the attention tolerance) or 1 (faster, ~3 significant
+        bits of P)."""
+        _check(lib().fp8vit_set_attn_p_terms(self.handle, terms), "fp8vit_set_attn_p_terms")
 
     def close(self):
         if getattr(self, "handle", None):

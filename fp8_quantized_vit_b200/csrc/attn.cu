@@ -255,6 +255,7 @@ __device__ __forceinline__ float tile_row_max(const uint32_t (&r)[NCH][32]) {
 // conversions/subtracts per pair, written stage by stage over the chunk.  The
 // words are combined from zero-extended halves with shifts (packing two
 // 16-bit asm results with mov.b32 {a, b} was miscompiled here).
+template <bool PLO>
 __device__ __forceinline__ void p_chunk(const uint32_t (&r)[32], uint64_t c2, uint64_t nb2,
                                         uint64_t& l0, uint64_t& l1, uint32_t (&pk)[16]) {
     float p[32];
@@ -274,41 +275,65 @@ __device__ __forceinline__ void p_chunk(const uint32_t (&r)[32], uint64_t c2, ui
         l0 = fadd2(l0, f2pack(p[2 * i], p[2 * i + 1]));
         l1 = fadd2(l1, f2pack(p[2 * i + 2], p[2 * i + 3]));
     }
-    uint32_t h[16], e[16], d[16];
+    if constexpr (!PLO) {
+        // single e4m3 term: P rounded once, straight from fp32
 #pragma unroll
-    for (int i = 0; i < 16; ++i) h[i] = cvt_f16x2(p[2 * i], p[2 * i + 1]);
+        for (int w = 0; w < 8; ++w)
+            pk[w] = (uint32_t)f32x2_to_e4m3x2(p[4 * w], p[4 * w + 1]) |
+                    ((uint32_t)f32x2_to_e4m3x2(p[4 * w + 2], p[4 * w + 3]) << 16);
+    } else {
+        uint32_t h[16], e[16], d[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) e[i] = e4m3x2_of_f16x2(h[i]);
+        for (int i = 0; i < 16; ++i) h[i] = cvt_f16x2(p[2 * i], p[2 * i + 1]);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) d[i] = hsub2(h[i], f16x2_of_e4m3x2(e[i]));
+        for (int i = 0; i < 16; ++i) e[i] = e4m3x2_of_f16x2(h[i]);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) d[i] = e4m3x2_of_f16x2(d[i]);
+        for (int i = 0; i < 16; ++i) d[i] = hsub2(h[i], f16x2_of_e4m3x2(e[i]));
 #pragma unroll
-    for (int w = 0; w < 8; ++w) {
-        pk[w] = e[2 * w] | (e[2 * w + 1] << 16);
-        pk[8 + w] = d[2 * w] | (d[2 * w + 1] << 16);
+        for (int i = 0; i < 16; ++i) d[i] = e4m3x2_of_f16x2(d[i]);
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            pk[w] = e[2 * w] | (e[2 * w + 1] << 16);
+            pk[8 + w] = d[2 * w] | (d[2 * w + 1] << 16);
+        }
+    }
+}
+
+// One chunk's P words into TMEM: hi in the first 8 columns, lo (when kept)
+// in the next 8.
+template <bool PLO>
+__device__ __forceinline__ void tmem_st_p(uint32_t taddr, const uint32_t (&pk)[16]) {
+    if constexpr (PLO) {
+        tmem_st16(taddr, pk);
+    } else {
+        uint32_t hi[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) hi[i] = pk[i];
+        tmem_st8(taddr, hi);
     }
 }
 
 // P of one 64-key tile written to a 32-column P slot: chunk c (keys
 // 32c..32c+31) goes to columns [16c, 16c+8) (hi) and [16c+8, 16c+16) (lo).
 // Returns the tile's probability sum.
+template <bool PLO>
 __device__ __forceinline__ float tile_p(const uint32_t (&a)[32], const uint32_t (&b)[32],
                                         uint32_t tPb, uint64_t c2, uint64_t nb2) {
     uint32_t pk[16];
     uint64_t l0 = f2pack(0.0f, 0.0f), l1 = l0;
-    p_chunk(a, c2, nb2, l0, l1, pk);
-    tmem_st16(tPb, pk);
-    p_chunk(b, c2, nb2, l0, l1, pk);
-    tmem_st16(tPb + 16, pk);
+    p_chunk<PLO>(a, c2, nb2, l0, l1, pk);
+    tmem_st_p<PLO>(tPb, pk);
+    p_chunk<PLO>(b, c2, nb2, l0, l1, pk);
+    tmem_st_p<PLO>(tPb + 16, pk);
     float s0, s1;
     f2unpack(fadd2(l0, l1), s0, s1);
     return s0 + s1;
 }
 
 // FP8OUT selects the epilogue at compile time (e4m3 through output_scale, or
-// bf16), so each instance carries one epilogue only.
-template <int D, bool FP8OUT>
+// bf16), so each instance carries one epilogue only; PLO keeps P as two e4m3
+// terms (hi + lo, two PV MMAs) or, when false, as one.
+template <int D, bool FP8OUT, bool PLO>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ dq_p,
@@ -483,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 for (int kk = 0; kk < C::BN / 32; ++kk) {
                     const uint64_t bdesc = desc_mn_sw32<L::KVT>(vbase + kk * 32 * kBox);
                     umma_f8_ts(tO, tPb + 16 * kk, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-                    umma_f8_ts(tO, tPb + 16 * kk + 8, bdesc, idesc_pv, 1u);
+                    if constexpr (PLO) umma_f8_ts(tO, tPb + 16 * kk + 8, bdesc, idesc_pv, 1u);
                 }
                 umma_commit(b_o_ready(j & 1));
                 umma_commit(b_kv_empty(s));
@@ -570,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 // P slot b held P(j - 2).  PV(j - 2) was issued before QK(j),
                 // and the commit that completed s_full(j) tracks every earlier
                 // MMA of the issuer, so PV(j - 2) has completed: the slot is free.
-                l_run = l_run * alpha + tile_p(r[0], r[1], tP + 32 * b, c2, nb2);
+                l_run = l_run * alpha + tile_p<PLO>(r[0], r[1], tP + 32 * b, c2, nb2);
                 if (rescale) {
                     // O holds PV(0..j-1): wait for PV(j - 1), then scale it.
                     ok = mbar_wait_bounded(b_o_ready((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag,
@@ -586,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 uint64_t l0 = f2pack(0.0f, 0.0f), l1 = l0;
                 uint32_t pk[NCH][16];
 #pragma unroll
-                for (int c = 0; c < NCH; ++c) p_chunk(r[c], c2, nb2, l0, l1, pk[c]);
+                for (int c = 0; c < NCH; ++c) p_chunk<PLO>(r[c], c2, nb2, l0, l1, pk[c]);
                 float s0, s1;
                 f2unpack(fadd2(l0, l1), s0, s1);
                 l_run = l_run * alpha + (s0 + s1);
@@ -598,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                     tc_fence_after();
                 }
 #pragma unroll
-                for (int c = 0; c < NCH; ++c) tmem_st16(tP + 16 * c, pk[c]);
+                for (int c = 0; c < NCH; ++c) tmem_st_p<PLO>(tP + 16 * c, pk[c]);
                 if (rescale) rescale_o<C::NPV>(tO, alpha);
             }
             tmem_wait_st();
@@ -682,17 +707,20 @@ fp8vit_status launch(fp8vit_ctx* ctx, const uint8_t* q8, const uint8_t* k8, cons
         !encode_map(&mv, v8, T, row_bytes, Cfg<D>::BN))
         return FP8VIT_ECUDA;
     // The dynamic shared-memory limit is a per-device setting of each kernel
-    // instance: raise it once per (device, output type).
-    static std::atomic<uint64_t> attr_set[2];
-    auto kern = out_fp8 ? attn_fwd_kernel<D, true> : attn_fwd_kernel<D, false>;
+    // instance: raise it once per (device, instance).
+    static std::atomic<uint64_t> attr_set[4];
+    const bool two_terms = ctx->attn_p_terms != 1;
+    const int inst = (out_fp8 ? 1 : 0) + (two_terms ? 2 : 0);
+    auto kern = out_fp8 ? (two_terms ? attn_fwd_kernel<D, true, true> : attn_fwd_kernel<D, true, false>)
+                        : (two_terms ? attn_fwd_kernel<D, false, true> : attn_fwd_kernel<D, false, false>);
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FP8VIT_ECUDA;
     const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
-    if (!bit || !(attr_set[out_fp8 ? 1 : 0].load() & bit)) {
+    if (!bit || !(attr_set[inst].load() & bit)) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Smem<D>::ALLOC) != cudaSuccess)
             return FP8VIT_ECUDA;
-        attr_set[out_fp8 ? 1 : 0].fetch_or(bit);
+        attr_set[inst].fetch_or(bit);
     }
     dim3 grid((unsigned)((max_seqlen + kBM - 1) / kBM), (unsigned)H, (unsigned)num_seqs);
     kern<<<grid, kThreads, Smem<D>::ALLOC, st>>>(mq, mk, mv, dq, dk, dv, cu, max_seqlen, T, H,

@@ -38,6 +38,7 @@ fp8vit_status fp8vit_create(int32_t device, fp8vit_ctx** out) {
     c->device = device;
     c->num_sms = sms;
     c->d_scratch = scr;
+    c->attn_p_terms = 2;
     *out = c;
     return FP8VIT_OK;
 }
@@ -47,6 +48,12 @@ fp8vit_status fp8vit_destroy(fp8vit_ctx* ctx) {
     cudaError_t e = cudaFree(ctx->d_scratch);
     delete ctx;
     return e == cudaSuccess ? FP8VIT_OK : FP8VIT_ECUDA;
+}
+
+fp8vit_status fp8vit_set_attn_p_terms(fp8vit_ctx* ctx, int32_t terms) {
+    if (!ctx || (terms != 1 && terms != 2)) return FP8VIT_EINVAL;
+    ctx->attn_p_terms = terms;
+    return FP8VIT_OK;
 }
 
 fp8vit_status fp8vit_check(fp8vit_ctx* ctx, void* stream, int32_t* site) {

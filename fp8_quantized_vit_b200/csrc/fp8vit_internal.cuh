@@ -24,6 +24,7 @@ struct fp8vit_ctx {
     int32_t device;
     int32_t num_sms;
     fp8vit_scratch* d_scratch;
+    int32_t attn_p_terms;  // 2 = P as e4m3 hi + lo (default), 1 = single e4m3 term
 };
 
 // Ring state layout (FP8VIT_RING_BYTES == 256).

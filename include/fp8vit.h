@@ -76,6 +76,19 @@ fp8vit_status fp8vit_check(fp8vit_ctx* ctx, void* stream, int32_t* site);
 
 const char* fp8vit_status_string(fp8vit_status s);
 
+/* How many e4m3 terms the probabilities P of fp8_varlen_attn_fwd are kept in
+ * for the PV product on this context (both run on the FP8 tensor cores):
+ *   2 (the default): P = hi + lo, hi = e4m3(p), lo = e4m3(p - hi), two PV
+ *     MMAs into one fp32 accumulator; about 8 significant bits of P.  This is
+ *     the mode that meets the attention tolerance (max-abs 3e-2 over the BF16
+ *     rounding, mean-abs 3e-3, cosine 0.999) on inputs with x8 outlier
+ *     channels.
+ *   1: P = e4m3(p) alone, 3 significant bits; one PV MMA and a cheaper
+ *     softmax.  On the same inputs its max-abs error exceeds 3e-2 several
+ *     times over (mean-abs and cosine stay inside the tolerance).
+ * Other values: FP8VIT_EINVAL.  Host only; affects later launches. */
+fp8vit_status fp8vit_set_attn_p_terms(fp8vit_ctx* ctx, int32_t terms);
+
 /* Library ABI version (major * 100 + minor). */
 int32_t fp8vit_version(void);
 

@@ -114,6 +114,16 @@ def test_scale_file_round_trip_with_margin(tmp_path):
         assert got == want
 
 
+def test_attn_p_terms_setting_is_checked_on_the_host():
+    lib = fv.lib()
+    fake_ctx = ctypes.create_string_buffer(64)  # host-only call: the struct is never on the GPU
+    assert lib.fp8vit_set_attn_p_terms(None, 2) == fv.EINVAL
+    for bad in (0, 3, -1):
+        assert lib.fp8vit_set_attn_p_terms(fake_ctx, bad) == fv.EINVAL
+    assert lib.fp8vit_set_attn_p_terms(fake_ctx, 1) == fv.OK
+    assert lib.fp8vit_set_attn_p_terms(fake_ctx, 2) == fv.OK
+
+
 def test_host_argument_checks_need_no_gpu():
     lib = fv.lib()
     fake_ctx = ctypes.create_string_buffer(64)

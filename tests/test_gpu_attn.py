@@ -18,8 +18,8 @@ import torch
 
 import oracle
 import synth
-from _helpers import (assert_attn_close, assert_fp8_out_close, bf16_bits_to_f64,
-                      code_step_distance, sample_pairs)
+from _helpers import (ATTN_COS, ATTN_MEAN_ABS, assert_attn_close, assert_fp8_out_close,
+                      attn_errors, bf16_bits_to_f64, code_step_distance, sample_pairs)
 
 pytestmark = pytest.mark.gpu
 
@@ -167,6 +167,51 @@ def test_fp8_output_c4_sampled(ctx):
     assert_fp8_out_close(g, ref, out_scale, oracle.e4m3_decode, "c4 fp8 out")
     big = np.abs(ref) >= np.abs(ref).max() / 16
     assert code_step_distance(g, want)[big].max() <= 1
+
+
+@pytest.mark.parametrize("lens,H,D,name", [((300, 129), 2, 72, None), ((513,), 2, 128, None),
+                                         (None, None, None, "c2"), (None, None, None, "c5")])
+def test_single_term_p_mode(lens, H, D, name):
+    """P as one e4m3 term (fp8vit_set_attn_p_terms(ctx, 1)): the mode takes
+    effect, stays inside the mean-abs and cosine gates, and its max-abs error
+    is reported (it exceeds the 3e-2 gate on these outlier inputs, which is
+    why two terms are the default).  Setting 2 again restores the default
+    kernel's output bit for bit."""
+    c = fv.Context()
+    if name is None:
+        cu, codes, desc = _prepare(lens, H, D, seed=sum(lens) + 7)
+        sm = np.float32(1.0 / math.sqrt(D))
+        ref = oracle.attn_full(*codes, *desc, cu, H, D, sm)
+        pick = slice(None)
+        max_seqlen = max(lens)
+    else:
+        w = synth.WORKLOADS[name]
+        H, D = w.heads, w.head_dim
+        q, k, v = w.qkv(0)
+        amax = [oracle.amax_bf16(x) for x in (q, k, v)]
+        desc = list(oracle.Ring().update(amax))
+        codes = [oracle.quantize_per_tensor(x, d).reshape(w.tokens, H, D)
+                 for x, d in zip((q, k, v), desc)]
+        cu = synth.cu_seqlens(w.seg_lens)
+        toks, hs = sample_pairs(cu, H, per_seg=24, seed=len(name))
+        ref = oracle.attn_pairs(*codes, *desc, cu, H, D, w.softmax_scale, toks, hs)
+        pick = (toks, hs)
+        max_seqlen = max(w.seg_lens)
+    two = _run_gpu(c, cu, codes, desc, H, D, max_seqlen)
+    c.set_attn_p_terms(1)
+    one = _run_gpu(c, cu, codes, desc, H, D, max_seqlen)
+    c.set_attn_p_terms(2)
+    again = _run_gpu(c, cu, codes, desc, H, D, max_seqlen)
+    assert torch.equal(two.view(torch.int16), again.view(torch.int16))
+    assert not torch.equal(two.view(torch.int16), one.view(torch.int16))
+    got1 = _gpu_bf16_to_f64(one)[pick]
+    assert not np.isnan(got1).any()
+    e1 = attn_errors(got1, ref)
+    e2 = attn_errors(_gpu_bf16_to_f64(two)[pick], ref)
+    print(name or (lens, H, D), "one term", e1, "two terms", e2)
+    assert e1["mean_abs"] <= ATTN_MEAN_ABS and e1["cos"] >= ATTN_COS, e1
+    assert e1["max_excess"] > e2["max_excess"]
+    c.close()
 
 
 def test_bad_cu_seqlens_reports_einval(ctx):
