@@ -84,8 +84,10 @@ const char* fp8vit_status_string(fp8vit_status s);
  *     rounding, mean-abs 3e-3, cosine 0.999) on inputs with x8 outlier
  *     channels.
  *   1: P = e4m3(p) alone, 3 significant bits; one PV MMA and a cheaper
- *     softmax.  On the same inputs its max-abs error exceeds 3e-2 several
- *     times over (mean-abs and cosine stay inside the tolerance).
+ *     softmax (12-18 % less attention time).  On the same inputs its max-abs
+ *     error is 3-4x the 3e-2 tolerance on images of a few hundred tokens and
+ *     just inside it on images of 8192 and more (mean-abs and cosine stay
+ *     inside the tolerance).
  * Other values: FP8VIT_EINVAL.  Host only; affects later launches. */
 fp8vit_status fp8vit_set_attn_p_terms(fp8vit_ctx* ctx, int32_t terms);
 
