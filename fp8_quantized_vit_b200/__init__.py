@@ -44,6 +44,8 @@ _SIGNATURES = {
     "fp8_quantize_qkv_per_tensor": (_I32, [_P, _P, _P, _P, _I64, _P, _P, _P, _P, _P]),
     "fp8_varlen_attn_fwd": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I64, _I32, _I32,
                                    _F32, _P, _I32, _P, _P]),
+    "fp8_varlen_attn_fwd_group_quant": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I64,
+                                               _I32, _I32, _F32, _P, _P, _P]),
     "per_token_group_quant_fp8": (_I32, [_P, _P, _I64, _I64, _I32, _P, _P, _P]),
     "fp8_static_scales_load": (_I32, [ctypes.c_char_p, ctypes.c_char_p, _P]),
     "fp8_static_scales_save": (_I32, [ctypes.c_char_p, _I32, ctypes.POINTER(ctypes.c_char_p),
@@ -254,6 +256,28 @@ def fp8_varlen_attn_fwd(q8, k8, v8, q_descale, k_descale, v_descale, cu_seqlens,
         _ptr(output_scale, torch.float32, "output_scale"), _stream(stream)),
         "fp8_varlen_attn_fwd")
     return out
+
+
+def fp8_varlen_attn_fwd_group_quant(q8, k8, v8, q_descale, k_descale, v_descale, cu_seqlens,
+                                    max_seqlen, softmax_scale, xq, scales, ctx=None, stream=None):
+    """Attention with the group-128 quantizer fused into the epilogue
+    (head_dim 128): xq e4m3 [T, H * 128], scales fp32 [T, H]; the same bytes as
+    fp8_varlen_attn_fwd (bf16 out) followed by per_token_group_quant_fp8."""
+    if q8.dim() != 3:
+        raise ValueError("q8 must be [T, H, D]")
+    T, H, D = q8.shape
+    if k8.shape != q8.shape or v8.shape != q8.shape:
+        raise ValueError("q8, k8 and v8 must have the same [T, H, D] shape")
+    if xq.numel() != T * H * D or scales.numel() != T * H * D // 128:
+        raise ValueError("xq must hold T * H * D codes and scales T * H * D / 128 floats")
+    _check(lib().fp8_varlen_attn_fwd_group_quant(
+        _ctx(ctx), _ptr(q8, _FP8, "q8"), _ptr(k8, _FP8, "k8"), _ptr(v8, _FP8, "v8"),
+        _ptr(q_descale, torch.float32, "q_descale"), _ptr(k_descale, torch.float32, "k_descale"),
+        _ptr(v_descale, torch.float32, "v_descale"), _ptr(cu_seqlens, torch.int32, "cu_seqlens"),
+        cu_seqlens.numel() - 1, int(max_seqlen), T, H, D, float(softmax_scale),
+        _ptr(xq, _FP8, "xq"), _ptr(scales, torch.float32, "scales"), _stream(stream)),
+        "fp8_varlen_attn_fwd_group_quant")
+    return xq, scales
 
 
 # ---- static scales ------------------------------------------------------------------

@@ -330,17 +330,41 @@ __device__ __forceinline__ float tile_p(const uint32_t (&a)[32], const uint32_t 
     return s0 + s1;
 }
 
-// FP8OUT selects the epilogue at compile time (e4m3 through output_scale, or
-// bf16), so each instance carries one epilogue only; PLO keeps P as two e4m3
-// terms (hi + lo, two PV MMAs) or, when false, as one.
-template <int D, bool FP8OUT, bool PLO>
+// Eight O columns of this thread's lane times inv, rounded to bf16 (RNE) and
+// packed two per word: the values the bf16 epilogue stores.
+__device__ __forceinline__ uint4 bf16x8_of_o(uint32_t taddr, float inv) {
+    uint32_t r[8];
+    tmem_ld8_sync(taddr, r);
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float(r[2 * i]) * inv,
+                                                 __uint_as_float(r[2 * i + 1]) * inv);
+        w[i] = *reinterpret_cast<uint32_t*>(&b);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Output modes, one epilogue per kernel instance.
+enum : int {
+    kOutBf16 = 0,     // o as bf16
+    kOutE4m3 = 1,     // e4m3(o / output_scale)
+    kOutGroupQ = 2,   // the bf16 o of each head quantized as one 128-wide group:
+                      // e4m3 codes + one fp32 scale per (token, head); head_dim 128
+};
+
+// OUT selects the epilogue at compile time; PLO keeps P as two e4m3 terms
+// (hi + lo, two PV MMAs) or, when false, as one.
+template <int D, int OUT, bool PLO>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ dq_p,
                     const float* __restrict__ dk_p, const float* __restrict__ dv_p,
                     const int32_t* __restrict__ cu, int32_t max_seqlen, int64_t total_tokens,
-                    int32_t num_heads, float sm_scale, void* __restrict__ out, int32_t out_fp8,
-                    const float* __restrict__ out_scale_p, fp8vit_scratch* __restrict__ scr) {
+                    int32_t num_heads, float sm_scale, void* __restrict__ out,
+                    const float* __restrict__ out_scale_p, float* __restrict__ gscales,
+                    fp8vit_scratch* __restrict__ scr) {
+    static_assert(OUT != kOutGroupQ || D == 128, "a 128-wide group is one head at head_dim 128");
     using C = Cfg<D>;
     using L = Smem<D>;
     constexpr int NS = C::NS;
@@ -643,31 +667,59 @@ __global__ void __launch_bounds__(kThreads, 2)
             const float inv = __fdiv_rn(dv, l_run);
             const int64_t tok = (int64_t)seg_start + q0 + row;
             const int64_t off = (tok * num_heads + h) * D;
-            const float oscale = FP8OUT ? *out_scale_p : 1.0f;
+            if constexpr (OUT == kOutGroupQ) {
+                // The row's bf16 output values, exactly as the bf16 epilogue
+                // would store them, quantized as one group of 128: pass 1 takes
+                // their amax, pass 2 reloads O and writes the codes.
+                uint32_t am = 0;
 #pragma unroll
-            for (int c = 0; c < D / 8; ++c) {
-                uint32_t r[8];
-                tmem_ld8_sync(tO + col_off + 8 * c, r);
-                float o[8];
+                for (int c = 0; c < D / 8; ++c) {
+                    const uint4 w = bf16x8_of_o(tO + 8 * c, inv);
+                    am = __vmaxu2(am, w.x & 0x7FFF7FFFu);
+                    am = __vmaxu2(am, w.y & 0x7FFF7FFFu);
+                    am = __vmaxu2(am, w.z & 0x7FFF7FFFu);
+                    am = __vmaxu2(am, w.w & 0x7FFF7FFFu);
+                }
+                am = max(am & 0xFFFFu, am >> 16);
+                const float sc = group_scale_of_amax(bf16_bits_to_f32(am));
+                const float nr = -__frcp_rn(sc);
+                const uint64_t s2 = f2_pack(sc, sc), nr2 = f2_pack(nr, nr);
+                uint8_t* xq = reinterpret_cast<uint8_t*>(out) + off;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) o[i] = __uint_as_float(r[i]) * inv;
-                if (!valid) continue;
-                if constexpr (FP8OUT) {
-                    uint32_t w0 = (uint32_t)f32x2_to_e4m3x2(__fdiv_rn(o[0], oscale), __fdiv_rn(o[1], oscale)) |
-                                  ((uint32_t)f32x2_to_e4m3x2(__fdiv_rn(o[2], oscale), __fdiv_rn(o[3], oscale)) << 16);
-                    uint32_t w1 = (uint32_t)f32x2_to_e4m3x2(__fdiv_rn(o[4], oscale), __fdiv_rn(o[5], oscale)) |
-                                  ((uint32_t)f32x2_to_e4m3x2(__fdiv_rn(o[6], oscale), __fdiv_rn(o[7], oscale)) << 16);
-                    *reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(out) + off + 8 * c) =
-                        make_uint2(w0, w1);
-                } else {
-                    uint32_t w[4];
+                for (int c = 0; c < D / 8; c += 2) {
+                    const uint2 a = quant8_small(bf16x8_of_o(tO + 8 * c, inv), s2, nr2);
+                    const uint2 b = quant8_small(bf16x8_of_o(tO + 8 * c + 8, inv), s2, nr2);
+                    if (valid)
+                        *reinterpret_cast<uint4*>(xq + 8 * c) = make_uint4(a.x, a.y, b.x, b.y);
+                }
+                if (valid) gscales[tok * num_heads + h] = sc;
+            } else {
+                const float oscale = OUT == kOutE4m3 ? *out_scale_p : 1.0f;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        __nv_bfloat162 b = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
-                        w[i] = *reinterpret_cast<uint32_t*>(&b);
+                for (int c = 0; c < D / 8; ++c) {
+                    uint32_t r[8];
+                    tmem_ld8_sync(tO + col_off + 8 * c, r);
+                    float o[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) o[i] = __uint_as_float(r[i]) * inv;
+                    if (!valid) continue;
+                    if constexpr (OUT == kOutE4m3) {
+                        uint32_t w0 = (uint32_t)f32x2_to_e4m3x2(__fdiv_rn(o[0], oscale), __fdiv_rn(o[1], oscale)) |
+                                      ((uint32_t)f32x2_to_e4m3x2(__fdiv_rn(o[2], oscale), __fdiv_rn(o[3], oscale)) << 16);
+                        uint32_t w1 = (uint32_t)f32x2_to_e4m3x2(__fdiv_rn(o[4], oscale), __fdiv_rn(o[5], oscale)) |
+                                      ((uint32_t)f32x2_to_e4m3x2(__fdiv_rn(o[6], oscale), __fdiv_rn(o[7], oscale)) << 16);
+                        *reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(out) + off + 8 * c) =
+                            make_uint2(w0, w1);
+                    } else {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            __nv_bfloat162 b = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
+                            w[i] = *reinterpret_cast<uint32_t*>(&b);
+                        }
+                        *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out) + off + 8 * c) =
+                            make_uint4(w[0], w[1], w[2], w[3]);
                     }
-                    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out) + off + 8 * c) =
-                        make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
         }
@@ -695,11 +747,11 @@ bool encode_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_by
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, int OUT>
 fp8vit_status launch(fp8vit_ctx* ctx, const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
                      const float* dq, const float* dk, const float* dv, const int32_t* cu,
                      int32_t num_seqs, int32_t max_seqlen, int64_t T, int32_t H, float sm_scale,
-                     void* out, int32_t out_fp8, const float* out_scale, cudaStream_t st) {
+                     void* out, const float* out_scale, float* gscales, cudaStream_t st) {
     CUtensorMap mq, mk, mv;
     const int64_t row_bytes = (int64_t)H * D;
     if (!encode_map(&mq, q8, T, row_bytes, kBM) ||
@@ -708,11 +760,10 @@ fp8vit_status launch(fp8vit_ctx* ctx, const uint8_t* q8, const uint8_t* k8, cons
         return FP8VIT_ECUDA;
     // The dynamic shared-memory limit is a per-device setting of each kernel
     // instance: raise it once per (device, instance).
-    static std::atomic<uint64_t> attr_set[4];
+    static std::atomic<uint64_t> attr_set[2];
     const bool two_terms = ctx->attn_p_terms != 1;
-    const int inst = (out_fp8 ? 1 : 0) + (two_terms ? 2 : 0);
-    auto kern = out_fp8 ? (two_terms ? attn_fwd_kernel<D, true, true> : attn_fwd_kernel<D, true, false>)
-                        : (two_terms ? attn_fwd_kernel<D, false, true> : attn_fwd_kernel<D, false, false>);
+    const int inst = two_terms ? 1 : 0;
+    auto kern = two_terms ? attn_fwd_kernel<D, OUT, true> : attn_fwd_kernel<D, OUT, false>;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FP8VIT_ECUDA;
     const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
@@ -724,7 +775,7 @@ fp8vit_status launch(fp8vit_ctx* ctx, const uint8_t* q8, const uint8_t* k8, cons
     }
     dim3 grid((unsigned)((max_seqlen + kBM - 1) / kBM), (unsigned)H, (unsigned)num_seqs);
     kern<<<grid, kThreads, Smem<D>::ALLOC, st>>>(mq, mk, mv, dq, dk, dv, cu, max_seqlen, T, H,
-                                                 sm_scale, out, out_fp8, out_scale,
+                                                 sm_scale, out, out_scale, gscales,
                                                  ctx->d_scratch);
     return cudaGetLastError() == cudaSuccess ? FP8VIT_OK : FP8VIT_ECUDA;
 }
@@ -759,10 +810,47 @@ extern "C" fp8vit_status fp8_varlen_attn_fwd(
     if (num_seqs == 0 || max_seqlen == 0 || total_tokens == 0) return FP8VIT_OK;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (head_dim == 72)
-        return launch<72>(ctx, d_q8, d_k8, d_v8, d_q_descale, d_k_descale, d_v_descale,
-                          d_cu_seqlens, num_seqs, max_seqlen, total_tokens, num_heads,
-                          softmax_scale, d_out, out_dtype, d_output_scale, st);
-    return launch<128>(ctx, d_q8, d_k8, d_v8, d_q_descale, d_k_descale, d_v_descale, d_cu_seqlens,
-                       num_seqs, max_seqlen, total_tokens, num_heads, softmax_scale, d_out,
-                       out_dtype, d_output_scale, st);
+        return out_dtype == 0
+                   ? launch<72, kOutBf16>(ctx, d_q8, d_k8, d_v8, d_q_descale, d_k_descale,
+                                          d_v_descale, d_cu_seqlens, num_seqs, max_seqlen,
+                                          total_tokens, num_heads, softmax_scale, d_out, nullptr,
+                                          nullptr, st)
+                   : launch<72, kOutE4m3>(ctx, d_q8, d_k8, d_v8, d_q_descale, d_k_descale,
+                                          d_v_descale, d_cu_seqlens, num_seqs, max_seqlen,
+                                          total_tokens, num_heads, softmax_scale, d_out,
+                                          d_output_scale, nullptr, st);
+    return out_dtype == 0
+               ? launch<128, kOutBf16>(ctx, d_q8, d_k8, d_v8, d_q_descale, d_k_descale,
+                                       d_v_descale, d_cu_seqlens, num_seqs, max_seqlen,
+                                       total_tokens, num_heads, softmax_scale, d_out, nullptr,
+                                       nullptr, st)
+               : launch<128, kOutE4m3>(ctx, d_q8, d_k8, d_v8, d_q_descale, d_k_descale,
+                                       d_v_descale, d_cu_seqlens, num_seqs, max_seqlen,
+                                       total_tokens, num_heads, softmax_scale, d_out,
+                                       d_output_scale, nullptr, st);
+}
+
+extern "C" fp8vit_status fp8_varlen_attn_fwd_group_quant(
+    fp8vit_ctx* ctx, const uint8_t* d_q8, const uint8_t* d_k8, const uint8_t* d_v8,
+    const float* d_q_descale, const float* d_k_descale, const float* d_v_descale,
+    const int32_t* d_cu_seqlens, int32_t num_seqs, int32_t max_seqlen, int64_t total_tokens,
+    int32_t num_heads, int32_t head_dim, float softmax_scale, uint8_t* d_xq, float* d_scales,
+    void* stream) {
+    if (!ctx || !d_q8 || !d_k8 || !d_v8 || !d_q_descale || !d_k_descale || !d_v_descale ||
+        !d_cu_seqlens || !d_xq || !d_scales)
+        return FP8VIT_EINVAL;
+    if (num_seqs < 0 || max_seqlen < 0 || total_tokens < 0 || total_tokens > INT32_MAX ||
+        num_heads < 1)
+        return FP8VIT_EINVAL;
+    if (!(softmax_scale > 0.0f) || !isfinite(softmax_scale)) return FP8VIT_EINVAL;
+    if (head_dim != 128) return FP8VIT_EUNSUPPORTED;
+    if (misaligned(d_q8, 16) || misaligned(d_k8, 16) || misaligned(d_v8, 16) ||
+        misaligned(d_xq, 16) || misaligned(d_scales, 4) || misaligned(d_cu_seqlens, 4))
+        return FP8VIT_EINVAL;
+    if (num_heads > 65535 || num_seqs > 65535) return FP8VIT_EUNSUPPORTED;
+    if (num_seqs == 0 || max_seqlen == 0 || total_tokens == 0) return FP8VIT_OK;
+    return launch<128, kOutGroupQ>(ctx, d_q8, d_k8, d_v8, d_q_descale, d_k_descale, d_v_descale,
+                                   d_cu_seqlens, num_seqs, max_seqlen, total_tokens, num_heads,
+                                   softmax_scale, d_xq, nullptr, d_scales,
+                                   reinterpret_cast<cudaStream_t>(stream));
 }

@@ -78,6 +78,67 @@ __device__ __forceinline__ float2 e4m3x2_to_f32x2(uint16_t v) {
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
 
 // ---------------------------------------------------------------------------
+// Per-token-group quantization arithmetic (atrex-bench "#025
+// per_token_group_quant_fp8": scale = max(amax / 448, 1e-10), code =
+// e4m3(clamp(x / scale, +-448))), shared by the group quantizer and the
+// attention epilogue that fuses it, so both produce the same bytes.
+// ---------------------------------------------------------------------------
+
+// packed fp32 pairs (sm_100a f32x2 arithmetic)
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// The group scale max(amax / 448, 1e-10) with the IEEE fp32 quotient, formed
+// without a divide: q0 = RN(amax * RN(1/448)) and one FMA correction
+// (Markstein, IBM J. Res. Dev. 34(1), 1990); exact for every non-negative
+// finite bf16 amax (checked with exact rational arithmetic over all 32640).
+__device__ __forceinline__ float group_scale_of_amax(float af) {
+    const float q0 = __fmul_rn(af, 1.0f / 448.0f);
+    const float sc = __fmaf_rn(__fmaf_rn(-448.0f, q0, af), 1.0f / 448.0f, q0);
+    return sc > 1e-10f ? sc : 1e-10f;
+}
+
+// 8 bf16 / scale -> 8 e4m3 codes for quotients known to stay below 1024 in
+// magnitude (inside a group |x| <= amax = 448 * scale), given s2 = (s, s)
+// and nr2 = -(RN(1/s)) twice; two lanes per instruction, computed on -x:
+//   q0 = RN((-x) * (-r)),  e = RN(q0 * s - x) (exact),  q = RN(q0 - e * r),
+// the correctly rounded quotient (Markstein).  Working on -x keeps the sign
+// of a zero quotient (x = -0 gives q = -0 and code 0x80) without a copysign:
+// the only cancellation is q0 + (-0) terms, which then carry the operand's sign.
+__device__ __forceinline__ uint2 quant8_small(const uint4& x, uint64_t s2, uint64_t nr2) {
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t c[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float nlo = __uint_as_float((w[i] << 16) ^ 0x80000000u);
+        const float nhi = __uint_as_float((w[i] & 0xFFFF0000u) ^ 0x80000000u);
+        const uint64_t nx = f2_pack(nlo, nhi);
+        const uint64_t q0 = f2_mul(nx, nr2);
+        const uint64_t e = f2_fma(q0, s2, nx);
+        float qlo, qhi;
+        f2_unpack(f2_fma(e, nr2, q0), qlo, qhi);
+        c[i] = f32x2_to_e4m3x2(qlo, qhi);
+    }
+    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+// ---------------------------------------------------------------------------
 // sm_100a PTX wrappers
 // ---------------------------------------------------------------------------
 

@@ -161,50 +161,6 @@ __device__ __forceinline__ uint2 quant8(const uint4& x, float s, float r) {
     return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
-// ---- packed fp32 pairs (sm_100a f32x2 arithmetic) ----
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-
-// 8 bf16 / scale -> 8 e4m3 codes for quotients known to stay below 1024 in
-// magnitude (the group quantizer: |x| <= the group's amax = 448 * scale).
-// Same quotient as div_by_scale, two lanes per instruction, computed on -x:
-//   q0 = RN((-x) * (-r)),  e = RN(q0 * s - x) (exact),  q = RN(q0 - e * r).
-// Working on -x keeps the sign of a zero quotient (x = -0 gives q = -0 and
-// code 0x80) without a copysign: the only cancellation is q0 + (-0) terms,
-// which then carry the operand's sign.
-__device__ __forceinline__ uint2 quant8_small(const uint4& x, uint64_t s2, uint64_t nr2) {
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-    uint32_t c[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float nlo = __uint_as_float((w[i] << 16) ^ 0x80000000u);
-        const float nhi = __uint_as_float((w[i] & 0xFFFF0000u) ^ 0x80000000u);
-        const uint64_t nx = f2_pack(nlo, nhi);
-        const uint64_t q0 = f2_mul(nx, nr2);
-        const uint64_t e = f2_fma(q0, s2, nx);
-        float qlo, qhi;
-        f2_unpack(f2_fma(e, nr2, q0), qlo, qhi);
-        c[i] = f32x2_to_e4m3x2(qlo, qhi);
-    }
-    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
-}
-
 // One tensor's grid-stride share: four 16-byte loads in flight per thread.
 __device__ __forceinline__ void quant_share(const uint4* __restrict__ p, uint2* __restrict__ o,
                                             int64_t n_elems, float s) {
@@ -267,12 +223,7 @@ __global__ void __launch_bounds__(kGroupThreads) group_quant_kernel(
 #pragma unroll
             for (int off = LPG / 2; off > 0; off >>= 1)
                 a = max(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
-            // amax / 448 in IEEE fp32: Markstein with RN(1/448), exact for
-            // every non-negative bf16 amax
-            const float af = bf16_bits_to_f32(a);
-            const float q0 = __fmul_rn(af, 1.0f / 448.0f);
-            float sc = __fmaf_rn(__fmaf_rn(-448.0f, q0, af), 1.0f / 448.0f, q0);
-            sc = sc > 1e-10f ? sc : 1e-10f;
+            const float sc = group_scale_of_amax(bf16_bits_to_f32(a));
             if (g < total_groups) {
                 const float nr = -__frcp_rn(sc);
                 __stcs(xq + g * LPG + gl, quant8_small(xv[u], f2_pack(sc, sc), f2_pack(nr, nr)));

@@ -198,6 +198,27 @@ fp8vit_status fp8_varlen_attn_fwd(fp8vit_ctx* ctx, const uint8_t* d_q8, const ui
                                   int32_t head_dim, float softmax_scale, void* d_out,
                                   int32_t out_dtype, const float* d_output_scale, void* stream);
 
+/* fp8_varlen_attn_fwd with the per-token-group quantizer fused into its
+ * epilogue (vLLM issue "fused fp8 output for FlashAttention 3": the output
+ * quantization moves into the attention kernel; atrex-bench "#025
+ * per_token_group_quant_fp8": group 128, fp32 scales, the o-proj input).
+ * head_dim must be 128, so that each 128-column group of a token row of
+ * [total_tokens, num_heads * 128] is exactly one head (head_dim 72 groups
+ * straddle heads: FP8VIT_EUNSUPPORTED; use fp8_varlen_attn_fwd plus
+ * per_token_group_quant_fp8).  The attention output is rounded to BF16 as
+ * fp8_varlen_attn_fwd's out_dtype 0 stores it, then quantized exactly as
+ * per_token_group_quant_fp8(group = 128) does: the bytes of d_xq and the bits
+ * of d_scales equal those two calls' results, and no BF16 output is written.
+ * d_xq: e4m3 [total_tokens, num_heads * 128], 16-byte aligned.
+ * d_scales: fp32 [total_tokens, num_heads], 4-byte aligned.
+ * Other arguments, checks and faults as fp8_varlen_attn_fwd. */
+fp8vit_status fp8_varlen_attn_fwd_group_quant(
+    fp8vit_ctx* ctx, const uint8_t* d_q8, const uint8_t* d_k8, const uint8_t* d_v8,
+    const float* d_q_descale, const float* d_k_descale, const float* d_v_descale,
+    const int32_t* d_cu_seqlens, int32_t num_seqs, int32_t max_seqlen, int64_t total_tokens,
+    int32_t num_heads, int32_t head_dim, float softmax_scale, uint8_t* d_xq, float* d_scales,
+    void* stream);
+
 /* ---- per-token-group quantizer (atrex-bench "#025 per_token_group_quant_fp8",
  *      Reference Implementation) --------------------------------------------- */
 

@@ -149,6 +149,16 @@ def test_host_argument_checks_need_no_gpu():
     odd = ctypes.c_void_p(0x10001)
     assert lib.fp8_varlen_attn_fwd(fake_ctx, odd, dummy, dummy, dummy, dummy, dummy, dummy, 1,
                                    8, 8, 2, 72, 0.1, dummy, 0, None, None) == fv.EINVAL
+    # fused attention + group quant: head_dim 72 (groups straddle heads), null outputs
+    assert lib.fp8_varlen_attn_fwd_group_quant(fake_ctx, dummy, dummy, dummy, dummy, dummy, dummy,
+                                               dummy, 1, 8, 8, 2, 72, 0.1, dummy, dummy,
+                                               None) == fv.EUNSUPPORTED
+    assert lib.fp8_varlen_attn_fwd_group_quant(fake_ctx, dummy, dummy, dummy, dummy, dummy, dummy,
+                                               dummy, 1, 8, 8, 2, 128, 0.1, None, dummy,
+                                               None) == fv.EINVAL
+    assert lib.fp8_varlen_attn_fwd_group_quant(fake_ctx, dummy, dummy, dummy, dummy, dummy, dummy,
+                                               dummy, 1, 8, 8, 2, 128, 0.1, dummy, odd,
+                                               None) == fv.EINVAL
     # group quant: n not a multiple of group, unsupported group
     assert lib.per_token_group_quant_fp8(fake_ctx, dummy, 4, 200, 128, dummy, dummy,
                                          None) == fv.EINVAL

@@ -253,3 +253,52 @@ def test_end_to_end_dynamic_pipeline(ctx):
         assert (layer.descale.cpu().numpy().view(np.uint32) ==
                 np.asarray(desc, np.float32).view(np.uint32)).all()
         assert_attn_close(_gpu_bf16_to_f64(out), ref, f"forward {f}")
+
+
+@pytest.mark.parametrize("lens,H,name", [((513, 129, 0, 300), 2, None), ((1,), 1, None),
+                                         (None, None, "c2")])
+def test_fused_group_quant(ctx, lens, H, name):
+    """fp8_varlen_attn_fwd_group_quant (head_dim 128) writes, byte for byte and
+    bit for bit, what the oracle's group quantizer (group 128) gives for the
+    kernel's own BF16 attention output; that BF16 output is gated against the
+    fp64 oracle attention here as everywhere else, and the fused result equals
+    the two-kernel path (attention, then per_token_group_quant_fp8)."""
+    D = 128
+    if name is None:
+        cu, codes, desc = _prepare(lens, H, D, seed=sum(lens) + 11)
+        max_seqlen, sm = max(lens), np.float32(1.0 / math.sqrt(D))
+    else:
+        w = synth.WORKLOADS[name]
+        H = w.heads
+        q, k, v = w.qkv(0)
+        desc = list(oracle.Ring().update([oracle.amax_bf16(x) for x in (q, k, v)]))
+        codes = [oracle.quantize_per_tensor(x, d).reshape(w.tokens, H, D)
+                 for x, d in zip((q, k, v), desc)]
+        cu = synth.cu_seqlens(w.seg_lens)
+        max_seqlen, sm = max(w.seg_lens), w.softmax_scale
+    T = codes[0].shape[0]
+    out = _run_gpu(ctx, cu, codes, desc, H, D, max_seqlen)
+    got = _gpu_bf16_to_f64(out)
+    if name is None:
+        assert_attn_close(got, oracle.attn_full(*codes, *desc, cu, H, D, sm), (lens, H))
+    else:
+        toks, hs = sample_pairs(cu, H, per_seg=24, seed=9)
+        ref = oracle.attn_pairs(*codes, *desc, cu, H, D, sm, toks, hs)
+        assert_attn_close(got[toks, hs], ref, name)
+    want_q, want_s = oracle.group_quant(out.view(torch.int16).cpu().numpy().view(np.uint16)
+                                        .reshape(T, H * D), 128)
+    q8, k8, v8 = (_dev(c) for c in codes)
+    d = [torch.tensor([x], dtype=torch.float32, device="cuda") for x in desc]
+    cu_d = _dev(cu)
+    xq = torch.full((T, H * D), 0x7F, dtype=torch.uint8, device="cuda")
+    xs = torch.full((T, H), float("nan"), dtype=torch.float32, device="cuda")
+    fv.fp8_varlen_attn_fwd_group_quant(q8, k8, v8, d[0], d[1], d[2], cu_d, max_seqlen, sm, xq, xs,
+                                       ctx=ctx)
+    st, site = ctx.check()
+    assert st == fv.OK, (fv.status_string(st), site)
+    assert np.array_equal(xq.cpu().numpy(), want_q)
+    assert np.array_equal(xs.cpu().numpy().view(np.uint32), want_s.view(np.uint32))
+    xq2 = torch.empty_like(xq)
+    xs2 = torch.empty_like(xs)
+    fv.per_token_group_quant_fp8(out.view(T, H * D), 128, xq2, xs2, ctx=ctx)
+    assert torch.equal(xq, xq2) and torch.equal(xs.view(torch.int32), xs2.view(torch.int32))
