@@ -42,6 +42,7 @@ _SIGNATURES = {
     "fp8_amax3": (_I32, [_P, _P, _P, _P, _I64, _P, _P]),
     "fp8_ring_push": (_I32, [_P, _P, _P, _P]),
     "fp8_quantize_qkv_per_tensor": (_I32, [_P, _P, _P, _P, _I64, _P, _P, _P, _P, _P]),
+    "fp8_amax_ring_quantize_qkv": (_I32, [_P, _P, _P, _P, _I64, _P, _P, _P, _P, _P, _P]),
     "fp8_varlen_attn_fwd": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I64, _I32, _I32,
                                    _F32, _P, _I32, _P, _P]),
     "fp8_varlen_attn_fwd_group_quant": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I64,
@@ -224,6 +225,21 @@ def fp8_quantize_qkv_per_tensor(q, k, v, descale3, q8, k8, v8, ctx=None, stream=
     return q8, k8, v8
 
 
+def fp8_amax_ring_quantize_qkv(q, k, v, ring, descale3, q8, k8, v8, ctx=None, stream=None):
+    """fp8_amax_ring_update followed by fp8_quantize_qkv_per_tensor in one
+    cooperative launch (same ring state, descales and codes)."""
+    n = q.numel()
+    for t in (k, v, q8, k8, v8):
+        if t.numel() != n:
+            raise ValueError("all tensors must have the same number of elements")
+    _check(lib().fp8_amax_ring_quantize_qkv(
+        _ctx(ctx), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+        _ptr(v, torch.bfloat16, "v"), n, _ptr(ring, torch.float32, "ring"),
+        _ptr(descale3, torch.float32, "descale3"), _ptr(q8, _FP8, "q8"), _ptr(k8, _FP8, "k8"),
+        _ptr(v8, _FP8, "v8"), _stream(stream)), "fp8_amax_ring_quantize_qkv")
+    return q8, k8, v8
+
+
 def per_token_group_quant_fp8(x, group, xq, scales, ctx=None, stream=None):
     if x.dim() != 2:
         raise ValueError("x must be [m, n]")
@@ -309,6 +325,7 @@ class FP8EncoderAttention:
     Holds the layer's scale state (a device ring for dynamic scaling, or
     static descales), and runs
         [amax ring update] -> per-tensor quantize -> varlen FP8 attention
+    (the first two as one cooperative launch on one GPU)
         [-> per-token-group quantize of the BF16 output]
     on the current stream.  Intermediate FP8 buffers are allocated once per
     token count and reused (no allocation per call at steady state).
@@ -371,10 +388,13 @@ class FP8EncoderAttention:
             fp8_amax3(q, k, v, self._amax3, ctx=self.ctx)
             allreduce_amax3(self._amax3, self.process_group)
             fp8_ring_push(self._amax3, self.ring, self.descale)
-        elif self.ring is not None:
-            fp8_amax_ring_update(q, k, v, self.ring, self.descale, ctx=self.ctx)
-        fp8_quantize_qkv_per_tensor(q, k, v, self.descale, b["q8"], b["k8"], b["v8"],
-                                    ctx=self.ctx)
+        if self.ring is not None and self.process_group is None:
+            # amax, ring rule and quantization in one cooperative launch
+            fp8_amax_ring_quantize_qkv(q, k, v, self.ring, self.descale, b["q8"], b["k8"],
+                                       b["v8"], ctx=self.ctx)
+        else:
+            fp8_quantize_qkv_per_tensor(q, k, v, self.descale, b["q8"], b["k8"], b["v8"],
+                                        ctx=self.ctx)
         o = b["out"] if out is None else out
         fp8_varlen_attn_fwd(b["q8"], b["k8"], b["v8"], self.descale[0:1], self.descale[1:2],
                             self.descale[2:3], cu_seqlens, max_seqlen, self.softmax_scale, o,

@@ -27,6 +27,8 @@ fp8vit_status fp8vit_create(int32_t device, fp8vit_ctx** out) {
     FP8VIT_CUDA_TRY(cudaSetDevice(device));
     int sms = 0;
     FP8VIT_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device));
+    int l2 = 0;
+    FP8VIT_CUDA_TRY(cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, device));
     fp8vit_scratch* scr = nullptr;
     FP8VIT_CUDA_TRY(cudaMalloc(&scr, sizeof(fp8vit_scratch)));
     if (cudaMemset(scr, 0, sizeof(fp8vit_scratch)) != cudaSuccess ||
@@ -39,6 +41,7 @@ fp8vit_status fp8vit_create(int32_t device, fp8vit_ctx** out) {
     c->num_sms = sms;
     c->d_scratch = scr;
     c->attn_p_terms = 2;
+    c->l2_bytes = l2;
     *out = c;
     return FP8VIT_OK;
 }

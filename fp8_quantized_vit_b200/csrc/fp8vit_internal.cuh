@@ -17,7 +17,9 @@ struct fp8vit_scratch {
     int32_t site;          // kernel-specific location code of that fault
     uint32_t amax_bits[3]; // running |x| maxima (bf16 bit patterns) of q, k, v
     uint32_t arrivals;     // CTAs of the current amax launch that have finished
-    uint32_t pad[26];      // to 128 bytes
+    uint32_t release;      // generation counter of the fused amax/quantize grid barrier
+    float descale[3];      // descales published across that barrier
+    uint32_t pad[22];      // to 128 bytes
 };
 
 struct fp8vit_ctx {
@@ -25,6 +27,7 @@ struct fp8vit_ctx {
     int32_t num_sms;
     fp8vit_scratch* d_scratch;
     int32_t attn_p_terms;  // 2 = P as e4m3 hi + lo (default), 1 = single e4m3 term
+    int64_t l2_bytes;      // the device's L2 size
 };
 
 // Ring state layout (FP8VIT_RING_BYTES == 256).
@@ -41,6 +44,8 @@ static_assert(sizeof(fp8vit_ring) == FP8VIT_RING_BYTES, "ring layout");
         if (e_ != cudaSuccess) return FP8VIT_ECUDA;    \
     } while (0)
 
+static_assert(sizeof(fp8vit_scratch) == 128, "scratch layout");
+
 // Site codes recorded with a device fault.
 enum : int32_t {
     SITE_ATTN_SEQLENS = 100,
@@ -54,6 +59,7 @@ enum : int32_t {
     SITE_ATTN_WAIT_QREADY = 117,
     SITE_ATTN_DRAIN = 118,
     SITE_ATTN_WAIT_SFREE = 119,
+    SITE_QUANT_BARRIER = 200,
 };
 
 __device__ __forceinline__ void fp8vit_report(fp8vit_scratch* s, int32_t status, int32_t site) {

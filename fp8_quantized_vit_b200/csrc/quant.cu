@@ -32,6 +32,27 @@ __device__ __forceinline__ uint32_t absmax_vec(uint32_t acc, const uint4& x) {
     return absmax2(acc, x.w);
 }
 
+// 16-byte load that asks L2 to keep the line (evict_last priority): the
+// fused amax/quantize kernel reads each vector again right after.
+__device__ __forceinline__ uint64_t keep_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ uint4 ld_keep(const uint4* p, uint64_t pol) {
+    uint4 v;
+    asm volatile("ld.global.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p), "l"(pol));
+    return v;
+}
+
+template <bool KEEP>
+__device__ __forceinline__ uint4 ld_amax(const uint4* p, uint64_t pol) {
+    if constexpr (KEEP) return ld_keep(p, pol);
+    else return __ldcs(p);
+}
+
 // |x| max of one tensor over this thread's grid-stride share, four 16-byte
 // loads in flight per thread.
 __device__ __forceinline__ uint32_t amax_share(const uint4* __restrict__ p, int64_t n_elems) {
@@ -194,6 +215,177 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quant3_kernel(
     quant_share(v, v8, n_elems, descale3[2]);
 }
 
+// amax + ring rule + quantize in one launch, for the dynamic-scale path.
+// The launch is cooperative (every block resident at once), so the blocks can
+// meet at a grid barrier: phase 1 reduces the three amaxes as
+// amax_ring_kernel does; the last block to arrive runs the ring rule and
+// publishes the descales in the scratch; the others wait for the barrier's
+// generation counter to move (bounded: a timeout records FP8VIT_ETIMEOUT
+// and the block returns); phase 2 quantizes as quant3_kernel does.  The BF16
+// tensors are read twice; KEEP (chosen when the three tensors fit in L2)
+// loads them with evict_last priority in phase 1, and phase 2 quantizes the
+// most recently read tensor first, so its reads come from L2.
+constexpr uint64_t kBarrierTimeoutNs = 2000000000ull;
+
+// |x| maxima of q, k and v over this thread's grid-stride share in one loop:
+// six 16-byte loads in flight per thread (two vectors of each tensor), so
+// tensors of a few tens of MB, where each thread owns only a dozen vectors,
+// do not pay three separate load ramps.
+template <bool KEEP>
+__device__ __forceinline__ void amax3_share(const uint4* __restrict__ q,
+                                            const uint4* __restrict__ k,
+                                            const uint4* __restrict__ v, int64_t n_elems,
+                                            uint32_t (&m)[3]) {
+    const int64_t nvec = n_elems >> 3;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const uint64_t pol = KEEP ? keep_policy() : 0;
+    uint32_t a[3] = {0u, 0u, 0u}, b[3] = {0u, 0u, 0u};
+    for (; i + stride < nvec; i += 2 * stride) {
+        const uint4 q0 = ld_amax<KEEP>(q + i, pol), k0 = ld_amax<KEEP>(k + i, pol);
+        const uint4 v0 = ld_amax<KEEP>(v + i, pol), q1 = ld_amax<KEEP>(q + i + stride, pol);
+        const uint4 k1 = ld_amax<KEEP>(k + i + stride, pol);
+        const uint4 v1 = ld_amax<KEEP>(v + i + stride, pol);
+        a[0] = absmax_vec(a[0], q0);
+        a[1] = absmax_vec(a[1], k0);
+        a[2] = absmax_vec(a[2], v0);
+        b[0] = absmax_vec(b[0], q1);
+        b[1] = absmax_vec(b[1], k1);
+        b[2] = absmax_vec(b[2], v1);
+    }
+    if (i < nvec) {
+        a[0] = absmax_vec(a[0], ld_amax<KEEP>(q + i, pol));
+        a[1] = absmax_vec(a[1], ld_amax<KEEP>(k + i, pol));
+        a[2] = absmax_vec(a[2], ld_amax<KEEP>(v + i, pol));
+    }
+    const int tail = (int)(n_elems & 7);
+    if (blockIdx.x == 0 && (int)threadIdx.x < tail) {
+        const int64_t e = (nvec << 3) + threadIdx.x;
+        a[0] = absmax2(a[0], reinterpret_cast<const uint16_t*>(q)[e]);
+        a[1] = absmax2(a[1], reinterpret_cast<const uint16_t*>(k)[e]);
+        a[2] = absmax2(a[2], reinterpret_cast<const uint16_t*>(v)[e]);
+    }
+#pragma unroll
+    for (int t = 0; t < 3; ++t) {
+        const uint32_t c = __vmaxu2(a[t], b[t]);
+        m[t] = max(c & 0xFFFFu, c >> 16);
+    }
+}
+
+// quant_share for q, k and v in one loop (v, k, q order: in the fused kernel
+// the tensor read last in phase 1 is the likeliest to still be in L2).
+__device__ __forceinline__ void quant3_share(const uint4* __restrict__ q,
+                                             const uint4* __restrict__ k,
+                                             const uint4* __restrict__ v, uint2* __restrict__ q8,
+                                             uint2* __restrict__ k8, uint2* __restrict__ v8,
+                                             int64_t n_elems, const float (&s)[3]) {
+    const float rq = __frcp_rn(s[0]), rk = __frcp_rn(s[1]), rv = __frcp_rn(s[2]);
+    const int64_t nvec = n_elems >> 3;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (; i + stride < nvec; i += 2 * stride) {
+        const uint4 v0 = __ldcs(v + i), k0 = __ldcs(k + i), q0 = __ldcs(q + i);
+        const uint4 v1 = __ldcs(v + i + stride), k1 = __ldcs(k + i + stride);
+        const uint4 q1 = __ldcs(q + i + stride);
+        __stcs(v8 + i, quant8(v0, s[2], rv));
+        __stcs(k8 + i, quant8(k0, s[1], rk));
+        __stcs(q8 + i, quant8(q0, s[0], rq));
+        __stcs(v8 + i + stride, quant8(v1, s[2], rv));
+        __stcs(k8 + i + stride, quant8(k1, s[1], rk));
+        __stcs(q8 + i + stride, quant8(q1, s[0], rq));
+    }
+    if (i < nvec) {
+        __stcs(v8 + i, quant8(__ldcs(v + i), s[2], rv));
+        __stcs(k8 + i, quant8(__ldcs(k + i), s[1], rk));
+        __stcs(q8 + i, quant8(__ldcs(q + i), s[0], rq));
+    }
+    const int tail = (int)(n_elems & 7);
+    if (blockIdx.x == 0 && (int)threadIdx.x < tail) {
+        const int64_t e = (nvec << 3) + threadIdx.x;
+        const uint4* src[3] = {q, k, v};
+        uint2* dst[3] = {q8, k8, v8};
+        const float r[3] = {rq, rk, rv};
+#pragma unroll
+        for (int t = 0; t < 3; ++t) {
+            const float y = div_by_scale(
+                bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(src[t])[e]), s[t], r[t]);
+            reinterpret_cast<uint8_t*>(dst[t])[e] = (uint8_t)(f32x2_to_e4m3x2(y, 0.0f) & 0xFF);
+        }
+    }
+}
+
+template <bool KEEP>
+__global__ void __launch_bounds__(kQuantThreads, 4) amax_ring_quant_kernel(
+    const uint4* __restrict__ q, const uint4* __restrict__ k, const uint4* __restrict__ v,
+    int64_t n_elems, fp8vit_ring* __restrict__ ring, float* __restrict__ descale3,
+    uint2* __restrict__ q8, uint2* __restrict__ k8, uint2* __restrict__ v8,
+    fp8vit_scratch* __restrict__ scr) {
+    __shared__ uint32_t red[3][kQuantThreads / 32];
+    __shared__ float sdesc[3];
+    __shared__ int proceed;
+    volatile uint32_t* release = &scr->release;
+    // The generation before this launch's barrier: read before this block
+    // arrives, so the last block cannot have advanced it yet.
+    const uint32_t gen0 = threadIdx.x == 0 ? *release : 0u;
+    uint32_t m[3];
+    amax3_share<KEEP>(q, k, v, n_elems, m);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int t = 0; t < 3; ++t) {
+        uint32_t w = __reduce_max_sync(0xFFFFFFFFu, m[t]);
+        if (lane == 0) red[t][warp] = w;
+    }
+    __syncthreads();
+    if (warp == 0) {
+#pragma unroll
+        for (int t = 0; t < 3; ++t) {
+            uint32_t x = lane < (int)(blockDim.x >> 5) ? red[t][lane] : 0u;
+            x = __reduce_max_sync(0xFFFFFFFFu, x);
+            if (lane == 0) atomicMax(&scr->amax_bits[t], x);
+        }
+    }
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned ticket = atomicAdd(&scr->arrivals, 1u);
+        int go = 1;
+        if (ticket == gridDim.x - 1) {
+            // Every other block's atomicMax is visible: take and clear the
+            // maxima, run the ring rule, publish the descales, release.
+            __threadfence();
+            float amax[3];
+#pragma unroll
+            for (int t = 0; t < 3; ++t)
+                amax[t] = bf16_bits_to_f32(atomicExch(&scr->amax_bits[t], 0u));
+            atomicExch(&scr->arrivals, 0u);
+            ring_rule(ring, amax, descale3);
+            volatile float* pub = scr->descale;
+#pragma unroll
+            for (int t = 0; t < 3; ++t) pub[t] = descale3[t];
+            __threadfence();
+            atomicAdd(&scr->release, 1u);
+        } else {
+            const uint64_t t0 = globaltimer_ns();
+            while (*release == gen0) {
+                if (globaltimer_ns() - t0 > kBarrierTimeoutNs) {
+                    fp8vit_report(scr, FP8VIT_ETIMEOUT, SITE_QUANT_BARRIER);
+                    go = 0;
+                    break;
+                }
+                __nanosleep(64);
+            }
+            __threadfence();
+        }
+        const volatile float* pub = scr->descale;
+#pragma unroll
+        for (int t = 0; t < 3; ++t) sdesc[t] = pub[t];
+        proceed = go;
+    }
+    __syncthreads();
+    if (!proceed) return;
+    const float s3[3] = {sdesc[0], sdesc[1], sdesc[2]};
+    quant3_share(q, k, v, q8, k8, v8, n_elems, s3);
+}
+
 // LPG = lanes per group = group / 8; each lane owns one 16-byte vector of
 // its group; a warp covers 32 / LPG groups per step and keeps kUnroll steps
 // (kUnroll loads per lane) in flight.
@@ -327,6 +519,43 @@ fp8vit_status fp8_quantize_qkv_per_tensor(fp8vit_ctx* ctx, const uint16_t* d_q,
         reinterpret_cast<const uint4*>(d_v), n_elems, d_descale3, reinterpret_cast<uint2*>(d_q8),
         reinterpret_cast<uint2*>(d_k8), reinterpret_cast<uint2*>(d_v8));
     return cudaGetLastError() == cudaSuccess ? FP8VIT_OK : FP8VIT_ECUDA;
+}
+
+fp8vit_status fp8_amax_ring_quantize_qkv(fp8vit_ctx* ctx, const uint16_t* d_q,
+                                         const uint16_t* d_k, const uint16_t* d_v,
+                                         int64_t n_elems, void* d_ring, float* d_descale3,
+                                         uint8_t* d_q8, uint8_t* d_k8, uint8_t* d_v8,
+                                         void* stream) {
+    if (!ctx || !d_q || !d_k || !d_v || !d_ring || !d_descale3 || !d_q8 || !d_k8 || !d_v8 ||
+        n_elems < 0)
+        return FP8VIT_EINVAL;
+    if (misaligned(d_q, 16) || misaligned(d_k, 16) || misaligned(d_v, 16) ||
+        misaligned(d_ring, 16) || misaligned(d_descale3, 4) || misaligned(d_q8, 8) ||
+        misaligned(d_k8, 8) || misaligned(d_v8, 8))
+        return FP8VIT_EINVAL;
+    // Keep the BF16 lines in L2 between the two phases when the three tensors
+    // fill at most 3/4 of it (room for the codes written meanwhile).
+    const bool keep = n_elems <= ctx->l2_bytes / 8;
+    auto kern = keep ? amax_ring_quant_kernel<true> : amax_ring_quant_kernel<false>;
+    // one resident wave, which the cooperative launch requires anyway
+    const int per_sm = resident_blocks((const void*)kern, kQuantThreads);
+    const int grid = grid_for(n_elems >> 3, kQuantThreads, 4, per_sm * ctx->num_sms);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kQuantThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(
+        &cfg, kern, reinterpret_cast<const uint4*>(d_q),
+        reinterpret_cast<const uint4*>(d_k), reinterpret_cast<const uint4*>(d_v), n_elems,
+        reinterpret_cast<fp8vit_ring*>(d_ring), d_descale3, reinterpret_cast<uint2*>(d_q8),
+        reinterpret_cast<uint2*>(d_k8), reinterpret_cast<uint2*>(d_v8), ctx->d_scratch);
+    return e == cudaSuccess ? FP8VIT_OK : FP8VIT_ECUDA;
 }
 
 fp8vit_status per_token_group_quant_fp8(fp8vit_ctx* ctx, const uint16_t* d_x, int64_t m,

@@ -170,6 +170,24 @@ fp8vit_status fp8_quantize_qkv_per_tensor(fp8vit_ctx* ctx, const uint16_t* d_q,
                                           int64_t n_elems, const float* d_descale3, uint8_t* d_q8,
                                           uint8_t* d_k8, uint8_t* d_v8, void* stream);
 
+/* The dynamic-scale path in one launch (vLLM "FP8 ViT Encoder Attention":
+ * Usage, dynamic scaling; intro: Q/K/V quantized right before attention):
+ * exactly fp8_amax_ring_update(d_q, d_k, d_v, n_elems, d_ring, d_descale3)
+ * followed by fp8_quantize_qkv_per_tensor(..., d_descale3, d_q8, d_k8,
+ * d_v8): the same ring update, descales and codes, bit for bit.  The kernel
+ * is launched cooperatively (all its blocks resident at once) and meets at a
+ * grid barrier between the amax and the quantization, so the three small
+ * scale stages cost no extra launch and, when the BF16 tensors fit in L2,
+ * their second read comes from it.  A barrier wait that exceeds 2 s records
+ * FP8VIT_ETIMEOUT (read it with fp8vit_check) and leaves the codes unwritten.
+ * Alignment and ownership as the two calls; uses the context's scratch (one
+ * stream per context at a time). */
+fp8vit_status fp8_amax_ring_quantize_qkv(fp8vit_ctx* ctx, const uint16_t* d_q,
+                                         const uint16_t* d_k, const uint16_t* d_v,
+                                         int64_t n_elems, void* d_ring, float* d_descale3,
+                                         uint8_t* d_q8, uint8_t* d_k8, uint8_t* d_v8,
+                                         void* stream);
+
 /* ---- varlen FP8 attention (vLLM "FP8 ViT Encoder Attention"; vLLM issue
  *      "fused fp8 output for FlashAttention 3") ------------------------------ */
 

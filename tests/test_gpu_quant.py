@@ -257,3 +257,61 @@ def test_group_quant_every_bf16_value(ctx, group):
     bad = np.nonzero(got != want_q)
     assert bad[0].size == 0, (bad[0][:5], bad[1][:5], got[bad][:5], want_q[bad][:5])
     assert (_f32_bits(sc.cpu().numpy()) == _f32_bits(want_s)).all()
+
+
+def test_fused_amax_ring_quantize_over_20_forwards(ctx):
+    """fp8_amax_ring_quantize_qkv (one cooperative launch) over the 20
+    forwards of the 8192-token, head_dim-128 workload (the ring wraps after
+    16): every forward's descales, ring contents and e4m3 codes equal the
+    oracle's ring + quantizer bit for bit, and the two-call path's."""
+    w = synth.WORKLOADS["c2"]
+    n = w.tokens * w.hd
+    ring_f, ring_2 = fv.new_ring(), fv.new_ring()
+    desc_f = torch.zeros(3, dtype=torch.float32, device="cuda")
+    desc_2 = torch.zeros(3, dtype=torch.float32, device="cuda")
+    out_f = [torch.empty(n, dtype=torch.uint8, device="cuda") for _ in range(3)]
+    out_2 = [torch.empty(n, dtype=torch.uint8, device="cuda") for _ in range(3)]
+    ring_o = oracle.Ring()
+    for f in range(20):
+        x = w.qkv(f)
+        dev = [_dev_bf16(a).reshape(-1) for a in x]
+        want = ring_o.update([oracle.amax_bf16(a) for a in x])
+        fv.fp8_amax_ring_quantize_qkv(*dev, ring_f, desc_f, *out_f, ctx=ctx)
+        fv.fp8_amax_ring_update(*dev, ring_2, desc_2, ctx=ctx)
+        fv.fp8_quantize_qkv_per_tensor(*dev, desc_2, *out_2, ctx=ctx)
+        assert (_f32_bits(desc_f.cpu().numpy()) == _f32_bits(want)).all(), f
+        r = ring_f.cpu().numpy()
+        assert (_f32_bits(r[:48].reshape(3, 16)) == _f32_bits(ring_o.hist)).all(), f
+        assert r[48:49].view(np.int32)[0] == ring_o.pos[0]
+        assert torch.equal(ring_f, ring_2)
+        for t in range(3):
+            assert torch.equal(out_f[t], out_2[t]), (f, t)
+        if f in (0, 16):  # spot-check the codes against the oracle quantizer
+            for t in range(3):
+                assert np.array_equal(_host_u8(out_f[t]),
+                                      oracle.quantize_per_tensor(x[t], want[t]).reshape(-1)), (f, t)
+    _check_ok(ctx)
+
+
+@pytest.mark.parametrize("n", [0, 1, 7, 8, 9, 8 * 1000 + 5, 1 << 20, 3 * (1 << 22) + 3])
+def test_fused_amax_ring_quantize_ragged_sizes(ctx, n):
+    """Ragged lengths (tails below one 16-byte vector, a grid larger than
+    one block's share): codes and descales equal the oracle's bit for bit."""
+    bits = [np.ascontiguousarray(synth.bf16_tensor(synth.stream_key(n + 5, 1, t), 1, max(n, 1))[0, :n])
+            for t in range(3)]
+    if n:
+        for t in range(3):
+            bits[t][-1] = np.uint16(0xC2F0 + t)  # the largest magnitude sits in the tail
+    ring_d = fv.new_ring()
+    desc_d = torch.zeros(3, dtype=torch.float32, device="cuda")
+    dev = [_dev_bf16(b) if n else torch.empty(8, dtype=torch.bfloat16, device="cuda") for b in bits]
+    out = [torch.full((max(n, 8),), 0x7F, dtype=torch.uint8, device="cuda") for _ in range(3)]
+    assert fv.lib().fp8_amax_ring_quantize_qkv(
+        ctx.handle, dev[0].data_ptr(), dev[1].data_ptr(), dev[2].data_ptr(), n,
+        ring_d.data_ptr(), desc_d.data_ptr(), out[0].data_ptr(), out[1].data_ptr(),
+        out[2].data_ptr(), fv._stream()) == fv.OK
+    _check_ok(ctx)
+    want = oracle.Ring().update([oracle.amax_bf16(b) for b in bits])
+    assert (_f32_bits(desc_d.cpu().numpy()) == _f32_bits(want)).all()
+    for t in range(3):
+        assert np.array_equal(_host_u8(out[t])[:n], oracle.quantize_per_tensor(bits[t], want[t]))
