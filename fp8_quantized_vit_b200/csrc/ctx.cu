@@ -1,4 +1,5 @@
 // Context lifecycle, status reporting and the small host helpers of the ABI.
+#include <cstddef>
 #include <mutex>
 
 #include "fp8vit_internal.cuh"
@@ -68,11 +69,28 @@ fp8vit_status fp8vit_check(fp8vit_ctx* ctx, void* stream, int32_t* site) {
     FP8VIT_CUDA_TRY(cudaMemcpyAsync(hv, ctx->d_scratch, sizeof(hv), cudaMemcpyDeviceToHost, st));
     FP8VIT_CUDA_TRY(cudaStreamSynchronize(st));
     if (hv[0] != 0) {
-        FP8VIT_CUDA_TRY(cudaMemsetAsync(ctx->d_scratch, 0, sizeof(hv), st));
+        // A kernel gave up: clear the status word and the amax reduction state
+        // (maxima, arrival counter), which a launch that timed out can leave
+        // half-updated.  The stream is idle, and a context serves one stream.
+        FP8VIT_CUDA_TRY(cudaMemsetAsync(ctx->d_scratch, 0,
+                                        offsetof(fp8vit_scratch, release), st));
         FP8VIT_CUDA_TRY(cudaStreamSynchronize(st));
     }
     if (site) *site = hv[1];
     return static_cast<fp8vit_status>(hv[0]);
+}
+
+fp8vit_status fp8vit_inject_lost_arrival(fp8vit_ctx* ctx, void* stream) {
+    if (!ctx) return FP8VIT_EINVAL;
+    // An arrival count no block can complete: the next fused amax/quantize
+    // launch on this context finds no last block, so its barrier wait runs out.
+    const uint32_t bogus = 0x40000000u;
+    FP8VIT_CUDA_TRY(cudaMemcpyAsync(reinterpret_cast<uint8_t*>(ctx->d_scratch) +
+                                        offsetof(fp8vit_scratch, arrivals),
+                                    &bogus, sizeof(bogus), cudaMemcpyHostToDevice,
+                                    reinterpret_cast<cudaStream_t>(stream)));
+    FP8VIT_CUDA_TRY(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+    return FP8VIT_OK;
 }
 
 fp8vit_status fp8vit_ring_init(void* d_ring, void* stream) {

@@ -71,10 +71,21 @@ fp8vit_status fp8vit_destroy(fp8vit_ctx* ctx);
 
 /* Synchronize `stream`, then return and clear the first fault recorded on the
  * device since the last check (FP8VIT_OK if none).  *site, if not NULL,
- * receives a kernel-specific location code of that fault (0 if none). */
+ * receives a kernel-specific location code of that fault (0 if none).  After
+ * a fault it also resets the context's amax reduction state, which a launch
+ * that gave up can leave half-updated. */
 fp8vit_status fp8vit_check(fp8vit_ctx* ctx, void* stream, int32_t* site);
 
 const char* fp8vit_status_string(fp8vit_status s);
+
+/* Failure injection for tests, on the host side: record on the context an
+ * arrival that never happens, so that the next fp8_amax_ring_quantize_qkv on
+ * it cannot complete its grid barrier.  Each of that launch's blocks gives up
+ * after its bounded 2 s wait and returns; fp8vit_check then reports
+ * FP8VIT_ETIMEOUT (site 200) and resets the context's reduction state, after
+ * which the context works normally.  No GPU fault is involved.  Synchronizes
+ * `stream`.  Not for production use. */
+fp8vit_status fp8vit_inject_lost_arrival(fp8vit_ctx* ctx, void* stream);
 
 /* How many e4m3 terms the probabilities P of fp8_varlen_attn_fwd are kept in
  * for the PV product on this context (both run on the FP8 tensor cores):

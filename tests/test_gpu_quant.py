@@ -315,3 +315,30 @@ def test_fused_amax_ring_quantize_ragged_sizes(ctx, n):
     assert (_f32_bits(desc_d.cpu().numpy()) == _f32_bits(want)).all()
     for t in range(3):
         assert np.array_equal(_host_u8(out[t])[:n], oracle.quantize_per_tensor(bits[t], want[t]))
+
+
+def test_fused_barrier_timeout_is_reported_and_recovered():
+    """A lost arrival (injected on the host) makes the fused kernel's grid
+    barrier wait run out: every block gives up after its bounded wait and
+    returns, fp8vit_check reports FP8VIT_ETIMEOUT at site 200 and resets the
+    reduction state, and the next call on the same context is bit-exact."""
+    c = fv.Context()
+    x = [synth.bf16_tensor(synth.stream_key(31, 0, t), 64, 1152) for t in range(3)]
+    dev = [_dev_bf16(a).reshape(-1) for a in x]
+    n = dev[0].numel()
+    out = [torch.empty(n, dtype=torch.uint8, device="cuda") for _ in range(3)]
+    ring_d = fv.new_ring()
+    desc_d = torch.zeros(3, dtype=torch.float32, device="cuda")
+    assert fv.lib().fp8vit_inject_lost_arrival(c.handle, fv._stream()) == fv.OK
+    fv.fp8_amax_ring_quantize_qkv(*dev, ring_d, desc_d, *out, ctx=c)
+    st, site = c.check()
+    assert st == fv.ETIMEOUT and site == 200, (fv.status_string(st), site)
+    assert c.check() == (fv.OK, 0)  # the fault was cleared
+    ring_d = fv.new_ring()
+    fv.fp8_amax_ring_quantize_qkv(*dev, ring_d, desc_d, *out, ctx=c)
+    _check_ok(c)
+    want = oracle.Ring().update([oracle.amax_bf16(a) for a in x])
+    assert (_f32_bits(desc_d.cpu().numpy()) == _f32_bits(want)).all()
+    for t in range(3):
+        assert np.array_equal(_host_u8(out[t]), oracle.quantize_per_tensor(x[t], want[t]).reshape(-1))
+    c.close()
