@@ -55,6 +55,8 @@ def _load_signatures(lib):
         "orc_attn_full": (ctypes.c_int, [_P, _P, _P, _F32, _F32, _F32, _P, _I32, _I32, _I32,
                                          _F32, _P]),
         "orc_fp8_output": (None, [_P, _I64, _F32, _P]),
+        "orc_attn_pairs_bf16": (ctypes.c_int, [_P, _P, _P, _P, _I32, _I32, _I32, _F32, _P, _P,
+                                               _I64, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -202,6 +204,40 @@ def attn_full(q8, k8, v8, dq, dk, dv, cu_seqlens, heads: int, head_dim: int,
                                heads, head_dim, float(sm_scale), out.ctypes.data)
     if rc != 0:
         raise ValueError(f"orc_attn_full failed ({rc})")
+    return out
+
+
+def attn_pairs_bf16(q, k, v, cu_seqlens, heads: int, head_dim: int, sm_scale: float, tokens,
+                    head_ids, want_psum: bool = False):
+    """fp64 attention over BF16 inputs (bit patterns, [T, H*D] or [T, H, D])
+    for the (token, head) pairs; returns out [n, D] (and the probability sums)."""
+    q, pq = _c(q, np.uint16)
+    k, pk = _c(k, np.uint16)
+    v, pv = _c(v, np.uint16)
+    cu, pc = _c(cu_seqlens, np.int32)
+    toks, pt = _c(tokens, np.int64)
+    hs, ph = _c(head_ids, np.int32)
+    n = toks.size
+    out = np.empty((n, head_dim), dtype=np.float64)
+    psum = np.empty(n, dtype=np.float64) if want_psum else None
+    rc = _load().orc_attn_pairs_bf16(pq, pk, pv, pc, cu.size - 1, heads, head_dim,
+                                     float(sm_scale), pt, ph, n, out.ctypes.data,
+                                     psum.ctypes.data if want_psum else None)
+    if rc != 0:
+        raise ValueError(f"orc_attn_pairs_bf16 failed ({rc})")
+    return (out, psum) if want_psum else out
+
+
+def attn_full_bf16(q, k, v, cu_seqlens, heads: int, head_dim: int, sm_scale: float) -> np.ndarray:
+    """fp64 attention over BF16 inputs for every token and head; returns [T, H, D]."""
+    cu = np.asarray(cu_seqlens, dtype=np.int32)
+    T = int(cu[-1])
+    toks = np.repeat(np.arange(int(cu[0]), T, dtype=np.int64), heads)
+    hs = np.tile(np.arange(heads, dtype=np.int32), T - int(cu[0]))
+    out = np.zeros((T, heads, head_dim), dtype=np.float64)
+    if toks.size:
+        out[int(cu[0]):] = attn_pairs_bf16(q, k, v, cu, heads, head_dim, sm_scale, toks,
+                                           hs).reshape(T - int(cu[0]), heads, head_dim)
     return out
 
 

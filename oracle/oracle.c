@@ -315,6 +315,74 @@ int orc_attn_full(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, float
     return rc;
 }
 
+/* ------------------------------------------------------------------------ */
+/* fp64 varlen attention over BF16 tensors: the BF16 side of the pages'     */
+/* BF16-vs-FP8 attention comparison [vLLM-FP8ViT, Performance]             */
+/* ------------------------------------------------------------------------ */
+
+/* As orc_attn_pairs, with q, k, v given as BF16 bit patterns [T, H, D] and no
+ * descales: s_j = sm_scale * sum_d q[t,h,d] * k[j,h,d]; p = softmax(s);
+ * o[d] = sum_j p_j * v[j,h,d]; all in fp64. */
+int orc_attn_pairs_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                        const int32_t* cu_seqlens, int32_t num_seqs, int32_t H, int32_t D,
+                        float sm_scale, const int64_t* tokens, const int32_t* heads,
+                        int64_t n_pairs, double* out, double* psum) {
+    int32_t max_len = 0;
+    for (int32_t i = 0; i < num_seqs; ++i) {
+        int32_t len = cu_seqlens[i + 1] - cu_seqlens[i];
+        if (len > max_len) max_len = len;
+    }
+    double* s = (double*)malloc(sizeof(double) * (size_t)(max_len > 0 ? max_len : 1));
+    double* qv = (double*)malloc(sizeof(double) * (size_t)D);
+    if (!s || !qv) {
+        free(s);
+        free(qv);
+        return -2;
+    }
+    const int64_t row = (int64_t)H * D;
+    int rc = 0;
+    for (int64_t n = 0; n < n_pairs; ++n) {
+        int64_t t = tokens[n];
+        int32_t h = heads[n];
+        int32_t seg = orc_segment_of(cu_seqlens, num_seqs, t);
+        if (seg < 0 || h < 0 || h >= H) {
+            rc = -1;
+            break;
+        }
+        int64_t a = cu_seqlens[seg], b = cu_seqlens[seg + 1];
+        for (int32_t d = 0; d < D; ++d)
+            qv[d] = (double)orc_bf16_to_float(q[t * row + (int64_t)h * D + d]);
+        double smax = -INFINITY;
+        for (int64_t j = a; j < b; ++j) {
+            const uint16_t* kj = k + j * row + (int64_t)h * D;
+            double acc = 0.0;
+            for (int32_t d = 0; d < D; ++d) acc += qv[d] * (double)orc_bf16_to_float(kj[d]);
+            s[j - a] = (double)sm_scale * acc;
+            if (s[j - a] > smax) smax = s[j - a];
+        }
+        double l = 0.0;
+        for (int64_t j = a; j < b; ++j) {
+            s[j - a] = exp(s[j - a] - smax);
+            l += s[j - a];
+        }
+        double* o = out + n * D;
+        for (int32_t d = 0; d < D; ++d) o[d] = 0.0;
+        for (int64_t j = a; j < b; ++j) {
+            const uint16_t* vj = v + j * row + (int64_t)h * D;
+            double p = s[j - a] / l;
+            for (int32_t d = 0; d < D; ++d) o[d] += p * (double)orc_bf16_to_float(vj[d]);
+        }
+        if (psum) {
+            double ps = 0.0;
+            for (int64_t j = a; j < b; ++j) ps += s[j - a] / l;
+            psum[n] = ps;
+        }
+    }
+    free(s);
+    free(qv);
+    return rc;
+}
+
 /* FP8 output reference [vLLM-29920]: out8 = e4m3(float(o) / output_scale). */
 void orc_fp8_output(const double* o, int64_t n, float output_scale, uint8_t* out8) {
     for (int64_t i = 0; i < n; ++i) out8[i] = orc_e4m3_encode((float)o[i] / output_scale);
