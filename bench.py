@@ -252,6 +252,33 @@ def _sdpa_comparator(w, inputs, dev, reps=10):
             "ms": ms, "tflops": w.attn_flops() / (ms * 1e-3) / 1e12}
 
 
+def _bf16_comparator(fv, ctx, w, inputs, dev, reps=10):
+    """This library's BF16 attention kernel (same skeleton as the FP8 one,
+    kind::f16 MMAs) on the same BF16 inputs: the BF16 side of the pages'
+    BF16-vs-FP8 comparison, for context, not the metric."""
+    import torch
+    import synth
+    T, H, D = w.tokens, w.heads, w.head_dim
+    q, k, v = inputs[0]
+    cu = torch.from_numpy(synth.cu_seqlens(w.seg_lens)).to(dev)
+    out = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    run = lambda: fv.bf16_varlen_attn_fwd(q, k, v, cu, max(w.seg_lens), w.softmax_scale, out,
+                                          ctx=ctx)
+    for _ in range(2):
+        run()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    return {"impl": "bf16_varlen_attn_fwd (this library, kind::f16)", "ms": ms,
+            "tflops": w.attn_flops() / (ms * 1e-3) / 1e12}
+
+
 def _quant_rooflines(fv, ctx, src, dev, hbm_gbs, reps=10):
     """HBM roofline of the three quantizer kernels on 3 x 32400-token, 16-head,
     head_dim-72 tensors ([97200, 1152] BF16 each, 224 MB): the resident BF16
@@ -491,6 +518,8 @@ def run_ours(args):
     }
     if args.compare_sdpa:
         line["comparator"] = _sdpa_comparator(w, inputs, dev)
+    if args.compare_bf16:
+        line["comparator_bf16_same_skeleton"] = _bf16_comparator(fv, ctx, w, inputs, dev)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         codes, dsc = _oracle_inputs(w)
         threads = _host_threads()
@@ -530,6 +559,8 @@ def main():
                          "the attention tolerance; 1: a single term, faster, less accurate)")
     ap.add_argument("--compare-sdpa", action="store_true",
                     help="also time torch BF16 SDPA on the same inputs (single-image workloads)")
+    ap.add_argument("--compare-bf16", action="store_true",
+                    help="also time this library's BF16 attention kernel on the same inputs")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

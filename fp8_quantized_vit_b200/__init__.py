@@ -46,6 +46,8 @@ _SIGNATURES = {
     "fp8_amax_ring_quantize_qkv": (_I32, [_P, _P, _P, _P, _I64, _P, _P, _P, _P, _P, _P]),
     "fp8_varlen_attn_fwd": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I64, _I32, _I32,
                                    _F32, _P, _I32, _P, _P]),
+    "bf16_varlen_attn_fwd": (_I32, [_P, _P, _P, _P, _P, _I32, _I32, _I64, _I32, _I32, _F32, _P,
+                                    _P]),
     "fp8_varlen_attn_fwd_group_quant": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I64,
                                                _I32, _I32, _F32, _P, _P, _P]),
     "per_token_group_quant_fp8": (_I32, [_P, _P, _I64, _I64, _I32, _P, _P, _P]),
@@ -272,6 +274,23 @@ def fp8_varlen_attn_fwd(q8, k8, v8, q_descale, k_descale, v_descale, cu_seqlens,
         _ptr(out, _FP8 if fp8_out else torch.bfloat16, "out"), 1 if fp8_out else 0,
         _ptr(output_scale, torch.float32, "output_scale"), _stream(stream)),
         "fp8_varlen_attn_fwd")
+    return out
+
+
+def bf16_varlen_attn_fwd(q, k, v, cu_seqlens, max_seqlen, softmax_scale, out, ctx=None,
+                         stream=None):
+    """BF16 attention on the same kernel skeleton (the comparator of the FP8
+    path): q, k, v, out BF16 [T, H, D]."""
+    if q.dim() != 3:
+        raise ValueError("q must be [T, H, D]")
+    T, H, D = q.shape
+    if k.shape != q.shape or v.shape != q.shape or out.shape != q.shape:
+        raise ValueError("q, k, v and out must have the same [T, H, D] shape")
+    _check(lib().bf16_varlen_attn_fwd(
+        _ctx(ctx), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+        _ptr(v, torch.bfloat16, "v"), _ptr(cu_seqlens, torch.int32, "cu_seqlens"),
+        cu_seqlens.numel() - 1, int(max_seqlen), T, H, D, float(softmax_scale),
+        _ptr(out, torch.bfloat16, "out"), _stream(stream)), "bf16_varlen_attn_fwd")
     return out
 
 

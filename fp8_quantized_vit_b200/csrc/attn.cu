@@ -32,6 +32,7 @@
 #include <math.h>
 
 #include <atomic>
+#include <type_traits>
 
 #include "fp8vit_internal.cuh"
 
@@ -73,16 +74,39 @@ struct Cfg<128> {
     static constexpr uint32_t TS = 0, TP = 64, TO = 128;
 };
 
+// BF16 inputs (the same skeleton with kind::f16 MMAs): a 32-byte box column
+// holds 16 elements, so the QK contraction takes KB = 8 k-blocks at
+// head_dim 128 and 5 at head_dim 72 (a 160-byte window over the head's 144
+// bytes; its last 16 bytes are zeroed in Q), V takes VA atoms of 16
+// columns, and one PV MMA covers 16 keys.  P (BF16) occupies the same TMEM
+// columns as the two e4m3 terms.  Stages: what two CTAs per SM leave room for.
 template <int D>
-struct Smem {
+struct CfgB;
+template <>
+struct CfgB<72> {
+    static constexpr int KB = 5, VA = 5, NPV = 80, NS = 3, BN = 96, PSLOTS = 1;
+    static constexpr uint32_t TS = 0, TP = 96, TO = 144;
+};
+template <>
+struct CfgB<128> {
+    static constexpr int KB = 8, VA = 8, NPV = 128, NS = 2, BN = 64, PSLOTS = 2;
+    static constexpr uint32_t TS = 0, TP = 64, TO = 128;
+};
+
+template <class C>
+struct SmemOf {
     static constexpr int Q = 0;
-    static constexpr int K = Q + Cfg<D>::KB * kQTileBytes;
-    static constexpr int KVT = kBox * Cfg<D>::BN;  // one [BN rows x 32 B] K or V box
-    static constexpr int V = K + Cfg<D>::NS * Cfg<D>::KB * KVT;
-    static constexpr int BAR = V + Cfg<D>::NS * Cfg<D>::VA * KVT;
+    static constexpr int K = Q + C::KB * kQTileBytes;
+    static constexpr int KVT = kBox * C::BN;  // one [BN rows x 32 B] K or V box
+    static constexpr int V = K + C::NS * C::KB * KVT;
+    static constexpr int BAR = V + C::NS * C::VA * KVT;
     static constexpr int TOTAL = BAR + 256;
     static constexpr int ALLOC = TOTAL + 1024;  // slack for 1024-byte alignment
 };
+template <int D>
+using Smem = SmemOf<Cfg<D>>;
+template <int D, bool BF>
+using CfgOf = std::conditional_t<BF, CfgB<D>, Cfg<D>>;
 
 // Shared-memory matrix descriptors (tcgen05 "version 1" format), 32-byte
 // swizzle.  K-major: rows of 32 bytes, 8-row groups 256 bytes apart (SBO).
@@ -102,6 +126,32 @@ __device__ __forceinline__ uint64_t desc_mn_sw32(uint32_t addr) {
 __host__ __device__ constexpr uint32_t idesc_e4m3(int n, bool b_mn_major) {
     return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(n >> 3) << 17) |
            ((uint32_t)(128 >> 4) << 24);
+}
+// Instruction descriptor, kind::f16: bf16 x bf16 -> f32 (A and B format
+// fields = 1), M = 128.
+__host__ __device__ constexpr uint32_t idesc_bf16(int n, bool b_mn_major) {
+    return idesc_e4m3(n, b_mn_major) | (1u << 7) | (1u << 10);
+}
+
+// D[tmem] (+)= A * B, kind::f16 (both operands bf16), issued by one thread;
+// A from shared memory (descriptor) or from TMEM.
+__device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
 __device__ __forceinline__ void tmem_ld8_sync(uint32_t taddr, uint32_t (&r)[8]) {
@@ -330,6 +380,45 @@ __device__ __forceinline__ float tile_p(const uint32_t (&a)[32], const uint32_t 
     return s0 + s1;
 }
 
+// BF16 probabilities of one 32-key chunk: p = 2^(s * c - bias), summed into
+// the packed accumulators, rounded to bf16 (RNE) two per word (key 2w in the
+// low half), 16 words = TMEM columns [0, 16) of the chunk.
+__device__ __forceinline__ void p_chunk_bf16(const uint32_t (&r)[32], uint64_t c2, uint64_t nb2,
+                                             uint64_t& l0, uint64_t& l1, uint32_t (&pk)[16]) {
+    float p[32];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        float x0, x1;
+        f2unpack(ffma2(f2pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), c2, nb2),
+                 x0, x1);
+        p[2 * i] = ex2_approx(x0);
+        p[2 * i + 1] = ex2_approx(x1);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+        l0 = fadd2(l0, f2pack(p[2 * i], p[2 * i + 1]));
+        l1 = fadd2(l1, f2pack(p[2 * i + 2], p[2 * i + 3]));
+    }
+#pragma unroll
+    for (int w = 0; w < 16; ++w) {
+        __nv_bfloat162 b = __floats2bfloat162_rn(p[2 * w], p[2 * w + 1]);
+        pk[w] = *reinterpret_cast<uint32_t*>(&b);
+    }
+}
+
+// P chunk into TMEM for either input type; returns nothing, sums accumulate.
+template <bool BF, bool PLO>
+__device__ __forceinline__ void p_chunk_any(const uint32_t (&r)[32], uint64_t c2, uint64_t nb2,
+                                            uint64_t& l0, uint64_t& l1, uint32_t (&pk)[16]) {
+    if constexpr (BF) p_chunk_bf16(r, c2, nb2, l0, l1, pk);
+    else p_chunk<PLO>(r, c2, nb2, l0, l1, pk);
+}
+template <bool BF, bool PLO>
+__device__ __forceinline__ void tmem_st_p_any(uint32_t taddr, const uint32_t (&pk)[16]) {
+    if constexpr (BF) tmem_st16(taddr, pk);
+    else tmem_st_p<PLO>(taddr, pk);
+}
+
 // Eight O columns of this thread's lane times inv, rounded to bf16 (RNE) and
 // packed two per word: the values the bf16 epilogue stores.
 __device__ __forceinline__ uint4 bf16x8_of_o(uint32_t taddr, float inv) {
@@ -354,8 +443,9 @@ enum : int {
 };
 
 // OUT selects the epilogue at compile time; PLO keeps P as two e4m3 terms
-// (hi + lo, two PV MMAs) or, when false, as one.
-template <int D, int OUT, bool PLO>
+// (hi + lo, two PV MMAs) or, when false, as one.  BF: the inputs are BF16
+// (no descales) and both products run as kind::f16 MMAs with P in BF16.
+template <int D, int OUT, bool PLO, bool BF = false>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ dq_p,
@@ -365,8 +455,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                     const float* __restrict__ out_scale_p, float* __restrict__ gscales,
                     fp8vit_scratch* __restrict__ scr) {
     static_assert(OUT != kOutGroupQ || D == 128, "a 128-wide group is one head at head_dim 128");
-    using C = Cfg<D>;
-    using L = Smem<D>;
+    static_assert(!BF || OUT == kOutBf16, "bf16 inputs: bf16 output");
+    using C = CfgOf<D, BF>;
+    using L = SmemOf<C>;
+    constexpr int E = BF ? 2 : 1;  // bytes per element
     constexpr int NS = C::NS;
 
     const int qt = blockIdx.x, h = blockIdx.y, seg = blockIdx.z;
@@ -438,8 +530,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t tmem = *tmem_slot;
 
     // x coordinate (bytes) of the head's window: head offset rounded down to 16.
-    const int32_t x0 = (h * D) & ~15;
-    const int col_off = h * D - x0;  // 0, or 8 for odd heads at D = 72
+    const int32_t x0 = (h * D * E) & ~15;
+    const int col_off = (h * D * E - x0) / E;  // 0, or 8 for odd heads at D = 72 (e4m3)
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -483,17 +575,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         // P(j) is waited for, so the tensor cores compute the next scores
         // while the softmax warps work on the current ones.
         if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_e4m3(C::BN, false);
-            constexpr uint32_t idesc_pv = idesc_e4m3(C::NPV, true);
+            constexpr uint32_t idesc_qk = BF ? idesc_bf16(C::BN, false) : idesc_e4m3(C::BN, false);
+            constexpr uint32_t idesc_pv = BF ? idesc_bf16(C::NPV, true) : idesc_e4m3(C::NPV, true);
             const uint32_t tO = tmem + C::TO;
             auto issue_qk = [&](int j) {
                 const int s = j % NS;
                 const uint32_t tSb = tmem + C::TS;
 #pragma unroll
-                for (int kb = 0; kb < C::KB; ++kb)
-                    umma_f8_ss(tSb, desc_k_sw32(sQ + kb * kQTileBytes),
-                               desc_k_sw32(sK + (s * C::KB + kb) * L::KVT), idesc_qk,
-                               kb > 0 ? 1u : 0u);
+                for (int kb = 0; kb < C::KB; ++kb) {
+                    const uint64_t ad = desc_k_sw32(sQ + kb * kQTileBytes);
+                    const uint64_t bd = desc_k_sw32(sK + (s * C::KB + kb) * L::KVT);
+                    if constexpr (BF) umma_bf16_ss(tSb, ad, bd, idesc_qk, kb > 0 ? 1u : 0u);
+                    else umma_f8_ss(tSb, ad, bd, idesc_qk, kb > 0 ? 1u : 0u);
+                }
                 umma_commit(b_s_full);
             };
             bool ok = mbar_wait_bounded(b_q_ready, 0, abort_flag, scr, SITE_ATTN_WAIT_QREADY,
@@ -531,8 +625,15 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 32; ++kk) {
                     const uint64_t bdesc = desc_mn_sw32<L::KVT>(vbase + kk * 32 * kBox);
-                    umma_f8_ts(tO, tPb + 16 * kk, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-                    if constexpr (PLO) umma_f8_ts(tO, tPb + 16 * kk + 8, bdesc, idesc_pv, 1u);
+                    if constexpr (BF) {
+                        // keys 32kk..32kk+15 at P columns +0, the next 16 keys at +8
+                        const uint64_t bdesc2 = desc_mn_sw32<L::KVT>(vbase + (kk * 32 + 16) * kBox);
+                        umma_bf16_ts(tO, tPb + 16 * kk, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                        umma_bf16_ts(tO, tPb + 16 * kk + 8, bdesc2, idesc_pv, 1u);
+                    } else {
+                        umma_f8_ts(tO, tPb + 16 * kk, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                        if constexpr (PLO) umma_f8_ts(tO, tPb + 16 * kk + 8, bdesc, idesc_pv, 1u);
+                    }
                 }
                 umma_commit(b_o_ready(j & 1));
                 umma_commit(b_kv_empty(s));
@@ -549,12 +650,18 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int row = quarter * 32 + lane;  // query row in the tile == TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         const uint32_t tS = lane_base + C::TS, tP = lane_base + C::TP, tO = lane_base + C::TO;
-        const float dq = *dq_p, dk = *dk_p, dv = *dv_p;
+        const float dq = BF ? 1.0f : *dq_p, dk = BF ? 1.0f : *dk_p, dv = BF ? 1.0f : *dv_p;
         const float scale_log2 = sm_scale * dq * dk * 1.4426950408889634f;
 
         bool ok = mbar_wait_bounded(b_q_full, 0, abort_flag, scr, SITE_ATTN_WAIT_Q, kTimeoutNs);
         ok = __all_sync(0xFFFFFFFFu, ok);
-        if (ok && D == 72) {
+        if (ok && D == 72 && BF) {
+            // BF16: the 160-byte window's last 16 bytes (chunk 1 of k-block 4)
+            // belong to the next head.
+            const int sw = (row >> 2) & 1;
+            *reinterpret_cast<uint4*>(sm + L::Q + 4 * kQTileBytes + row * kBox + ((1 ^ sw) << 4)) =
+                make_uint4(0, 0, 0, 0);
+        } else if (ok && D == 72) {
             // Zero the window bytes outside this head: [72,96) for even heads,
             // [0,8) and [80,96) for odd heads.  SW32 layout: row r of k-block
             // kb at kb*4096 + r*32, 16-byte chunk c stored at chunk c ^ ((r>>2)&1).
@@ -619,7 +726,19 @@ __global__ void __launch_bounds__(kThreads, 2)
                 // P slot b held P(j - 2).  PV(j - 2) was issued before QK(j),
                 // and the commit that completed s_full(j) tracks every earlier
                 // MMA of the issuer, so PV(j - 2) has completed: the slot is free.
-                l_run = l_run * alpha + tile_p<PLO>(r[0], r[1], tP + 32 * b, c2, nb2);
+                if constexpr (BF) {
+                    uint32_t pk[16];
+                    uint64_t l0 = f2pack(0.0f, 0.0f), l1 = l0;
+                    p_chunk_bf16(r[0], c2, nb2, l0, l1, pk);
+                    tmem_st16(tP + 32 * b, pk);
+                    p_chunk_bf16(r[1], c2, nb2, l0, l1, pk);
+                    tmem_st16(tP + 32 * b + 16, pk);
+                    float s0, s1;
+                    f2unpack(fadd2(l0, l1), s0, s1);
+                    l_run = l_run * alpha + (s0 + s1);
+                } else {
+                    l_run = l_run * alpha + tile_p<PLO>(r[0], r[1], tP + 32 * b, c2, nb2);
+                }
                 if (rescale) {
                     // O holds PV(0..j-1): wait for PV(j - 1), then scale it.
                     ok = mbar_wait_bounded(b_o_ready((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag,
@@ -635,7 +754,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 uint64_t l0 = f2pack(0.0f, 0.0f), l1 = l0;
                 uint32_t pk[NCH][16];
 #pragma unroll
-                for (int c = 0; c < NCH; ++c) p_chunk<PLO>(r[c], c2, nb2, l0, l1, pk[c]);
+                for (int c = 0; c < NCH; ++c) p_chunk_any<BF, PLO>(r[c], c2, nb2, l0, l1, pk[c]);
                 float s0, s1;
                 f2unpack(fadd2(l0, l1), s0, s1);
                 l_run = l_run * alpha + (s0 + s1);
@@ -647,7 +766,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                     tc_fence_after();
                 }
 #pragma unroll
-                for (int c = 0; c < NCH; ++c) tmem_st_p<PLO>(tP + 16 * c, pk[c]);
+                for (int c = 0; c < NCH; ++c) tmem_st_p_any<BF, PLO>(tP + 16 * c, pk[c]);
                 if (rescale) rescale_o<C::NPV>(tO, alpha);
             }
             tmem_wait_st();
@@ -780,6 +899,35 @@ fp8vit_status launch(fp8vit_ctx* ctx, const uint8_t* q8, const uint8_t* k8, cons
     return cudaGetLastError() == cudaSuccess ? FP8VIT_OK : FP8VIT_ECUDA;
 }
 
+template <int D>
+fp8vit_status launch_bf16(fp8vit_ctx* ctx, const uint16_t* q, const uint16_t* k,
+                          const uint16_t* v, const int32_t* cu, int32_t num_seqs,
+                          int32_t max_seqlen, int64_t T, int32_t H, float sm_scale, void* out,
+                          cudaStream_t st) {
+    using C = CfgB<D>;
+    using L = SmemOf<C>;
+    CUtensorMap mq, mk, mv;
+    const int64_t row_bytes = (int64_t)H * D * 2;
+    if (!encode_map(&mq, q, T, row_bytes, kBM) || !encode_map(&mk, k, T, row_bytes, C::BN) ||
+        !encode_map(&mv, v, T, row_bytes, C::BN))
+        return FP8VIT_ECUDA;
+    static std::atomic<uint64_t> attr_set;
+    auto kern = attn_fwd_kernel<D, kOutBf16, true, true>;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FP8VIT_ECUDA;
+    const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
+    if (!bit || !(attr_set.load() & bit)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC) !=
+            cudaSuccess)
+            return FP8VIT_ECUDA;
+        attr_set.fetch_or(bit);
+    }
+    dim3 grid((unsigned)((max_seqlen + kBM - 1) / kBM), (unsigned)H, (unsigned)num_seqs);
+    kern<<<grid, kThreads, L::ALLOC, st>>>(mq, mk, mv, nullptr, nullptr, nullptr, cu, max_seqlen, T,
+                                           H, sm_scale, out, nullptr, nullptr, ctx->d_scratch);
+    return cudaGetLastError() == cudaSuccess ? FP8VIT_OK : FP8VIT_ECUDA;
+}
+
 inline bool misaligned(const void* p, uintptr_t a) {
     return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0;
 }
@@ -853,4 +1001,30 @@ extern "C" fp8vit_status fp8_varlen_attn_fwd_group_quant(
                                    d_cu_seqlens, num_seqs, max_seqlen, total_tokens, num_heads,
                                    softmax_scale, d_xq, nullptr, d_scales,
                                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" fp8vit_status bf16_varlen_attn_fwd(fp8vit_ctx* ctx, const uint16_t* d_q,
+                                              const uint16_t* d_k, const uint16_t* d_v,
+                                              const int32_t* d_cu_seqlens, int32_t num_seqs,
+                                              int32_t max_seqlen, int64_t total_tokens,
+                                              int32_t num_heads, int32_t head_dim,
+                                              float softmax_scale, uint16_t* d_out,
+                                              void* stream) {
+    if (!ctx || !d_q || !d_k || !d_v || !d_cu_seqlens || !d_out) return FP8VIT_EINVAL;
+    if (num_seqs < 0 || max_seqlen < 0 || total_tokens < 0 || total_tokens > INT32_MAX ||
+        num_heads < 1)
+        return FP8VIT_EINVAL;
+    if (!(softmax_scale > 0.0f) || !isfinite(softmax_scale)) return FP8VIT_EINVAL;
+    if (head_dim != 72 && head_dim != 128) return FP8VIT_EUNSUPPORTED;
+    if (misaligned(d_q, 16) || misaligned(d_k, 16) || misaligned(d_v, 16) ||
+        misaligned(d_out, 16) || misaligned(d_cu_seqlens, 4))
+        return FP8VIT_EINVAL;
+    if (num_heads > 65535 || num_seqs > 65535) return FP8VIT_EUNSUPPORTED;
+    if (num_seqs == 0 || max_seqlen == 0 || total_tokens == 0) return FP8VIT_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (head_dim == 72)
+        return launch_bf16<72>(ctx, d_q, d_k, d_v, d_cu_seqlens, num_seqs, max_seqlen,
+                               total_tokens, num_heads, softmax_scale, d_out, st);
+    return launch_bf16<128>(ctx, d_q, d_k, d_v, d_cu_seqlens, num_seqs, max_seqlen, total_tokens,
+                            num_heads, softmax_scale, d_out, st);
 }

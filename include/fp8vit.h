@@ -227,6 +227,22 @@ fp8vit_status fp8_varlen_attn_fwd(fp8vit_ctx* ctx, const uint8_t* d_q8, const ui
                                   int32_t head_dim, float softmax_scale, void* d_out,
                                   int32_t out_dtype, const float* d_output_scale, void* stream);
 
+/* The BF16 attention that the pages compare FP8 against (vLLM "FP8 ViT
+ * Encoder Attention", Performance: BF16 vs FP8 attention time), on the same
+ * kernel skeleton as fp8_varlen_attn_fwd: QK^T and PV as kind::f16 tcgen05
+ * MMAs with fp32 accumulation, P rounded to BF16, online softmax.
+ *   o[r,h,:] = sum_j softmax_j(softmax_scale * <q[r,h,:], k[j,h,:]>) v[j,h,:]
+ * over the keys j of r's image.  d_q, d_k, d_v, d_out: BF16
+ * [total_tokens, num_heads, head_dim], 16-byte aligned; no scales.
+ * head_dim 72 or 128 (else FP8VIT_EUNSUPPORTED).  cu_seqlens, checks and
+ * faults as fp8_varlen_attn_fwd.  A comparator for the FP8 path; the
+ * library's FP8 path does not call it. */
+fp8vit_status bf16_varlen_attn_fwd(fp8vit_ctx* ctx, const uint16_t* d_q, const uint16_t* d_k,
+                                   const uint16_t* d_v, const int32_t* d_cu_seqlens,
+                                   int32_t num_seqs, int32_t max_seqlen, int64_t total_tokens,
+                                   int32_t num_heads, int32_t head_dim, float softmax_scale,
+                                   uint16_t* d_out, void* stream);
+
 /* fp8_varlen_attn_fwd with the per-token-group quantizer fused into its
  * epilogue (vLLM issue "fused fp8 output for FlashAttention 3": the output
  * quantization moves into the attention kernel; atrex-bench "#025
