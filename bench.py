@@ -299,11 +299,13 @@ def _quant_rooflines(fv, ctx, src, dev, hbm_gbs, reps=10):
                              3 * n * 2),
         "quant3_kernel": (lambda: fv.fp8_quantize_qkv_per_tensor(*big, desc, q8, k8, v8,
                                                                  ctx=ctx), 3 * n * 3),
-        # amax + ring + quantize in one launch: 2 B read for the amax, then
-        # 2 B read + 1 B written for the codes per element
-        "amax_ring_quant_kernel": (lambda: fv.fp8_amax_ring_quantize_qkv(*big, ring, desc, q8,
-                                                                          k8, v8, ctx=ctx),
-                                   3 * n * 5),
+        # the dynamic path's entry point (at this size it takes the two
+        # kernels above): 2 B read for the amax, then 2 B read + 1 B written
+        # for the codes per element
+        "fp8_amax_ring_quantize_qkv": (lambda: fv.fp8_amax_ring_quantize_qkv(*big, ring, desc,
+                                                                              q8, k8, v8,
+                                                                              ctx=ctx),
+                                       3 * n * 5),
         "group_quant_kernel": (lambda: fv.per_token_group_quant_fp8(x2, 128, xq, xs, ctx=ctx),
                                n * 3 + (n // 128) * 4),
     }

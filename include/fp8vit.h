@@ -185,11 +185,13 @@ fp8vit_status fp8_quantize_qkv_per_tensor(fp8vit_ctx* ctx, const uint16_t* d_q,
  * Usage, dynamic scaling; intro: Q/K/V quantized right before attention):
  * exactly fp8_amax_ring_update(d_q, d_k, d_v, n_elems, d_ring, d_descale3)
  * followed by fp8_quantize_qkv_per_tensor(..., d_descale3, d_q8, d_k8,
- * d_v8): the same ring update, descales and codes, bit for bit.  The kernel
- * is launched cooperatively (all its blocks resident at once) and meets at a
- * grid barrier between the amax and the quantization, so the three small
- * scale stages cost no extra launch and, when the BF16 tensors fit in L2,
- * their second read comes from it.  A barrier wait that exceeds 2 s records
+ * d_v8): the same ring update, descales and codes, bit for bit.  Up to
+ * about twice the L2 size of BF16 inputs, one kernel is launched
+ * cooperatively (all its blocks resident at once) and meets at a grid
+ * barrier between the amax and the quantization, so the scale stages cost no
+ * extra launch and part of the second read of the inputs comes from L2;
+ * larger tensors take those two calls' kernels, which stream HBM faster
+ * without the barrier.  A barrier wait that exceeds 2 s records
  * FP8VIT_ETIMEOUT (read it with fp8vit_check) and leaves the codes unwritten.
  * Alignment and ownership as the two calls; uses the context's scratch (one
  * stream per context at a time). */

@@ -293,10 +293,12 @@ def test_fused_amax_ring_quantize_over_20_forwards(ctx):
     _check_ok(ctx)
 
 
-@pytest.mark.parametrize("n", [0, 1, 7, 8, 9, 8 * 1000 + 5, 1 << 20, 3 * (1 << 22) + 3])
+@pytest.mark.parametrize("n", [0, 1, 7, 8, 9, 8 * 1000 + 5, 1 << 20, 3 * (1 << 22) + 3,
+                               44 * (1 << 20) + 5])
 def test_fused_amax_ring_quantize_ragged_sizes(ctx, n):
     """Ragged lengths (tails below one 16-byte vector, a grid larger than
-    one block's share): codes and descales equal the oracle's bit for bit."""
+    one block's share, inputs above twice L2, which take the two-kernel
+    path): codes and descales equal the oracle's bit for bit."""
     bits = [np.ascontiguousarray(synth.bf16_tensor(synth.stream_key(n + 5, 1, t), 1, max(n, 1))[0, :n])
             for t in range(3)]
     if n:
