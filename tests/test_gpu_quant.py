@@ -344,3 +344,17 @@ def test_fused_barrier_timeout_is_reported_and_recovered():
     for t in range(3):
         assert np.array_equal(_host_u8(out[t]), oracle.quantize_per_tensor(x[t], want[t]).reshape(-1))
     c.close()
+
+
+@pytest.mark.parametrize("m,n", [(1, 2048), (1, 7168), (726, 7168), (1933, 7168), (37504, 2048)])
+def test_group_quant_table_shapes(ctx, m, n):
+    """Shapes of the per_token_group_quant_fp8 benchmark table (token_count x
+    hidden_size): codes and scales equal the oracle's bit for bit."""
+    x = synth.bf16_tensor(synth.stream_key(m, n, 0), m, n)
+    xq = torch.empty((m, n), dtype=torch.uint8, device="cuda")
+    sc = torch.empty((m, n // 128), dtype=torch.float32, device="cuda")
+    fv.per_token_group_quant_fp8(_dev_bf16(x).reshape(m, n), 128, xq, sc, ctx=ctx)
+    _check_ok(ctx)
+    want_q, want_s = oracle.group_quant(x, 128)
+    assert np.array_equal(_host_u8(xq), want_q)
+    assert (_f32_bits(sc.cpu().numpy()) == _f32_bits(want_s)).all()
