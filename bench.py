@@ -339,6 +339,65 @@ def _group_quant_table(fv, ctx, dev, hbm_gbs, reps=10):
     return {"kernel": "group_quant_kernel (group 128)", "peak_GBps": hbm_gbs, "rows": rows}
 
 
+def _attn_sweep(fv, ctx, dev, reps=10):
+    """The pages' attention tables, on this library's kernels: for the
+    head_dim-72 sequence sweep (2304..16384 tokens, 16 heads; the FP8 call
+    includes the Q/K/V quantization, as in the pages' AITER table) and the
+    8192-token head_dim-128 image: the full FP8 call (dynamic amax + ring +
+    quantize, then attention), the FP8 attention alone, this library's BF16
+    attention and torch's BF16 SDPA, all on the same BF16 inputs; CUDA
+    events over `reps` back-to-back calls."""
+    import torch
+    import torch.nn.functional as F
+    import synth
+    rows = []
+    for name in ("c3_2304", "c3_4096", "c3_8192", "c3_16384", "c2"):
+        w = synth.WORKLOADS[name]
+        T, H, D = w.tokens, w.heads, w.head_dim
+        q, k, v = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).reshape(T, H, D)
+                   .to(dev) for x in w.qkv(0))
+        cu = torch.from_numpy(synth.cu_seqlens(w.seg_lens)).to(dev)
+        ring = fv.new_ring(dev)
+        desc = torch.zeros(3, dtype=torch.float32, device=dev)
+        q8, k8, v8 = (torch.empty((T, H, D), dtype=torch.uint8, device=dev) for _ in range(3))
+        out = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+
+        def fp8_attn():
+            fv.fp8_varlen_attn_fwd(q8, k8, v8, desc[0:1], desc[1:2], desc[2:3], cu, T,
+                                   w.softmax_scale, out, ctx=ctx)
+
+        def fp8_full():
+            fv.fp8_amax_ring_quantize_qkv(q, k, v, ring, desc, q8, k8, v8, ctx=ctx)
+            fp8_attn()
+
+        qs, ks, vs = (x.view(1, T, H, D).transpose(1, 2) for x in (q, k, v))
+        calls = {
+            "fp8_with_quant": fp8_full,
+            "fp8_attention": fp8_attn,
+            "bf16_this_library": lambda: fv.bf16_varlen_attn_fwd(q, k, v, cu, T, w.softmax_scale,
+                                                                 out, ctx=ctx),
+            "bf16_torch_sdpa": lambda: F.scaled_dot_product_attention(qs, ks, vs,
+                                                                      scale=w.softmax_scale),
+        }
+        row = {"tokens": T, "heads": H, "head_dim": D}
+        for key, fn in calls.items():
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / reps
+            row[key] = {"ms": ms, "tflops": w.attn_flops() / (ms * 1e-3) / 1e12}
+        rows.append(row)
+        del q, k, v, q8, k8, v8, out
+    return rows
+
+
 def _quant_rooflines(fv, ctx, src, dev, hbm_gbs, reps=10):
     """HBM roofline of the three quantizer kernels on 3 x 32400-token, 16-head,
     head_dim-72 tensors ([97200, 1152] BF16 each, 224 MB): the resident BF16
@@ -584,6 +643,8 @@ def run_ours(args):
         line["comparator_bf16_same_skeleton"] = _bf16_comparator(fv, ctx, w, inputs, dev)
     if args.group_quant_table:
         line["group_quant_table"] = _group_quant_table(fv, ctx, dev, peaks["hbm"])
+    if args.attn_sweep:
+        line["attn_sweep"] = _attn_sweep(fv, ctx, dev)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         codes, dsc = _oracle_inputs(w)
         threads = _host_threads()
@@ -625,6 +686,9 @@ def main():
                     help="also time torch BF16 SDPA on the same inputs (single-image workloads)")
     ap.add_argument("--compare-bf16", action="store_true",
                     help="also time this library's BF16 attention kernel on the same inputs")
+    ap.add_argument("--attn-sweep", action="store_true",
+                    help="also time the pages' attention tables (head_dim-72 sequence sweep, "
+                         "8192-token head_dim 128): FP8 with and without quantization, BF16")
     ap.add_argument("--group-quant-table", action="store_true",
                     help="also time the group quantizer on the shapes of the pages' table")
     args = ap.parse_args()
