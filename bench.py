@@ -37,7 +37,7 @@ import numpy as np  # noqa: E402
 
 METRIC = "FP8 varlen attention TFLOP/s (counted 4*S^2*D*H) over the full step"
 UNIT = "TFLOP/s"
-WORKLOAD = "c2"
+WORKLOAD = "1x8192_d128"
 
 
 def _dist():
@@ -351,7 +351,7 @@ def _attn_sweep(fv, ctx, dev, reps=10):
     import torch.nn.functional as F
     import synth
     rows = []
-    for name in ("c3_2304", "c3_4096", "c3_8192", "c3_16384", "c2"):
+    for name in ("1x2304_d72", "1x4096_d72", "1x8192_d72", "1x16384_d72", "1x8192_d128"):
         w = synth.WORKLOADS[name]
         T, H, D = w.tokens, w.heads, w.head_dim
         q, k, v = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).reshape(T, H, D)

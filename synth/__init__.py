@@ -154,21 +154,21 @@ class Workload:
 # tables; image sizes at 16x16 patches: 1440x2560 -> 14400 tokens,
 # 2160x3840 -> 32400 tokens).
 WORKLOADS = {
-    "c1": Workload("c1: 1x1024 tokens, 16 heads, head_dim 72, static scales",
+    "1x1024_d72": Workload("1x1024 tokens, 16 heads, head_dim 72, static scales",
                    (1024,), 16, 72, "static", (1,)),
-    "c2": Workload("c2: 1x8192 tokens, 16 heads, head_dim 128, dynamic ring over 20 forwards",
+    "1x8192_d128": Workload("1x8192 tokens, 16 heads, head_dim 128, dynamic ring over 20 forwards",
                    (8192,), 16, 128, "dynamic", tuple(range(100, 120)), group_quant=True),
-    "c3_2304": Workload("c3: 1x2304 tokens, 16 heads, head_dim 72, dynamic",
+    "1x2304_d72": Workload("1x2304 tokens, 16 heads, head_dim 72, dynamic",
                         (2304,), 16, 72, "dynamic", (300,)),
-    "c3_4096": Workload("c3: 1x4096 tokens, 16 heads, head_dim 72, dynamic",
+    "1x4096_d72": Workload("1x4096 tokens, 16 heads, head_dim 72, dynamic",
                         (4096,), 16, 72, "dynamic", (301,)),
-    "c3_8192": Workload("c3: 1x8192 tokens, 16 heads, head_dim 72, dynamic",
+    "1x8192_d72": Workload("1x8192 tokens, 16 heads, head_dim 72, dynamic",
                         (8192,), 16, 72, "dynamic", (302,)),
-    "c3_16384": Workload("c3: 1x16384 tokens, 16 heads, head_dim 72, dynamic",
+    "1x16384_d72": Workload("1x16384 tokens, 16 heads, head_dim 72, dynamic",
                          (16384,), 16, 72, "dynamic", (303,)),
-    "c4": Workload("c4: 3x14400 tokens, 16 heads, head_dim 72, static scales, fp8 output",
+    "3x14400_d72": Workload("3x14400 tokens, 16 heads, head_dim 72, static scales, fp8 output",
                    (14400, 14400, 14400), 16, 72, "static", (400,), fp8_out=True),
-    "c5": Workload("c5: 3x32400 tokens, 16 heads, head_dim 72, 27 layers, dynamic, group quant",
+    "3x32400_d72": Workload("3x32400 tokens, 16 heads, head_dim 72, 27 layers, dynamic, group quant",
                    (32400, 32400, 32400), 16, 72, "dynamic", tuple(range(500, 527)),
                    group_quant=True),
 }

@@ -93,9 +93,9 @@ def test_small_shapes_full_oracle(ctx, lens, H, D):
     assert_attn_close(got, ref, (lens, H, D))
 
 
-def test_c1_full_oracle(ctx):
+def test_1024_tokens_full_oracle(ctx):
     """1024 tokens, 16 heads, head_dim 72, static scales: every output."""
-    w = synth.WORKLOADS["c1"]
+    w = synth.WORKLOADS["1x1024_d72"]
     q, k, v = w.qkv(0)
     amax = [oracle.amax_bf16(x) for x in (q, k, v)]
     desc = [oracle.descale_from_amax(np.float32(1.5) * np.float32(a)) for a in amax]
@@ -104,11 +104,11 @@ def test_c1_full_oracle(ctx):
     cu = synth.cu_seqlens(w.seg_lens)
     ref = oracle.attn_full(*codes, *desc, cu, w.heads, w.head_dim, w.softmax_scale)
     out = _run_gpu(ctx, cu, codes, desc, w.heads, w.head_dim, max(w.seg_lens))
-    e = assert_attn_close(_gpu_bf16_to_f64(out), ref, "c1")
-    print("c1 errors", e)
+    e = assert_attn_close(_gpu_bf16_to_f64(out), ref, "1x1024_d72")
+    print("1024 tokens errors", e)
 
 
-@pytest.mark.parametrize("name", ["c2", "c3_2304", "c3_16384", "c4", "c5"])
+@pytest.mark.parametrize("name", ["1x8192_d128", "1x2304_d72", "1x16384_d72", "3x14400_d72", "3x32400_d72"])
 def test_workload_sampled_rows(ctx, name):
     w = synth.WORKLOADS[name]
     q, k, v = w.qkv(0)
@@ -146,11 +146,11 @@ def test_fp8_output_small_full(ctx):
     assert dist[big].max() <= 1
 
 
-def test_fp8_output_c4_sampled(ctx):
+def test_fp8_output_3x14400_sampled(ctx):
     """3 x 14400 tokens, static scales, fused FP8 output.  output_scale is
     the amax of the oracle's sampled rows / 448 (the full amax needs the full
     fp64 attention); larger values saturate on both sides alike."""
-    w = synth.WORKLOADS["c4"]
+    w = synth.WORKLOADS["3x14400_d72"]
     q, k, v = w.qkv(0)
     amax = [oracle.amax_bf16(x) for x in (q, k, v)]
     desc = [oracle.descale_from_amax(np.float32(1.5) * np.float32(a)) for a in amax]
@@ -164,13 +164,13 @@ def test_fp8_output_c4_sampled(ctx):
     got = _run_gpu(ctx, cu, codes, desc, w.heads, w.head_dim, max(w.seg_lens),
                    output_scale=out_scale)
     g = got.cpu().numpy()[toks, hs]
-    assert_fp8_out_close(g, ref, out_scale, oracle.e4m3_decode, "c4 fp8 out")
+    assert_fp8_out_close(g, ref, out_scale, oracle.e4m3_decode, "3x14400 fp8 out")
     big = np.abs(ref) >= np.abs(ref).max() / 16
     assert code_step_distance(g, want)[big].max() <= 1
 
 
 @pytest.mark.parametrize("lens,H,D,name", [((300, 129), 2, 72, None), ((513,), 2, 128, None),
-                                         (None, None, None, "c2"), (None, None, None, "c5")])
+                                         (None, None, None, "1x8192_d128"), (None, None, None, "3x32400_d72")])
 def test_single_term_p_mode(lens, H, D, name):
     """P as one e4m3 term (fp8vit_set_attn_p_terms(ctx, 1)): the mode takes
     effect, stays inside the mean-abs and cosine gates, and its max-abs error
@@ -256,7 +256,7 @@ def test_end_to_end_dynamic_pipeline(ctx):
 
 
 @pytest.mark.parametrize("lens,H,name", [((513, 129, 0, 300), 2, None), ((1,), 1, None),
-                                         (None, None, "c2")])
+                                         (None, None, "1x8192_d128")])
 def test_fused_group_quant(ctx, lens, H, name):
     """fp8_varlen_attn_fwd_group_quant (head_dim 128) writes, byte for byte and
     bit for bit, what the oracle's group quantizer (group 128) gives for the

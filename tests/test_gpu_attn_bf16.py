@@ -53,7 +53,7 @@ def test_bf16_small_shapes_full_oracle(ctx, lens, H, D):
     assert_attn_close(got, ref, (lens, H, D))
 
 
-@pytest.mark.parametrize("name", ["c1", "c2", "c3_16384", "c5"])
+@pytest.mark.parametrize("name", ["1x1024_d72", "1x8192_d128", "1x16384_d72", "3x32400_d72"])
 def test_bf16_workload_sampled_rows(ctx, name):
     w = synth.WORKLOADS[name]
     x = w.qkv(0)

@@ -40,7 +40,7 @@ def test_ring_descales_bit_exact_over_20_forwards(ctx):
     """Dynamic scaling over the 20 forwards of the 8192-token, head_dim-128
     workload: the ring wraps after 16; every forward's descales and the ring
     contents must equal the oracle's bit for bit."""
-    w = synth.WORKLOADS["c2"]
+    w = synth.WORKLOADS["1x8192_d128"]
     ring_d = fv.new_ring()
     desc_d = torch.zeros(3, dtype=torch.float32, device="cuda")
     ring_o = oracle.Ring()
@@ -103,7 +103,7 @@ def _quant_case(ctx, q, k, v, desc):
         assert (got == want).all(), (np.nonzero(got != want)[0][:5])
 
 
-@pytest.mark.parametrize("name", ["c1", "c2", "c4", "c5"])
+@pytest.mark.parametrize("name", ["1x1024_d72", "1x8192_d128", "3x14400_d72", "3x32400_d72"])
 def test_quantize_per_tensor_bit_exact(ctx, name):
     """Static (margin 1.5) and dynamic descales on every workload's tensors."""
     w = synth.WORKLOADS[name]
@@ -111,7 +111,7 @@ def test_quantize_per_tensor_bit_exact(ctx, name):
     amax = [oracle.amax_bf16(x) for x in (q, k, v)]
     static = [oracle.descale_from_amax(np.float32(1.5) * np.float32(a)) for a in amax]
     _quant_case(ctx, q, k, v, static)
-    if name in ("c1", "c2"):
+    if name in ("1x1024_d72", "1x8192_d128"):
         tight = [oracle.descale_from_amax(a) for a in amax]  # amax maps onto exactly 448
         _quant_case(ctx, q, k, v, tight)
 
@@ -160,7 +160,7 @@ def test_group_quant_other_group_sizes(ctx, group):
 def test_amax3_then_ring_push_equals_fused_update(ctx):
     """The split path used when one batch is spread over several GPUs
     (amax, all-reduce, ring push) gives the fused update's bits on one GPU."""
-    w = synth.WORKLOADS["c2"]
+    w = synth.WORKLOADS["1x8192_d128"]
     ring_a, ring_b = fv.new_ring(), fv.new_ring()
     da = torch.zeros(3, dtype=torch.float32, device="cuda")
     db = torch.zeros(3, dtype=torch.float32, device="cuda")
@@ -264,7 +264,7 @@ def test_fused_amax_ring_quantize_over_20_forwards(ctx):
     forwards of the 8192-token, head_dim-128 workload (the ring wraps after
     16): every forward's descales, ring contents and e4m3 codes equal the
     oracle's ring + quantizer bit for bit, and the two-call path's."""
-    w = synth.WORKLOADS["c2"]
+    w = synth.WORKLOADS["1x8192_d128"]
     n = w.tokens * w.hd
     ring_f, ring_2 = fv.new_ring(), fv.new_ring()
     desc_f = torch.zeros(3, dtype=torch.float32, device="cuda")

@@ -47,7 +47,7 @@ def test_bf16_rounding_matches_torch():
 
 
 def test_workloads():
-    w = synth.WORKLOADS["c4"]
+    w = synth.WORKLOADS["3x14400_d72"]
     assert w.tokens == 43200 and list(synth.cu_seqlens(w.seg_lens)) == [0, 14400, 28800, 43200]
-    assert synth.WORKLOADS["c2"].attn_flops() == 4.0 * 8192 ** 2 * 128 * 16
+    assert synth.WORKLOADS["1x8192_d128"].attn_flops() == 4.0 * 8192 ** 2 * 128 * 16
     assert synth.outlier_count(2048) == 20 and synth.outlier_count(1152) == 12
