@@ -302,3 +302,17 @@ def test_fused_group_quant(ctx, lens, H, name):
     xs2 = torch.empty_like(xs)
     fv.per_token_group_quant_fp8(out.view(T, H * D), 128, xq2, xs2, ctx=ctx)
     assert torch.equal(xq, xq2) and torch.equal(xs.view(torch.int32), xs2.view(torch.int32))
+
+
+@pytest.mark.parametrize("lens,H,D,max_seqlen", [((200,), 1, 128, 200), ((150, 40), 40, 128, 512),
+                                                 ((97, 3), 6, 72, 300), ((1, 1, 1), 2, 72, 1)])
+def test_head_counts_and_slack_max_seqlen(ctx, lens, H, D, max_seqlen):
+    """One head, many heads, and a max_seqlen above the longest image (the
+    grid then holds query tiles with no rows, which exit at once): every
+    output against the oracle."""
+    cu, codes, desc = _prepare(lens, H, D, seed=H * 1000 + sum(lens))
+    sm = np.float32(1.0 / math.sqrt(D))
+    ref = oracle.attn_full(*codes, *desc, cu, H, D, sm)
+    got = _gpu_bf16_to_f64(_run_gpu(ctx, cu, codes, desc, H, D, max_seqlen))
+    assert not np.isnan(got).any()
+    assert_attn_close(got, ref, (lens, H, D, max_seqlen))
