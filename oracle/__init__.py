@@ -2,8 +2,9 @@
 
 The oracle is the plain, slow, single-threaded statement of what the path
 computes (``oracle.c``): the e4m3 codec, the amax / ring-buffer / scale rules,
-the per-tensor and per-token-group quantizers and fp64 softmax attention over
-the dequantised FP8 tensors.  Only the tests, ``__graft_entry__.smoke()`` and
+the per-tensor and per-token-group quantizers, fp64 softmax attention over
+the dequantised FP8 tensors, and the same attention over BF16 tensors (the
+BF16 comparator's reference).  Only the tests, ``__graft_entry__.smoke()`` and
 the benchmark's CPU-baseline leg may import it.  It shares no code with the
 CUDA library and never imports it.
 """
