@@ -42,6 +42,16 @@ MUTANTS = [
     ("key row off by one", "const uint8_t* kj = k8 + j * row + (int64_t)h * D;",
      "const uint8_t* kj = k8 + (j > a ? j - 1 : j) * row + (int64_t)h * D;"),
     ("v read with the k pointer", "const uint8_t* vj = v8 + j * row", "const uint8_t* vj = k8 + j * row"),
+    # the BF16 attention (the comparator's reference)
+    ("bf16: key of head 0", "const uint16_t* kj = k + j * row + (int64_t)h * D;",
+     "const uint16_t* kj = k + j * row;"),
+    ("bf16: v read with the k pointer", "const uint16_t* vj = v + j * row",
+     "const uint16_t* vj = k + j * row"),
+    ("bf16: query of head 0", "qv[d] = (double)orc_bf16_to_float(q[t * row + (int64_t)h * D + d]);",
+     "qv[d] = (double)orc_bf16_to_float(q[t * row + d]);"),
+    ("bf16: score without the softmax scale",
+     "for (int32_t d = 0; d < D; ++d) acc += qv[d] * (double)orc_bf16_to_float(kj[d]);\n            s[j - a] = (double)sm_scale * acc;",
+     "for (int32_t d = 0; d < D; ++d) acc += qv[d] * (double)orc_bf16_to_float(kj[d]);\n            s[j - a] = acc;"),
 ]
 
 
@@ -106,6 +116,17 @@ def _pins():
         o = torch.einsum("hst,thd->shd", torch.softmax(sc_, -1), v[a:b]).numpy()
         ok &= np.allclose(got[a:b], o, rtol=1e-12, atol=1e-14)
     out["attention"] = bool(ok)
+    # BF16 attention vs torch fp64 on the same values
+    xb = [synth.bf16_tensor(synth.stream_key(5, 2, t), 15, H * D) for t in range(3)]
+    got = oracle.attn_full_bf16(*xb, cu, H, D, sm)
+    qb, kb, vb = (_bf16(x).to(torch.float64).reshape(15, H, D) for x in xb)
+    ok = True
+    for i in range(len(lens)):
+        a, b = int(cu[i]), int(cu[i + 1])
+        sc_ = torch.einsum("shd,thd->hst", qb[a:b], kb[a:b]) * sm
+        o = torch.einsum("hst,thd->shd", torch.softmax(sc_, -1), vb[a:b]).numpy()
+        ok &= np.allclose(got[a:b], o, rtol=1e-12, atol=1e-14)
+    out["bf16 attention"] = bool(ok)
     return out
 
 
