@@ -346,7 +346,7 @@ class FP8EncoderAttention:
     static descales), and runs
         [amax ring update] -> per-tensor quantize -> varlen FP8 attention
     (the first two as one cooperative launch on one GPU)
-        [-> per-token-group quantize of the BF16 output]
+        [-> per-token-group quantize of the output, fused at head_dim 128]
     on the current stream.  Intermediate FP8 buffers are allocated once per
     token count and reused (no allocation per call at steady state).
     """
@@ -396,9 +396,16 @@ class FP8EncoderAttention:
                                    out=mk(torch.uint8 if fp8_out else torch.bfloat16))
         return self._bufs[key]
 
-    def forward(self, q, k, v, cu_seqlens, max_seqlen: int, output_scale=None, out=None):
+    def forward(self, q, k, v, cu_seqlens, max_seqlen: int, output_scale=None, out=None,
+                group_quant: bool = False):
         """q, k, v: BF16 [T, H, D] on the device; cu_seqlens: int32 [B+1].
-        Returns the attention output (BF16, or e4m3 codes if output_scale)."""
+        Returns the attention output (BF16, or e4m3 codes if output_scale), or
+        with ``group_quant`` the o-proj input: (e4m3 codes [T, H*D], fp32
+        scales [T, H*D/128]) of the BF16 output's per-token groups of 128 --
+        fused into the attention epilogue at head_dim 128, a separate
+        per_token_group_quant_fp8 call otherwise."""
+        if group_quant and output_scale is not None:
+            raise ValueError("group_quant and output_scale are exclusive")
         T = q.shape[0]
         b = self._buffers(T, output_scale is not None)
         if self.ring is not None and self.process_group is not None:
@@ -415,6 +422,26 @@ class FP8EncoderAttention:
         else:
             fp8_quantize_qkv_per_tensor(q, k, v, self.descale, b["q8"], b["k8"], b["v8"],
                                         ctx=self.ctx)
+        if group_quant:
+            hd = self.H * self.D
+            if hd % 128 != 0:
+                raise ValueError("group_quant needs num_heads * head_dim to be a multiple of 128")
+            if "xq" not in b:
+                b["xq"] = torch.empty((T, hd), dtype=torch.uint8, device=self.device)
+                b["xs"] = torch.empty((T, hd // 128), dtype=torch.float32, device=self.device)
+            xq, xs = b["xq"], b["xs"]
+            if self.D == 128:
+                fp8_varlen_attn_fwd_group_quant(b["q8"], b["k8"], b["v8"], self.descale[0:1],
+                                                self.descale[1:2], self.descale[2:3], cu_seqlens,
+                                                max_seqlen, self.softmax_scale, xq, xs,
+                                                ctx=self.ctx)
+            else:
+                o = b["out"]
+                fp8_varlen_attn_fwd(b["q8"], b["k8"], b["v8"], self.descale[0:1],
+                                    self.descale[1:2], self.descale[2:3], cu_seqlens, max_seqlen,
+                                    self.softmax_scale, o, ctx=self.ctx)
+                per_token_group_quant_fp8(o.view(T, hd), 128, xq, xs, ctx=self.ctx)
+            return xq, xs
         o = b["out"] if out is None else out
         fp8_varlen_attn_fwd(b["q8"], b["k8"], b["v8"], self.descale[0:1], self.descale[1:2],
                             self.descale[2:3], cu_seqlens, max_seqlen, self.softmax_scale, o,

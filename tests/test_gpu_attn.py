@@ -316,3 +316,25 @@ def test_head_counts_and_slack_max_seqlen(ctx, lens, H, D, max_seqlen):
     got = _gpu_bf16_to_f64(_run_gpu(ctx, cu, codes, desc, H, D, max_seqlen))
     assert not np.isnan(got).any()
     assert_attn_close(got, ref, (lens, H, D, max_seqlen))
+
+
+@pytest.mark.parametrize("lens,H,D", [((333, 190), 4, 128), ((333, 190), 16, 72)])
+def test_layer_group_quant_output(lens, H, D):
+    """FP8EncoderAttention(group_quant=True) returns the o-proj input: the
+    codes and scales of per_token_group_quant_fp8 applied to the layer's own
+    BF16 output (fused epilogue at head_dim 128, two calls at 72), bit for
+    bit, on two layers fed the same inputs."""
+    cu = synth.cu_seqlens(lens)
+    T = int(cu[-1])
+    bf = [synth.bf16_tensor(synth.stream_key(88, 0, t), T, H * D) for t in range(3)]
+    dev = [_dev(x.view(np.int16)).view(torch.bfloat16).reshape(T, H, D) for x in bf]
+    a = fv.FP8EncoderAttention(H, D)
+    b = fv.FP8EncoderAttention(H, D)
+    xq, xs = a(*dev, _dev(cu), max(lens), group_quant=True)
+    o = b(*dev, _dev(cu), max(lens))
+    yq = torch.empty_like(xq)
+    ys = torch.empty_like(xs)
+    fv.per_token_group_quant_fp8(o.view(T, H * D), 128, yq, ys)
+    st, site = a.ctx.check()
+    assert st == fv.OK, (fv.status_string(st), site)
+    assert torch.equal(xq, yq) and torch.equal(xs.view(torch.int32), ys.view(torch.int32))
