@@ -338,3 +338,42 @@ def test_layer_group_quant_output(lens, H, D):
     st, site = a.ctx.check()
     assert st == fv.OK, (fv.status_string(st), site)
     assert torch.equal(xq, yq) and torch.equal(xs.view(torch.int32), ys.view(torch.int32))
+
+
+def test_calibrate_once_then_static(tmp_path):
+    """The pages' calibrate-once workflow end to end: 16 dynamic forwards fill
+    the ring, its per-tensor maxima are saved with the 1.5 margin, a static
+    layer loads the file (descales bit-exact against the oracle's rule), and a
+    fresh forward through the static layer stays within the gate."""
+    lens, H, D = (257, 100), 4, 72
+    cu = synth.cu_seqlens(lens)
+    T = int(cu[-1])
+    layer = fv.FP8EncoderAttention(H, D)
+    ring_o = oracle.Ring()
+    amax_max = np.zeros(3, dtype=np.float32)
+    for f in range(16):
+        bf = [synth.bf16_tensor(synth.stream_key(600 + f, f, t), T, H * D) for t in range(3)]
+        a = np.array([oracle.amax_bf16(x) for x in bf], dtype=np.float32)
+        ring_o.update(list(a))
+        amax_max = np.maximum(amax_max, a)
+        dev = [_dev(x.view(np.int16)).view(torch.bfloat16).reshape(T, H, D) for x in bf]
+        layer(*dev, _dev(cu), max(lens))
+    st, site = layer.ctx.check()
+    assert st == fv.OK, (fv.status_string(st), site)
+    got = np.asarray(fv.fp8_ring_read_amax(layer.ring), dtype=np.float32)
+    assert (got.view(np.uint32) == amax_max.view(np.uint32)).all()
+    path = str(tmp_path / "scales.json")
+    name = "visual.blocks.0.attn.attn"
+    fv.fp8_static_scales_save(path, [name], got.reshape(1, 3), margin=1.5)
+    static = fv.FP8EncoderAttention.from_scale_file(path, name, H, D)
+    want = [oracle.descale_from_amax(np.float32(1.5) * np.float32(x)) for x in amax_max]
+    assert (static.descale.cpu().numpy().view(np.uint32) ==
+            np.asarray(want, np.float32).view(np.uint32)).all()
+    bf = [synth.bf16_tensor(synth.stream_key(700, 0, t), T, H * D) for t in range(3)]
+    dev = [_dev(x.view(np.int16)).view(torch.bfloat16).reshape(T, H, D) for x in bf]
+    out = static(*dev, _dev(cu), max(lens))
+    st, site = static.ctx.check()
+    assert st == fv.OK, (fv.status_string(st), site)
+    codes = [oracle.quantize_per_tensor(x, d).reshape(T, H, D) for x, d in zip(bf, want)]
+    ref = oracle.attn_full(*codes, *want, cu, H, D, np.float32(1.0 / math.sqrt(D)))
+    assert_attn_close(_gpu_bf16_to_f64(out), ref, "static after calibration")
