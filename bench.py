@@ -433,14 +433,19 @@ def _quant_rooflines(fv, ctx, src, dev, hbm_gbs, reps=10):
     for name, (fn, nbytes) in runs.items():
         for _ in range(3):
             fn()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(reps)]
-        for a, b in evs:
+        # sustained rate: `reps` back-to-back launches between one pair of
+        # events (no event between launches), median of three such batches
+        batches = []
+        for _ in range(3):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            fn()
+            for _ in range(reps):
+                fn()
             b.record(stream)
-        torch.cuda.synchronize()
-        ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+            torch.cuda.synchronize()
+            batches.append(a.elapsed_time(b) / reps)
+        ms = statistics.median(batches)
         gbs = nbytes / (ms * 1e-3) / 1e9
         out[name] = {"bytes": nbytes, "ms": ms, "achieved_GBps": gbs, "peak_GBps": hbm_gbs,
                      "frac": gbs / hbm_gbs}
