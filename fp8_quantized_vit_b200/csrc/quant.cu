@@ -223,8 +223,8 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quant3_kernel(
 // generation counter to move (bounded: a timeout records FP8VIT_ETIMEOUT
 // and the block returns); phase 2 quantizes as quant3_kernel does.  The BF16
 // tensors are read twice; KEEP (chosen when the three tensors fit in L2)
-// loads them with evict_last priority in phase 1, and phase 2 quantizes the
-// most recently read tensor first, so its reads come from L2.
+// loads them with evict_last priority in phase 1, so that more of phase 2's
+// reads come from L2.
 constexpr uint64_t kBarrierTimeoutNs = 2000000000ull;
 
 // |x| maxima of q, k and v over this thread's grid-stride share in one loop:
@@ -535,10 +535,10 @@ fp8vit_status fp8_amax_ring_quantize_qkv(fp8vit_ctx* ctx, const uint16_t* d_q,
         return FP8VIT_EINVAL;
     // The one-launch kernel: faster than the two kernels up to about twice L2
     // of BF16 inputs (one launch, interleaved streams, part of the second read
-    // served by L2; with evict_last loads when the inputs fill at most 3/4 of
-    // it).  Larger tensors take the two kernels, which stream HBM slightly
-    // faster than the barrier-split launch.  The results are identical.
-    const bool keep = n_elems <= ctx->l2_bytes / 8;
+    // served by L2; with evict_last loads when the inputs fit in L2).  Larger
+    // tensors take the two kernels, which stream HBM slightly faster than the
+    // barrier-split launch.  The results are identical.
+    const bool keep = n_elems <= ctx->l2_bytes / 6;
     if (n_elems > ctx->l2_bytes / 3) {  // more than twice L2 in BF16 inputs
         const fp8vit_status st = fp8_amax_ring_update(ctx, d_q, d_k, d_v, n_elems, d_ring,
                                                       d_descale3, stream);
