@@ -36,6 +36,7 @@ _SIGNATURES = {
     "fp8vit_status_string": (ctypes.c_char_p, [_I32]),
     "fp8vit_set_attn_p_terms": (_I32, [_P, _I32]),
     "fp8vit_inject_lost_arrival": (_I32, [_P, _P]),
+    "fp8vit_inject_attn_timeout": (_I32, [_P, _P]),
     "fp8vit_version": (_I32, []),
     "fp8vit_ring_init": (_I32, [_P, _P]),
     "fp8_amax_ring_update": (_I32, [_P, _P, _P, _P, _I64, _P, _P, _P]),

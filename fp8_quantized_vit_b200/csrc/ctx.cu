@@ -93,6 +93,21 @@ fp8vit_status fp8vit_inject_lost_arrival(fp8vit_ctx* ctx, void* stream) {
     return FP8VIT_OK;
 }
 
+fp8vit_status fp8vit_inject_attn_timeout(fp8vit_ctx* ctx, void* stream) {
+    if (!ctx) return FP8VIT_EINVAL;
+    // Until the next fp8vit_check clears it, every attention CTA launched on
+    // this context skips the commit that announces its first scores, so its
+    // softmax warps' bounded wait runs out (the kernel then aborts, drains
+    // and returns).
+    const uint32_t one = 1u;
+    FP8VIT_CUDA_TRY(cudaMemcpyAsync(reinterpret_cast<uint8_t*>(ctx->d_scratch) +
+                                        offsetof(fp8vit_scratch, inject_attn),
+                                    &one, sizeof(one), cudaMemcpyHostToDevice,
+                                    reinterpret_cast<cudaStream_t>(stream)));
+    FP8VIT_CUDA_TRY(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+    return FP8VIT_OK;
+}
+
 fp8vit_status fp8vit_ring_init(void* d_ring, void* stream) {
     if (!d_ring || (reinterpret_cast<uintptr_t>(d_ring) & 15)) return FP8VIT_EINVAL;
     FP8VIT_CUDA_TRY(cudaMemsetAsync(d_ring, 0, FP8VIT_RING_BYTES,

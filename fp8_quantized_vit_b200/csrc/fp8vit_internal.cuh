@@ -17,9 +17,10 @@ struct fp8vit_scratch {
     int32_t site;          // kernel-specific location code of that fault
     uint32_t amax_bits[3]; // running |x| maxima (bf16 bit patterns) of q, k, v
     uint32_t arrivals;     // CTAs of the current amax launch that have finished
+    uint32_t inject_attn;  // test hook: attention CTAs skip their first S-ready commit
     uint32_t release;      // generation counter of the fused amax/quantize grid barrier
     float descale[3];      // descales published across that barrier
-    uint32_t pad[22];      // to 128 bytes
+    uint32_t pad[21];      // to 128 bytes
 };
 
 struct fp8vit_ctx {

@@ -377,3 +377,30 @@ def test_calibrate_once_then_static(tmp_path):
     codes = [oracle.quantize_per_tensor(x, d).reshape(T, H, D) for x, d in zip(bf, want)]
     ref = oracle.attn_full(*codes, *want, cu, H, D, np.float32(1.0 / math.sqrt(D)))
     assert_attn_close(_gpu_bf16_to_f64(out), ref, "static after calibration")
+
+
+def test_attention_timeout_is_reported_and_recovered():
+    """A skipped S-ready commit (injected on the host) makes the softmax warps'
+    bounded wait run out: the kernel stops its other roles, drains its copies
+    and MMAs, frees TMEM and returns; fp8vit_check reports FP8VIT_ETIMEOUT at
+    one of the two waits it starves and clears the injection, and the next launch on the
+    same context matches the oracle.  No GPU fault is involved."""
+    c = fv.Context()
+    lens, H, D = (129,), 2, 128
+    cu, codes, desc = _prepare(lens, H, D, seed=5)
+    T = codes[0].shape[0]
+    q8, k8, v8 = (_dev(x) for x in codes)
+    d = [torch.tensor([x], dtype=torch.float32, device="cuda") for x in desc]
+    out = torch.full((T, H, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    assert fv.lib().fp8vit_inject_attn_timeout(c.handle, fv._stream()) == fv.OK
+    fv.fp8_varlen_attn_fwd(q8, k8, v8, d[0], d[1], d[2], _dev(cu), max(lens),
+                           np.float32(1.0 / math.sqrt(D)), out, ctx=c)
+    st, site = c.check()
+    # the softmax warps wait for S(0) (site 113) while the issuer waits for
+    # the S buffer to be released (site 119): the first to give up records it
+    assert st == fv.ETIMEOUT and site in (113, 119), (fv.status_string(st), site)
+    assert c.check() == (fv.OK, 0)
+    got = _gpu_bf16_to_f64(_run_gpu(c, cu, codes, desc, H, D, max(lens)))
+    ref = oracle.attn_full(*codes, *desc, cu, H, D, np.float32(1.0 / math.sqrt(D)))
+    assert_attn_close(got, ref, "after the injected timeout")
+    c.close()
