@@ -124,6 +124,28 @@ def test_attn_p_terms_setting_is_checked_on_the_host():
     assert lib.fp8vit_set_attn_p_terms(fake_ctx, 2) == fv.OK
 
 
+def test_new_entry_points_check_arguments_on_the_host():
+    lib = fv.lib()
+    fake_ctx = ctypes.create_string_buffer(64)
+    dummy = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10001)
+    # BF16 attention: head_dim outside {72, 128}, misaligned input, null output
+    assert lib.bf16_varlen_attn_fwd(fake_ctx, dummy, dummy, dummy, dummy, 1, 8, 8, 2, 64, 0.1,
+                                    dummy, None) == fv.EUNSUPPORTED
+    assert lib.bf16_varlen_attn_fwd(fake_ctx, odd, dummy, dummy, dummy, 1, 8, 8, 2, 72, 0.1,
+                                    dummy, None) == fv.EINVAL
+    assert lib.bf16_varlen_attn_fwd(fake_ctx, dummy, dummy, dummy, dummy, 1, 8, 8, 2, 72, 0.1,
+                                    None, None) == fv.EINVAL
+    assert lib.bf16_varlen_attn_fwd(None, dummy, dummy, dummy, dummy, 1, 8, 8, 2, 72, 0.1,
+                                    dummy, None) == fv.EINVAL
+    # failure-injection hooks need a context
+    assert lib.fp8vit_inject_lost_arrival(None, None) == fv.EINVAL
+    assert lib.fp8vit_inject_attn_timeout(None, None) == fv.EINVAL
+    # the dynamic-path entry point: negative size
+    assert lib.fp8_amax_ring_quantize_qkv(fake_ctx, dummy, dummy, dummy, -1, dummy, dummy, dummy,
+                                          dummy, dummy, None) == fv.EINVAL
+
+
 def test_host_argument_checks_need_no_gpu():
     lib = fv.lib()
     fake_ctx = ctypes.create_string_buffer(64)
