@@ -48,6 +48,12 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;
 // reference max keeps P <= 2^(6 + 2.75) = 430 < 448 (e4m3 max).
 constexpr float kPLog2 = 6.0f;
 constexpr float kSlackLog2 = 2.75f;
+// head_dim 128 trades one binade of P's low end (values below 2^-11 of the
+// reference max turn e4m3-subnormal one binade earlier) for a wider slack,
+// 2^(5 + 3.75) = 430 as well: fewer O rescales (measured faster at 128,
+// slower at 72).
+constexpr float kPLog2D128 = 5.0f;
+constexpr float kSlackLog2D128 = 3.75f;
 
 template <int D>
 struct Cfg;
@@ -717,12 +723,14 @@ __global__ void __launch_bounds__(kThreads, 2)
             const float mx = tile_row_max<NCH>(r);
             const float mxc = mx * scale_log2;
             // j == 0 sets the reference; the first PV initialises O.
-            const bool need = j == 0 || mxc > m_ref + kSlackLog2;
+            constexpr float slack = (D == 128 && !BF) ? kSlackLog2D128 : kSlackLog2;
+            constexpr float plog2 = (D == 128 && !BF) ? kPLog2D128 : kPLog2;
+            const bool need = j == 0 || mxc > m_ref + slack;
             const bool rescale = j > 0 && __any_sync(0xFFFFFFFFu, need);
             const float alpha = (j > 0 && need) ? ex2_approx(m_ref - mxc) : 1.0f;
             if (need) m_ref = mxc;
             // P = 2^(x - bias), bias = m_ref - kPLog2
-            const float bias = m_ref - kPLog2;
+            const float bias = m_ref - plog2;
             const uint64_t c2 = f2pack(scale_log2, scale_log2);
             const uint64_t nb2 = f2pack(-bias, -bias);
             if constexpr (C::PSLOTS == 2) {
