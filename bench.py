@@ -461,6 +461,8 @@ def _config(w, n_fwd=None):
             "head_dim": w.head_dim, "forwards": n_fwd,
             "step": "amax ring + quantize q/k/v (one launch) + attention (bf16 out) + group quant (128)",
             "l2": f"inputs rotate over {n_fwd} forwards ({gb:.2f} GB; L2 is 126 MB)",
+            "rings": (f"one amax ring per layer ({n_fwd} layers)" if w.per_layer_rings
+                      else "one amax ring over the rotation"),
             "parallelism": "replicas"}
 
 
@@ -492,7 +494,9 @@ def run_ours(args):
                        .reshape(T, H, D).to(dev) for x in qkv])
     cu = torch.from_numpy(synth.cu_seqlens(w.seg_lens)).to(dev)
     max_s = max(w.seg_lens)
-    ring = fv.new_ring(dev)
+    # one ring for a rotation of forwards; one per layer when the seeds are the
+    # layers of one encoder forward (each layer keeps its own amax history)
+    rings = [fv.new_ring(dev) for _ in range(n_fwd if w.per_layer_rings else 1)]
     desc = torch.zeros(3, dtype=torch.float32, device=dev)
     q8, k8, v8 = (torch.empty((T, H, D), dtype=torch.uint8, device=dev) for _ in range(3))
     out = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
@@ -504,7 +508,7 @@ def run_ours(args):
 
     def step(i, timed=False):
         q, k, v = inputs[i % n_fwd]
-        fv.fp8_amax_ring_quantize_qkv(q, k, v, ring, desc, q8, k8, v8, ctx=ctx)
+        fv.fp8_amax_ring_quantize_qkv(q, k, v, rings[i % len(rings)], desc, q8, k8, v8, ctx=ctx)
         if timed:
             ev_a[i].record(stream)
         fv.fp8_varlen_attn_fwd(q8, k8, v8, desc[0:1], desc[1:2], desc[2:3], cu, max_s,
@@ -595,7 +599,8 @@ def run_ours(args):
         if i >= 2:
             stream.wait_event(ev_down[i - 2])  # dxq/dxs[i % 2] have been read back
         dq, dk, dv = dbuf[i % 2]
-        fv.fp8_amax_ring_quantize_qkv(dq, dk, dv, ring, desc, q8, k8, v8, ctx=ctx)
+        fv.fp8_amax_ring_quantize_qkv(dq, dk, dv, rings[i % len(rings)], desc, q8, k8, v8,
+                                      ctx=ctx)
         fv.fp8_varlen_attn_fwd(q8, k8, v8, desc[0:1], desc[1:2], desc[2:3], cu, max_s,
                                w.softmax_scale, out, ctx=ctx)
         fv.per_token_group_quant_fp8(out.view(T, H * D), 128, dxq[i % 2], dxs[i % 2], ctx=ctx)

@@ -124,6 +124,7 @@ class Workload:
     fp8_out: bool = False
     group_quant: bool = False
     margin: float = 1.5
+    per_layer_rings: bool = False  # the seeds are layers of one forward, each with its own ring
     notes: str = ""
     extra: dict = field(default_factory=dict)
 
@@ -170,5 +171,5 @@ WORKLOADS = {
                    (14400, 14400, 14400), 16, 72, "static", (400,), fp8_out=True),
     "3x32400_d72": Workload("3x32400 tokens, 16 heads, head_dim 72, 27 layers, dynamic, group quant",
                    (32400, 32400, 32400), 16, 72, "dynamic", tuple(range(500, 527)),
-                   group_quant=True),
+                   group_quant=True, per_layer_rings=True),
 }

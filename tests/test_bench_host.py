@@ -68,3 +68,15 @@ def test_group_quant_table_is_the_pages_table():
         if t_sol > 0:
             rate = (3 * m * n + 4 * m * n // 128) / (t_sol * 1e-6) / 1e12
             assert 5.0 < rate < 5.6, (m, n, rate)
+
+
+def test_layered_workload_keeps_one_ring_per_layer():
+    """The 3 x 32400 workload is 27 encoder layers, each with its own amax ring;
+    the 8192-token workload is one layer over 20 forwards, one ring."""
+    w = synth.WORKLOADS["3x32400_d72"]
+    assert w.per_layer_rings and len(w.seeds) == 27
+    assert bench._config(w)["rings"] == "one amax ring per layer (27 layers)"
+    assert w.attn_flops() == 3 * 4 * 32400 ** 2 * 72 * 16
+    w2 = synth.WORKLOADS[bench.WORKLOAD]
+    assert not w2.per_layer_rings
+    assert bench._config(w2)["rings"] == "one amax ring over the rotation"

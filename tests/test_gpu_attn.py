@@ -108,7 +108,8 @@ def test_1024_tokens_full_oracle(ctx):
     print("1024 tokens errors", e)
 
 
-@pytest.mark.parametrize("name", ["1x8192_d128", "1x2304_d72", "1x16384_d72", "3x14400_d72", "3x32400_d72"])
+@pytest.mark.parametrize("name", ["1x8192_d128", "1x2304_d72", "1x4096_d72", "1x8192_d72", "1x16384_d72",
+                                  "3x14400_d72", "3x32400_d72"])
 def test_workload_sampled_rows(ctx, name):
     w = synth.WORKLOADS[name]
     q, k, v = w.qkv(0)
