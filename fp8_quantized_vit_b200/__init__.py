@@ -348,8 +348,11 @@ class FP8EncoderAttention:
         [amax ring update] -> per-tensor quantize -> varlen FP8 attention
     (the first two as one cooperative launch on one GPU)
         [-> per-token-group quantize of the output, fused at head_dim 128]
-    on the current stream.  Intermediate FP8 buffers are allocated once per
-    token count and reused (no allocation per call at steady state).
+    on the current stream.  The intermediate FP8 buffers and the output are the
+    layer's own: they grow to the largest token count seen and are reused, so
+    a call allocates nothing once that size has been met, and the tensors a
+    call returns are overwritten by the layer's next call (pass ``out`` to
+    keep an output).
     """
 
     def __init__(self, num_heads: int, head_dim: int, softmax_scale: float | None = None,
@@ -388,14 +391,22 @@ class FP8EncoderAttention:
         self.descale.copy_(torch.tensor(d, dtype=torch.float32))
         self.ring = None
 
-    def _buffers(self, T: int, fp8_out: bool):
-        key = (T, fp8_out)
-        if key not in self._bufs:
+    def _buffers(self, T: int, fp8_out: bool, group_quant: bool = False) -> dict:
+        """Views of the first T tokens of the layer's buffers (one set per
+        output type, reallocated only when T exceeds the capacity held)."""
+        st = self._bufs.get(fp8_out)
+        if st is None or st["cap"] < T:
             shape = (T, self.H, self.D)
             mk = lambda dt: torch.empty(shape, dtype=dt, device=self.device)
-            self._bufs[key] = dict(q8=mk(torch.uint8), k8=mk(torch.uint8), v8=mk(torch.uint8),
-                                   out=mk(torch.uint8 if fp8_out else torch.bfloat16))
-        return self._bufs[key]
+            st = dict(cap=T, q8=mk(torch.uint8), k8=mk(torch.uint8), v8=mk(torch.uint8),
+                      out=mk(torch.uint8 if fp8_out else torch.bfloat16))
+            self._bufs[fp8_out] = st
+        if group_quant and "xq" not in st:
+            hd = self.H * self.D
+            st["xq"] = torch.empty((st["cap"], hd), dtype=torch.uint8, device=self.device)
+            st["xs"] = torch.empty((st["cap"], hd // 128), dtype=torch.float32,
+                                   device=self.device)
+        return {k: v[:T] for k, v in st.items() if k != "cap"}
 
     def forward(self, q, k, v, cu_seqlens, max_seqlen: int, output_scale=None, out=None,
                 group_quant: bool = False):
@@ -408,7 +419,9 @@ class FP8EncoderAttention:
         if group_quant and output_scale is not None:
             raise ValueError("group_quant and output_scale are exclusive")
         T = q.shape[0]
-        b = self._buffers(T, output_scale is not None)
+        if group_quant and (self.H * self.D) % 128 != 0:
+            raise ValueError("group_quant needs num_heads * head_dim to be a multiple of 128")
+        b = self._buffers(T, output_scale is not None, group_quant)
         if self.ring is not None and self.process_group is not None:
             # this rank holds some of the batch's images: agree on the
             # per-tensor amax with the other ranks before the ring update
@@ -425,11 +438,6 @@ class FP8EncoderAttention:
                                         ctx=self.ctx)
         if group_quant:
             hd = self.H * self.D
-            if hd % 128 != 0:
-                raise ValueError("group_quant needs num_heads * head_dim to be a multiple of 128")
-            if "xq" not in b:
-                b["xq"] = torch.empty((T, hd), dtype=torch.uint8, device=self.device)
-                b["xs"] = torch.empty((T, hd // 128), dtype=torch.float32, device=self.device)
             xq, xs = b["xq"], b["xs"]
             if self.D == 128:
                 fp8_varlen_attn_fwd_group_quant(b["q8"], b["k8"], b["v8"], self.descale[0:1],

@@ -9,6 +9,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 import fp8_quantized_vit_b200 as fv
 from fp8_quantized_vit_b200 import _build
@@ -196,3 +197,25 @@ def test_host_argument_checks_need_no_gpu():
                                           dummy, dummy, None) == fv.EINVAL
     assert lib.fp8_amax_ring_quantize_qkv(fake_ctx, dummy, dummy, dummy, 8, odd, dummy, dummy,
                                           dummy, dummy, None) == fv.EINVAL
+
+
+def test_layer_buffers_grow_to_the_largest_token_count_and_are_reused():
+    """The layer keeps one set of buffers per output type, sized for the
+    largest token count seen; a smaller call gets views of their first rows
+    (contiguous, no new allocation), a larger one replaces them."""
+    layer = object.__new__(fv.FP8EncoderAttention)
+    layer.H, layer.D, layer.device, layer._bufs = 16, 72, torch.device("cpu"), {}
+    b = layer._buffers(300, False)
+    assert b["q8"].shape == (300, 16, 72) and b["out"].dtype == torch.bfloat16
+    base = b["q8"].data_ptr()
+    s = layer._buffers(129, False, group_quant=True)
+    assert s["q8"].data_ptr() == base and s["q8"].shape == (129, 16, 72)
+    assert all(t.is_contiguous() for t in s.values())
+    assert s["xq"].shape == (129, 1152) and s["xs"].shape == (129, 9)
+    assert s["out"].view(129, 1152).shape == (129, 1152)
+    assert layer._buffers(300, False)["q8"].data_ptr() == base
+    f = layer._buffers(200, True)
+    assert f["out"].dtype == torch.uint8 and f["q8"].data_ptr() != base
+    g = layer._buffers(301, False)
+    assert g["q8"].shape == (301, 16, 72) and len(layer._bufs) == 2
+    assert layer._bufs[False]["cap"] == 301
