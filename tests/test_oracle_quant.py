@@ -3,7 +3,9 @@
 * amax: brute force over the bf16 values.
 * ring: hand-derived sequences (tests/golden/ring_sequences.txt).
 * per-tensor quantizer and group quantizer: an independent torch-CPU
-  restatement of the rule (torch's fp32 division, clamp and float8 cast).
+  restatement of the rule (torch's fp32 division, clamp and float8 cast),
+  and hand values: scales of exactly 1 and 2 map grid values to the golden
+  e4m3 codes, saturation, ties to the even code.
 """
 import os
 
@@ -126,3 +128,66 @@ def test_group_quant_zero_group_and_clamp():
 def test_group_quant_rejects_ragged_n():
     with pytest.raises(ValueError):
         oracle.group_quant(np.zeros((1, 200), np.uint16), 128)
+
+
+def _golden_grid():
+    """(code, value) of every finite, non-negative-zero row of the golden e4m3
+    table (tests/golden/e4m3_codes.txt, from the OCP format definition)."""
+    path = os.path.join(os.path.dirname(__file__), "golden", "e4m3_codes.txt")
+    rows = []
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        code, val = line.split()
+        v = float(val)
+        if np.isfinite(v) and not (v == 0.0 and np.signbit(v)):
+            rows.append((int(code, 16), v))
+    return rows
+
+
+def _bf16_bits(values) -> np.ndarray:
+    """BF16 bit patterns of values that BF16 holds exactly (every e4m3 value
+    and its doubles do: 3 mantissa bits against BF16's 7)."""
+    f = np.asarray(values, dtype=np.float32)
+    bits = f.view(np.uint32)
+    assert (bits & 0xFFFF == 0).all()
+    return (bits >> 16).astype(np.uint16)
+
+
+def test_per_tensor_quant_hand_values():
+    """With descale 1 (amax-domain value 448) a value on the e4m3 grid maps to
+    its own code; with descale 1/2 (amax 224) twice that value does; beyond
+    ±448 the code saturates; a tie between two codes goes to the even one."""
+    grid = _golden_grid()
+    codes = np.array([c for c, _ in grid], dtype=np.uint8)
+    vals = [v for _, v in grid]
+    d1 = oracle.descale_from_amax(448.0)
+    d_half = oracle.descale_from_amax(224.0)
+    assert d1 == 1.0 and d_half == 0.5
+    assert (oracle.quantize_per_tensor(_bf16_bits(vals), d1) == codes).all()
+    assert (oracle.quantize_per_tensor(_bf16_bits([v / 2 for v in vals]), d_half) == codes).all()
+    sat = oracle.quantize_per_tensor(_bf16_bits([512.0, -1024.0, 464.0]), d1)
+    assert list(sat) == [0x7E, 0xFE, 0x7E]
+    # 1.0625 lies halfway between 1.0 (0x38, mantissa 000) and 1.125 (0x39):
+    # the even code wins; 1.1875 between 1.125 and 1.25 (0x3A) goes up to 0x3A
+    ties = oracle.quantize_per_tensor(_bf16_bits([1.0625, 1.1875, -1.0625]), d1)
+    assert list(ties) == [0x38, 0x3A, 0xB8]
+
+
+def test_group_quant_hand_values():
+    """A group whose amax is 448 has scale 448/448 = 1, so its codes are the
+    grid values' own codes; a group with amax 896 has scale 2 and the codes of
+    half its values; the scales are stored as amax/448 (not its inverse)."""
+    grid = _golden_grid()
+    codes = np.array([c for c, _ in grid], dtype=np.uint8)
+    vals = [v for _, v in grid]
+    k = len(vals)
+    assert 448.0 in vals and k < 128
+    pad = [0.0] * (128 - k)
+    row = vals + pad + [2 * v for v in vals] + pad
+    x = _bf16_bits(row).reshape(1, 256)
+    xq, sc = oracle.group_quant(x, 128)
+    assert sc[0, 0] == np.float32(1.0) and sc[0, 1] == np.float32(2.0)
+    assert (xq[0, :k] == codes).all() and (xq[0, 128:128 + k] == codes).all()
+    assert (xq[0, k:128] == 0).all() and (xq[0, 128 + k:] == 0).all()
