@@ -87,15 +87,16 @@ const char* fp8vit_status_string(fp8vit_status s);
  * `stream`.  Not for production use. */
 fp8vit_status fp8vit_inject_lost_arrival(fp8vit_ctx* ctx, void* stream);
 
-/* Failure injection for tests: until the next fp8vit_check, attention
- * launches on this context (fp8_varlen_attn_fwd and its variants) never
- * announce their first tile of scores, so each CTA's softmax warps give up
- * after their bounded 2 s wait; the kernel then stops its other roles,
- * drains its copies and MMAs, frees TMEM and returns.  fp8vit_check reports
- * FP8VIT_ETIMEOUT (site 113, the softmax wait for the scores, or 119, the
- * issuer's wait for their buffer to be released, whichever gives up first)
- * and clears the injection.  No GPU fault is
- * involved.  Synchronizes `stream`.  Not for production use. */
+/* Failure injection for tests: attention launches on this context
+ * (fp8_varlen_attn_fwd and its variants) never announce their first tile of
+ * scores, so each CTA's softmax warps give up after their bounded 2 s wait;
+ * the kernel then stops its other roles, drains its copies and MMAs, frees
+ * TMEM and returns.  The injection stays set until fp8vit_check returns the
+ * fault it causes: FP8VIT_ETIMEOUT (site 113, the softmax wait for the
+ * scores, or 119, the issuer's wait for their buffer to be released,
+ * whichever gives up first); that check clears it together with the status
+ * word.  A check with no attention launch in between leaves it set.  No GPU
+ * fault is involved.  Synchronizes `stream`.  Not for production use. */
 fp8vit_status fp8vit_inject_attn_timeout(fp8vit_ctx* ctx, void* stream);
 
 /* How many e4m3 terms the probabilities P of fp8_varlen_attn_fwd are kept in
