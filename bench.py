@@ -187,6 +187,84 @@ def _oracle_inputs(w):
     return codes, desc
 
 
+def _sample_rows(cu: np.ndarray, heads: int, per_seg: int, seed: int):
+    """(token, head) rows per image: its first and last rows, the rows on both
+    sides of the first 128-row tile edge, its middle row and seeded random
+    rows, with the heads cycling."""
+    rng = np.random.default_rng(seed)
+    toks, hs = [], []
+    for i in range(len(cu) - 1):
+        a, L = int(cu[i]), int(cu[i + 1] - cu[i])
+        if L <= 0:
+            continue
+        fixed = sorted({0, L - 1, min(127, L - 1), min(128, L - 1), L // 2})
+        rows = fixed + [int(r) for r in rng.integers(0, L, size=max(0, per_seg - len(fixed)))]
+        for n, r in enumerate(rows):
+            toks.append(a + r)
+            hs.append((n + i) % heads)
+    return np.array(toks, dtype=np.int64), np.array(hs, dtype=np.int32)
+
+
+def _attn_error_stats(got: np.ndarray, ref: np.ndarray) -> dict:
+    """Raw max-abs, mean-abs, the max excess over half a BF16 spacing of the
+    exact value (the output format's own rounding) and the cosine."""
+    got = got.astype(np.float64).ravel()
+    ref = ref.astype(np.float64).ravel()
+    d = np.abs(got - ref)
+    a = np.abs(ref)
+    half_ulp = np.where(a > 0, 0.5 * np.exp2(np.floor(np.log2(np.where(a > 0, a, 1.0))) - 7), 0.0)
+    cos = float(np.dot(got, ref) / (np.linalg.norm(got) * np.linalg.norm(ref) + 1e-300))
+    return {"max_abs": float(d.max()), "mean_abs": float(d.mean()),
+            "max_excess_over_bf16_rounding": float(np.maximum(0.0, d - half_ulp).max()),
+            "cos": cos}
+
+
+def _parity_from_outputs(w, codes, desc, got_desc, got_codes, got_out_bits, per_seg=32,
+                         seed=11):
+    """Forward 0 of the workload, as the kernels computed it from a fresh ring,
+    against the oracle: descales and e4m3 codes bit for bit, and the attention
+    output on sampled (token, head) rows (fp64 oracle rows, computed one by
+    one) against the gate max-abs 3e-2 over the BF16 rounding, mean-abs 3e-3,
+    cosine 0.999."""
+    import oracle
+    import synth
+    cu = synth.cu_seqlens(w.seg_lens)
+    want_desc = np.asarray(desc, dtype=np.float32)
+    desc_exact = bool((np.asarray(got_desc, dtype=np.float32).view(np.uint32) ==
+                       want_desc.view(np.uint32)).all())
+    codes_exact = bool(all(np.array_equal(np.asarray(g).reshape(-1), np.asarray(c).reshape(-1))
+                           for g, c in zip(got_codes, codes)))
+    toks, hs = _sample_rows(cu, w.heads, per_seg, seed)
+    ref = oracle.attn_pairs(*codes, *desc, cu, w.heads, w.head_dim, w.softmax_scale, toks, hs)
+    got = synth.bf16_to_float(np.ascontiguousarray(got_out_bits[toks, hs])).astype(np.float64)
+    e = _attn_error_stats(got, ref)
+    e.update({"rows": int(len(toks)), "descales_bit_exact": desc_exact,
+              "codes_bit_exact": codes_exact,
+              "within_gate": bool(desc_exact and codes_exact and
+                                  e["max_excess_over_bf16_rounding"] <= 3e-2 and
+                                  e["mean_abs"] <= 3e-3 and e["cos"] >= 0.999)})
+    return e
+
+
+def _forward0_outputs(fv, ctx, w, qkv0, cu_d, max_s, q8, k8, v8, out, dev):
+    """Runs forward 0 again from a fresh ring (after the timed region) and
+    returns what the kernels produced: descales, e4m3 codes, BF16 output bits
+    (host arrays; compared with the oracle by the CPU-baseline leg)."""
+    import torch
+    ring0 = fv.new_ring(dev)
+    desc0 = torch.zeros(3, dtype=torch.float32, device=dev)
+    fv.fp8_amax_ring_quantize_qkv(*qkv0, ring0, desc0, q8, k8, v8, ctx=ctx)
+    fv.fp8_varlen_attn_fwd(q8, k8, v8, desc0[0:1], desc0[1:2], desc0[2:3], cu_d, max_s,
+                           w.softmax_scale, out, ctx=ctx)
+    st, site = ctx.check()
+    if st != fv.OK:
+        raise RuntimeError(f"device fault in the parity forward: {fv.status_string(st)} "
+                           f"site {site}")
+    got_out = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    got_codes = [t.cpu().numpy() for t in (q8, k8, v8)]
+    return desc0.cpu().numpy(), got_codes, got_out
+
+
 def run_reference(args):
     """The oracle (plain single-threaded C, run on rows of its own by every
     host thread) as the reference arm."""
@@ -623,6 +701,16 @@ def run_ours(args):
     h2d = 3 * T * H * D * 2
     d2h = xq.numel() + xs.numel() * 4
 
+    # forward 0 once more from a fresh ring (untimed), for the CPU-baseline
+    # leg's full-size parity check
+    cpu_leg = rank == 0 and ws == 1 and not args.no_cpu_baseline
+    fwd0 = None
+    if cpu_leg:
+        try:
+            fwd0 = _forward0_outputs(fv, ctx, w, inputs[0], cu, max_s, q8, k8, v8, out, dev)
+        except Exception as exc:  # reported in the line's parity field, not dropped
+            fwd0 = exc
+
     peaks = _peaks()
     fp8_peak = 2.0 * peaks["bf16"]  # dense FP8 = 2 x dense BF16 (nominal ratio)
     quant = None if args.no_quant_roofline else _quant_rooflines(fv, ctx, inputs[0], dev,
@@ -655,7 +743,7 @@ def run_ours(args):
         line["group_quant_table"] = _group_quant_table(fv, ctx, dev, peaks["hbm"])
     if args.attn_sweep:
         line["attn_sweep"] = _attn_sweep(fv, ctx, dev)
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+    if cpu_leg:
         codes, dsc = _oracle_inputs(w)
         threads = _host_threads()
         per_thread = max(1.0, args.cpu_seconds / threads)
@@ -665,7 +753,10 @@ def run_ours(args):
             "sample": f"{rows} seeded (token, head) query rows of forward 0's attention, "
                       f"{threads} host threads each running the single-threaded oracle on rows "
                       f"of its own for {per_thread:.1f} s ({sec:.1f} s wall; amax/quantize "
-                      f"stages excluded)"}
+                      f"stages excluded)",
+            # the same oracle, on the kernels' forward 0 at full size
+            "parity_of_forward0": ({"error": repr(fwd0)} if isinstance(fwd0, Exception)
+                                   else _parity_from_outputs(w, codes, dsc, *fwd0))}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:

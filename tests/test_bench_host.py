@@ -1,7 +1,9 @@
 """CPU checks of the benchmark's host logic: the traffic record is used only
 for the kernel source it was captured on, the workload description names
-the shape, the roofline denominators come from the measured peaks, and the
-group-quantizer table holds the benchmark page's 19 shapes."""
+the shape, the roofline denominators come from the measured peaks, the
+group-quantizer table holds the benchmark page's 19 shapes, and the CPU
+leg's full-size parity check of forward 0 passes exact outputs and catches
+wrong ones."""
 import hashlib
 import json
 import os
@@ -80,3 +82,76 @@ def test_layered_workload_keeps_one_ring_per_layer():
     w2 = synth.WORKLOADS[bench.WORKLOAD]
     assert not w2.per_layer_rings
     assert bench._config(w2)["rings"] == "one amax ring over the rotation"
+
+
+def test_forward0_parity_check_on_the_host():
+    """The CPU-baseline leg's full-size parity check: exact descales and codes
+    with the oracle's rows rounded to BF16 pass; a wrong row, a wrong code or a
+    descale one ulp off fail."""
+    import numpy as np
+    import torch
+
+    import oracle
+    w = synth.Workload("2 images, 300 + 77 tokens, 2 heads, head_dim 72", (300, 77), 2, 72,
+                       "dynamic", (5,))
+    codes, desc = bench._oracle_inputs(w)
+    cu = synth.cu_seqlens(w.seg_lens)
+    ref = oracle.attn_full(*codes, *desc, cu, w.heads, w.head_dim, w.softmax_scale)
+    bits = torch.from_numpy(ref).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    good = bench._parity_from_outputs(w, codes, desc, np.asarray(desc, np.float32), codes, bits)
+    assert good["within_gate"] and good["descales_bit_exact"] and good["codes_bit_exact"]
+    assert good["max_excess_over_bf16_rounding"] < 1e-6 and good["cos"] > 0.99999
+    assert good["rows"] == 2 * 32
+
+    toks, hs = bench._sample_rows(cu, w.heads, 32, 11)
+    assert ((toks >= 0) & (toks < 377)).all() and set(hs.tolist()) == {0, 1}
+    assert {0, 127, 128, 299, 300, 376} <= set(toks.tolist())
+    bad = bits.copy()
+    bad[toks[3], hs[3]] ^= 0x0400  # one output off by many BF16 steps
+    assert not bench._parity_from_outputs(w, codes, desc, desc, codes, bad)["within_gate"]
+    wrong_codes = [c.copy() for c in codes]
+    wrong_codes[1].reshape(-1)[7] ^= 1
+    e = bench._parity_from_outputs(w, codes, desc, desc, wrong_codes, bits)
+    assert not e["codes_bit_exact"] and not e["within_gate"]
+    off = np.asarray(desc, np.float32).copy()
+    off.view(np.uint32)[2] += 1
+    e = bench._parity_from_outputs(w, codes, desc, off, codes, bits)
+    assert not e["descales_bit_exact"] and not e["within_gate"]
+
+
+def test_forward0_capture_marshals_the_kernels_outputs():
+    """The bench's forward-0 capture, with the library's calls replaced by
+    host stand-ins that write known bytes: it returns the descales, the three
+    code tensors and the BF16 output bits as host arrays of the right shapes."""
+    import types
+
+    import numpy as np
+    import torch
+
+    T, H, D = 40, 2, 72
+    w = synth.Workload("1 image, 40 tokens", (T,), H, D, "dynamic", (1,))
+    calls = []
+
+    def quant(q, k, v, ring, desc, q8, k8, v8, ctx=None):
+        calls.append("quant")
+        desc.copy_(torch.tensor([0.5, 0.25, 0.125]))
+        for i, t in enumerate((q8, k8, v8)):
+            t.fill_(i + 1)
+
+    def attn(q8, k8, v8, dq, dk, dv, cu, max_s, sm, out, ctx=None):
+        calls.append(("attn", float(dq[0]), float(dv[0]), max_s))
+        out.fill_(1.5)
+
+    fake = types.SimpleNamespace(
+        new_ring=lambda dev: torch.zeros(64), OK=0, status_string=str,
+        fp8_amax_ring_quantize_qkv=quant, fp8_varlen_attn_fwd=attn)
+    ctx = types.SimpleNamespace(check=lambda: (0, 0))
+    qkv0 = [torch.zeros((T, H, D), dtype=torch.bfloat16) for _ in range(3)]
+    q8, k8, v8 = (torch.zeros((T, H, D), dtype=torch.uint8) for _ in range(3))
+    out = torch.zeros((T, H, D), dtype=torch.bfloat16)
+    desc, codes, bits = bench._forward0_outputs(fake, ctx, w, qkv0, torch.zeros(2), T, q8, k8, v8,
+                                                out, "cpu")
+    assert calls == ["quant", ("attn", 0.5, 0.125, T)]
+    assert desc.dtype == np.float32 and list(desc) == [0.5, 0.25, 0.125]
+    assert [c.shape for c in codes] == [(T, H, D)] * 3 and [int(c[0, 0, 0]) for c in codes] == [1, 2, 3]
+    assert bits.dtype == np.uint16 and bits.shape == (T, H, D) and (bits == 0x3FC0).all()
