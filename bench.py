@@ -246,6 +246,17 @@ def _parity_from_outputs(w, codes, desc, got_desc, got_codes, got_out_bits, per_
     return e
 
 
+def _parity_field(w, codes, desc, fwd0) -> dict:
+    """The line's parity record; a failure of the check itself is reported in
+    the record (with the exception) instead of costing the whole line."""
+    if isinstance(fwd0, Exception):
+        return {"error": repr(fwd0)}
+    try:
+        return _parity_from_outputs(w, codes, desc, *fwd0)
+    except Exception as exc:  # reported, not dropped
+        return {"error": repr(exc)}
+
+
 def _forward0_outputs(fv, ctx, w, qkv0, cu_d, max_s, q8, k8, v8, out, dev):
     """Runs forward 0 again from a fresh ring (after the timed region) and
     returns what the kernels produced: descales, e4m3 codes, BF16 output bits
@@ -755,8 +766,7 @@ def run_ours(args):
                       f"of its own for {per_thread:.1f} s ({sec:.1f} s wall; amax/quantize "
                       f"stages excluded)",
             # the same oracle, on the kernels' forward 0 at full size
-            "parity_of_forward0": ({"error": repr(fwd0)} if isinstance(fwd0, Exception)
-                                   else _parity_from_outputs(w, codes, dsc, *fwd0))}
+            "parity_of_forward0": _parity_field(w, codes, dsc, fwd0)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:

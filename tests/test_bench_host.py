@@ -155,3 +155,9 @@ def test_forward0_capture_marshals_the_kernels_outputs():
     assert desc.dtype == np.float32 and list(desc) == [0.5, 0.25, 0.125]
     assert [c.shape for c in codes] == [(T, H, D)] * 3 and [int(c[0, 0, 0]) for c in codes] == [1, 2, 3]
     assert bits.dtype == np.uint16 and bits.shape == (T, H, D) and (bits == 0x3FC0).all()
+
+
+def test_parity_field_reports_a_failed_check():
+    assert bench._parity_field(None, None, None, RuntimeError("fault"))["error"].startswith(
+        "RuntimeError")
+    assert "error" in bench._parity_field(None, None, None, (None, None, None))
