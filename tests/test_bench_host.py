@@ -161,3 +161,24 @@ def test_parity_field_reports_a_failed_check():
     assert bench._parity_field(None, None, None, RuntimeError("fault"))["error"].startswith(
         "RuntimeError")
     assert "error" in bench._parity_field(None, None, None, (None, None, None))
+
+
+def test_bench_line_carries_every_contract_key():
+    """The JSON line built by the GPU arm names every key of the benchmark
+    contract (read from the source: the arm itself needs a GPU)."""
+    import ast
+    src = open(bench.__file__).read()
+    tree = ast.parse(src)
+    run = next(n for n in tree.body if isinstance(n, ast.FunctionDef) and n.name == "run_ours")
+    keys = set()
+    for node in ast.walk(run):
+        if isinstance(node, ast.Dict):
+            keys |= {k.value for k in node.keys if isinstance(k, ast.Constant)}
+        if isinstance(node, ast.Subscript) and isinstance(node.slice, ast.Constant):
+            keys.add(node.slice.value)
+    need = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+            "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "roofline",
+            "bound", "achieved", "peak", "frac", "traffic", "e2e", "h2d_bytes_per_step",
+            "d2h_bytes_per_step", "gpu_launches", "clocks", "cpu_baseline", "cores", "kind",
+            "sample", "parity_of_forward0"}
+    assert need <= keys, need - keys
