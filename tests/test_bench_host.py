@@ -182,3 +182,16 @@ def test_bench_line_carries_every_contract_key():
             "d2h_bytes_per_step", "gpu_launches", "clocks", "cpu_baseline", "cores", "kind",
             "sample", "parity_of_forward0"}
     assert need <= keys, need - keys
+
+
+def test_reference_arm_prints_its_line(capsys):
+    """`--impl reference` (the oracle on the host cores) prints one line with
+    the contract keys, its own e2e and cpu_baseline, and impl = reference."""
+    import types
+    args = types.SimpleNamespace(workload="1x1024_d72", steps=1, warmup=0, ref_step_seconds=0.2)
+    assert bench.run_reference(args) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["value"] == line["value"] and line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["config"]["workload"].startswith("1x1024 tokens")
