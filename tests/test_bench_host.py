@@ -195,3 +195,15 @@ def test_reference_arm_prints_its_line(capsys):
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["value"] == line["value"] and line["e2e"]["h2d_bytes_per_step"] == 0
     assert line["config"]["workload"].startswith("1x1024 tokens")
+
+
+def test_reference_arm_runs_on_rank_0_only(capsys, monkeypatch):
+    """Under torchrun with N > 1 only rank 0 runs the oracle and prints; the
+    other ranks exit 0 without work."""
+    import types
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("LOCAL_RANK", "1")
+    args = types.SimpleNamespace(workload="1x1024_d72", steps=1, warmup=0, ref_step_seconds=0.2)
+    assert bench.run_reference(args) == 0
+    assert capsys.readouterr().out.strip() == ""
