@@ -17,6 +17,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+import threading
 
 import torch
 
@@ -59,6 +60,7 @@ _SIGNATURES = {
 }
 
 _lib = None
+_lock = threading.RLock()  # library loading and the per-device default contexts
 
 
 class FP8VitError(RuntimeError):
@@ -71,15 +73,17 @@ def lib():
     """The loaded libfp8vit.so; raises if it has not been built."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
-                               "`python -m fp8_quantized_vit_b200._build`")
-        handle = ctypes.CDLL(LIB_PATH)
-        for name, (res, args) in _SIGNATURES.items():
-            fn = getattr(handle, name)
-            fn.restype = res
-            fn.argtypes = args
-        _lib = handle
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(LIB_PATH):
+                    raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                       "`python -m fp8_quantized_vit_b200._build`")
+                handle = ctypes.CDLL(LIB_PATH)
+                for name, (res, args) in _SIGNATURES.items():
+                    fn = getattr(handle, name)
+                    fn.restype = res
+                    fn.argtypes = args
+                _lib = handle
     return _lib
 
 
@@ -152,10 +156,12 @@ _default_ctx: dict[int, Context] = {}
 
 
 def default_context() -> Context:
+    """The shared context of the current device (created on first use)."""
     dev = torch.cuda.current_device()
-    if dev not in _default_ctx:
-        _default_ctx[dev] = Context(dev)
-    return _default_ctx[dev]
+    with _lock:
+        if dev not in _default_ctx:
+            _default_ctx[dev] = Context(dev)
+        return _default_ctx[dev]
 
 
 def _ctx(ctx):
