@@ -35,6 +35,13 @@ MUTANTS = [
     ("group amax over half the group", "for (int32_t i = 0; i < group; ++i) {\n                float a = fabsf",
      "for (int32_t i = 0; i < group / 2; ++i) {\n                float a = fabsf"),
     ("group scale not divided by 448", "float s = amax / 448.0f;", "float s = amax / 240.0f;"),
+    ("group scale floor dropped", "if (s < ORC_SCALE_FLOOR) s = ORC_SCALE_FLOOR;", ""),
+    ("group amax of signed values", "float a = fabsf(orc_bf16_to_float(xs[i]));",
+     "float a = orc_bf16_to_float(xs[i]);"),
+    ("group quantize multiplies by the scale", "float y = orc_bf16_to_float(xs[i]) / s;",
+     "float y = orc_bf16_to_float(xs[i]) * s;"),
+    ("per-tensor quantize multiplies by the descale", "orc_bf16_to_float(x[i]) / descale);",
+     "orc_bf16_to_float(x[i]) * descale);"),
     ("softmax scale dropped", "s[j - a] = (double)sm_scale * acc;", "s[j - a] = acc;"),
     ("key of head 0", "const uint8_t* kj = k8 + j * row + (int64_t)h * D;",
      "const uint8_t* kj = k8 + j * row;"),
@@ -90,8 +97,17 @@ def _pins():
     got = [float(ring.update([a, a, a])[0]) for a in range(20, 0, -1)]
     want = [oracle.descale_from_amax(m) for m in [20.0] * 16 + [19.0, 18.0, 17.0, 16.0]]
     out["ring"] = got == want and int(ring.pos[0]) == 4
-    # group quant vs a torch restatement
+    # per-tensor quantize vs a torch restatement, and two hand values
+    xp = synth.bf16_tensor(synth.stream_key(4, 1, 1), 5, 256)
+    d = np.float32(1.5) * np.float32(oracle.amax_bf16(xp)) / np.float32(448.0)
+    rp = (_bf16(xp).float() / torch.tensor(d)).clamp(-448, 448).to(torch.float8_e4m3fn)
+    out["per-tensor quant"] = bool(
+        (oracle.quantize_per_tensor(xp, float(d)).reshape(-1) ==
+         rp.view(torch.uint8).numpy().reshape(-1)).all() and
+        list(oracle.quantize_per_tensor(np.array([0x4000, 0xC080], np.uint16), 0.5)) == [0x48, 0xD0])
+    # group quant vs a torch restatement (row 0's first group all zeros)
     xg = synth.bf16_tensor(synth.stream_key(3, 1, 1), 7, 512)
+    xg[0, :128] = 0
     xq, sc = oracle.group_quant(xg, 128)
     t = _bf16(xg).float().reshape(7, 4, 128)
     s = torch.clamp(t.abs().amax(-1) / 448.0, min=1e-10)
