@@ -368,6 +368,57 @@ def _bf16_comparator(fv, ctx, w, inputs, dev, reps=10):
             "tflops": w.attn_flops() / (ms * 1e-3) / 1e12}
 
 
+def _output_modes(fv, ctx, w, inputs, dev, reps=10, rounds=3):
+    """The attention call's output epilogues on the same e4m3 inputs (static
+    scales, 1.5 x the exact amax): BF16 output, FP8 output through an
+    output_scale (the amax of the BF16 output / 448), and at head_dim 128 the
+    fused group-128 quantizer.  Each mode is timed over `reps` launches
+    between two events, in `rounds` alternating rounds; the best round
+    counts."""
+    import torch
+    import synth
+    T, H, D = w.tokens, w.heads, w.head_dim
+    q, k, v = inputs[0]
+    cu = torch.from_numpy(synth.cu_seqlens(w.seg_lens)).to(dev)
+    amax3 = torch.zeros(3, dtype=torch.float32, device=dev)
+    fv.fp8_amax3(q, k, v, amax3, ctx=ctx)
+    desc = torch.tensor([fv.fp8_descale_from_amax(float(np.float32(1.5) * np.float32(a)))
+                         for a in amax3.cpu().numpy()], dtype=torch.float32, device=dev)
+    q8, k8, v8 = (torch.empty((T, H, D), dtype=torch.uint8, device=dev) for _ in range(3))
+    fv.fp8_quantize_qkv_per_tensor(q, k, v, desc, q8, k8, v8, ctx=ctx)
+    call = (q8, k8, v8, desc[0:1], desc[1:2], desc[2:3], cu, max(w.seg_lens), w.softmax_scale)
+    out = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    fv.fp8_varlen_attn_fwd(*call, out, ctx=ctx)
+    oscale = (out.float().abs().max() / 448.0).reshape(1).contiguous()
+    out8 = torch.empty((T, H, D), dtype=torch.uint8, device=dev)
+    runs = {"bf16": lambda: fv.fp8_varlen_attn_fwd(*call, out, ctx=ctx),
+            "fp8_output_scale": lambda: fv.fp8_varlen_attn_fwd(*call, out8, output_scale=oscale,
+                                                               ctx=ctx)}
+    if D == 128:
+        xq = torch.empty((T, H * D), dtype=torch.uint8, device=dev)
+        xs = torch.empty((T, H * D // 128), dtype=torch.float32, device=dev)
+        runs["fused_group_quant"] = lambda: fv.fp8_varlen_attn_fwd_group_quant(*call, xq, xs,
+                                                                               ctx=ctx)
+    best = {name: float("inf") for name in runs}
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    for _ in range(rounds):
+        for name, run in runs.items():
+            run()
+            e0.record()
+            for _ in range(reps):
+                run()
+            e1.record()
+            torch.cuda.synchronize()
+            best[name] = min(best[name], e0.elapsed_time(e1) / reps)
+    st, site = ctx.check()
+    if st != fv.OK:
+        raise RuntimeError(f"device fault in the output-mode timing: {fv.status_string(st)} "
+                           f"site {site}")
+    flops = w.attn_flops()
+    return {name: {"ms": ms, "tflops": flops / (ms * 1e-3) / 1e12} for name, ms in best.items()}
+
+
 # The shapes of atrex-bench "#025 per_token_group_quant_fp8" (token_count x
 # hidden_size), with the pages' speed-of-light and production times on their
 # hardware ("XPU-A"), in microseconds: context for the same kernel on B200.
@@ -754,6 +805,8 @@ def run_ours(args):
         line["group_quant_table"] = _group_quant_table(fv, ctx, dev, peaks["hbm"])
     if args.attn_sweep:
         line["attn_sweep"] = _attn_sweep(fv, ctx, dev)
+    if args.output_modes:
+        line["output_modes"] = _output_modes(fv, ctx, w, inputs, dev)
     if cpu_leg:
         codes, dsc = _oracle_inputs(w)
         threads = _host_threads()
@@ -797,6 +850,9 @@ def main():
                     help="also time torch BF16 SDPA on the same inputs (single-image workloads)")
     ap.add_argument("--compare-bf16", action="store_true",
                     help="also time this library's BF16 attention kernel on the same inputs")
+    ap.add_argument("--output-modes", action="store_true",
+                    help="also time the attention call with BF16 output, FP8 output "
+                         "(output_scale) and, at head_dim 128, the fused group quantizer")
     ap.add_argument("--attn-sweep", action="store_true",
                     help="also time the pages' attention tables (head_dim-72 sequence sweep, "
                          "8192-token head_dim 128): FP8 with and without quantization, BF16")

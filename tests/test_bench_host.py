@@ -132,13 +132,21 @@ def test_forward0_capture_marshals_the_kernels_outputs():
     w = synth.Workload("1 image, 40 tokens", (T,), H, D, "dynamic", (1,))
     calls = []
 
+    import inspect
+
+    import fp8_quantized_vit_b200 as fv
+
     def quant(q, k, v, ring, desc, q8, k8, v8, ctx=None):
+        inspect.signature(fv.fp8_amax_ring_quantize_qkv).bind(q, k, v, ring, desc, q8, k8, v8,
+                                                              ctx=ctx)
         calls.append("quant")
         desc.copy_(torch.tensor([0.5, 0.25, 0.125]))
         for i, t in enumerate((q8, k8, v8)):
             t.fill_(i + 1)
 
     def attn(q8, k8, v8, dq, dk, dv, cu, max_s, sm, out, ctx=None):
+        inspect.signature(fv.fp8_varlen_attn_fwd).bind(q8, k8, v8, dq, dk, dv, cu, max_s, sm, out,
+                                                       ctx=ctx)
         calls.append(("attn", float(dq[0]), float(dv[0]), max_s))
         out.fill_(1.5)
 
@@ -207,3 +215,67 @@ def test_reference_arm_runs_on_rank_0_only(capsys, monkeypatch):
     args = types.SimpleNamespace(workload="1x1024_d72", steps=1, warmup=0, ref_step_seconds=0.2)
     assert bench.run_reference(args) == 0
     assert capsys.readouterr().out.strip() == ""
+
+
+def test_output_modes_leg_calls_the_binding_as_declared(monkeypatch):
+    """The optional output-mode timing leg, run on the CPU with stand-ins for
+    the library calls and the CUDA events: every call binds to the real
+    binding's signature, each mode runs, and the result has one entry per mode
+    (three at head_dim 128)."""
+    import inspect
+    import types
+
+    import numpy as np
+    import torch
+
+    import fp8_quantized_vit_b200 as fv
+
+    seen = []
+
+    def stand_in(name, effect=None):
+        sig = inspect.signature(getattr(fv, name))
+
+        def f(*a, **k):
+            sig.bind(*a, **k)
+            seen.append(name)
+            if effect:
+                effect(*a, **k)
+        return f
+
+    def amax3(q, k, v, out, ctx=None):
+        out.copy_(torch.tensor([3.0, 4.0, 5.0]))
+
+    def attn(*a, **k):
+        a[9].fill_(1 if a[9].dtype == torch.uint8 else 2.0)
+
+    fake = types.SimpleNamespace(
+        OK=0, status_string=str,
+        fp8_amax3=stand_in("fp8_amax3", amax3),
+        fp8_descale_from_amax=lambda v: float(np.float32(v) / np.float32(448.0)),
+        fp8_quantize_qkv_per_tensor=stand_in("fp8_quantize_qkv_per_tensor"),
+        fp8_varlen_attn_fwd=stand_in("fp8_varlen_attn_fwd", attn),
+        fp8_varlen_attn_fwd_group_quant=stand_in("fp8_varlen_attn_fwd_group_quant"))
+    ctx = types.SimpleNamespace(check=lambda: (0, 0))
+
+    class Ev:
+        def __init__(self, enable_timing=False):
+            pass
+
+        def record(self, stream=None):
+            pass
+
+        def elapsed_time(self, other):
+            return 1.0
+
+    monkeypatch.setattr(torch.cuda, "Event", Ev)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a: None)
+    for D in (72, 128):
+        w = synth.Workload("1 image, 64 tokens", (64,), 2, D, "static", (1,))
+        inputs = [[torch.zeros((64, 2, D), dtype=torch.bfloat16) for _ in range(3)]]
+        seen.clear()
+        res = bench._output_modes(fake, ctx, w, inputs, "cpu", reps=2, rounds=1)
+        want = {"bf16", "fp8_output_scale"} | ({"fused_group_quant"} if D == 128 else set())
+        assert set(res) == want
+        assert all(r["ms"] == 0.5 and r["tflops"] > 0 for r in res.values())
+        assert seen[:2] == ["fp8_amax3", "fp8_quantize_qkv_per_tensor"]
+        assert ("fp8_varlen_attn_fwd_group_quant" in seen) == (D == 128)
