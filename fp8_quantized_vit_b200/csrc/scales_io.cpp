@@ -160,6 +160,8 @@ fp8vit_status parse_layer(Reader& r, float out[3]) {
             }
             double v;
             if (!r.number(&v)) return FP8VIT_EPARSE;
+            // an amax-domain value: non-negative and finite as the fp32 it is used as
+            if (!(v >= 0.0) || !std::isfinite((float)v)) return FP8VIT_EPARSE;
             if (have[which] && (float)val[which] != (float)v) return FP8VIT_EPARSE;
             have[which] = true;
             val[which] = v;

@@ -300,7 +300,8 @@ fp8vit_status per_token_group_quant_fp8(fp8vit_ctx* ctx, const uint16_t* d_x, in
  * with "q_scale"/"k_scale"/"v_scale" accepted as aliases (both spellings
  * with different values is FP8VIT_EPARSE).  The numbers are in the amax
  * domain (margin x observed amax); fp8_descale_from_amax turns one into a
- * descale.  Host only; no CUDA call. */
+ * descale.  A negative value, or one that is not finite as fp32, is
+ * FP8VIT_EPARSE.  Host only; no CUDA call. */
 fp8vit_status fp8_static_scales_load(const char* path, const char* layer, float out_qkv[3]);
 
 /* Write the scale file for n_layers layers: layer i gets

@@ -92,7 +92,10 @@ def test_scale_file_aliases_and_errors(tmp_path):
                  '{"a": {"q": 1, "q_scale": 2, "k": 1, "v": 1}}',  # conflicting alias
                  '{"a": {"q": 1, "k": 2, "v": 3}',                 # truncated
                  '{"a": {"q": "x", "k": 2, "v": 3}}',              # not a number
-                 '{"a": {"q": 1, "k": 2, "v": 3}} trailing']:
+                 '{"a": {"q": 1, "k": 2, "v": 3}} trailing',
+                 '{"a": {"q": -1, "k": 2, "v": 3}}',               # an amax is not negative
+                 '{"a": {"q": 1, "k": 1e39, "v": 3}}',             # beyond fp32
+                 '{"a": {"q": 1, "k": 2, "v": 1e99999}}']:         # beyond fp64
         bad.write_text(text)
         with pytest.raises(fv.FP8VitError) as e:
             fv.fp8_static_scales_load(str(bad), "a")
@@ -219,3 +222,44 @@ def test_layer_buffers_grow_to_the_largest_token_count_and_are_reused():
     g = layer._buffers(301, False)
     assert g["q8"].shape == (301, 16, 72) and len(layer._bufs) == 2
     assert layer._bufs[False]["cap"] == 301
+
+
+def test_scale_file_loader_survives_damaged_files(tmp_path):
+    """Every prefix of a valid scale file, and files with seeded byte damage,
+    load or fail with a status (no crash, no read past the text); a file the
+    loader accepts gives finite values.  Run in a child process, so that a
+    crash in the C++ reader fails this test instead of the whole session."""
+    import subprocess
+    import sys
+    script = r'''
+import os, random, sys
+sys.path.insert(0, sys.argv[1])
+import fp8_quantized_vit_b200 as fv
+text = open(sys.argv[2], "rb").read()
+p = os.path.join(sys.argv[3], "d.json")
+rng = random.Random(7)
+cases = [text[:i] for i in range(len(text) + 1)]
+for _ in range(400):
+    b = bytearray(text)
+    for _ in range(rng.randint(1, 4)):
+        b[rng.randrange(len(b))] = rng.choice(b'{}[]":,.-+eE0123456789 \\\x00\xff')
+    cases.append(bytes(b))
+cases += [b"", b"{", b'{"a":', b'{"a": {"q": 1e99999, "k": 1, "v": 1}}', b"[" * 5000,
+          b'{"a": {"q": -1, "k": 1, "v": 1}}', b'"' + b"x" * 100000]
+ok = bad = 0
+for c in cases:
+    open(p, "wb").write(c)
+    try:
+        vals = fv.fp8_static_scales_load(p, "visual.blocks.0.attn.attn")
+        assert all(v == v and abs(v) != float("inf") for v in vals), vals
+        ok += 1
+    except fv.FP8VitError as e:
+        assert e.status in (fv.EPARSE, fv.ENOTFOUND, fv.EIO), e.status
+        bad += 1
+print(ok, bad)
+'''
+    r = subprocess.run([sys.executable, "-c", script, ROOT, GOLDEN, str(tmp_path)],
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    ok, bad = map(int, r.stdout.split())
+    assert ok >= 1 and bad >= 100
