@@ -263,3 +263,22 @@ print(ok, bad)
     assert r.returncode == 0, r.stderr[-2000:]
     ok, bad = map(int, r.stdout.split())
     assert ok >= 1 and bad >= 100
+
+
+def test_boundary_is_usable_from_plain_c(tmp_path):
+    """A C11 program that includes only include/fp8vit.h, compiled with
+    warnings as errors and linked against libfp8vit.so, runs the calls that
+    need no GPU (tests/abi_from_c.c)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    exe = tmp_path / "abi_from_c"
+    libdir = os.path.dirname(fv.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror",
+                           "-I", os.path.join(ROOT, "include"),
+                           os.path.join(ROOT, "tests", "abi_from_c.c"), "-L", libdir, "-lfp8vit",
+                           f"-Wl,-rpath,{libdir}", "-lm", "-o", str(exe)])
+    r = subprocess.run([str(exe), GOLDEN, str(tmp_path / "s.json")], capture_output=True,
+                       text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stderr)
