@@ -6,7 +6,8 @@ the current CUDA stream.  The library must be built (``__graft_entry__.build``
 or ``python -m fp8_quantized_vit_b200._build``); there is no fallback.
 
 Entry points (same names as the C ABI):
-  fp8_amax_ring_update, fp8_amax3, fp8_ring_push, fp8_quantize_qkv_per_tensor,
+  fp8_amax_ring_update, fp8_amax_ring_update_noalloc, fp8_amax3, fp8_ring_push,
+  fp8_quantize_qkv_per_tensor,
   fp8_varlen_attn_fwd, per_token_group_quant_fp8, fp8_static_scales_load,
   fp8_static_scales_save, fp8_descale_from_amax, fp8_ring_read_amax, ring_init
 and ``FP8EncoderAttention``, which chains them for one attention layer
@@ -41,6 +42,7 @@ _SIGNATURES = {
     "fp8vit_version": (_I32, []),
     "fp8vit_ring_init": (_I32, [_P, _P]),
     "fp8_amax_ring_update": (_I32, [_P, _P, _P, _P, _I64, _P, _P, _P]),
+    "fp8_amax_ring_update_noalloc": (_I32, [_P, _P, _P, _I64, _P, _P, _P]),
     "fp8_ring_read_amax": (_I32, [_P, _P, _P]),
     "fp8_amax3": (_I32, [_P, _P, _P, _P, _I64, _P, _P]),
     "fp8_ring_push": (_I32, [_P, _P, _P, _P]),
@@ -190,6 +192,22 @@ def fp8_amax_ring_update(q, k, v, ring, descale3, ctx=None, stream=None):
         _ctx(ctx), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
         _ptr(v, torch.bfloat16, "v"), n, _ptr(ring, torch.float32, "ring"),
         _ptr(descale3, torch.float32, "descale3"), _stream(stream)), "fp8_amax_ring_update")
+    return descale3
+
+
+def fp8_amax_ring_update_noalloc(q, k, v, ring, descale3, stream=None):
+    """fp8_amax_ring_update without a context: the reduction scratch is a
+    fixed array inside the library, shared by every call on the device, so
+    calls that overlap on the GPU must not use it (order them, or use a
+    context).  The first call on a device must come before any stream
+    capture on it."""
+    n = q.numel()
+    if k.numel() != n or v.numel() != n:
+        raise ValueError("q, k, v must have the same number of elements")
+    _check(lib().fp8_amax_ring_update_noalloc(
+        _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"), _ptr(v, torch.bfloat16, "v"),
+        n, _ptr(ring, torch.float32, "ring"), _ptr(descale3, torch.float32, "descale3"),
+        _stream(stream)), "fp8_amax_ring_update_noalloc")
     return descale3
 
 

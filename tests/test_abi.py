@@ -282,3 +282,14 @@ def test_boundary_is_usable_from_plain_c(tmp_path):
     r = subprocess.run([str(exe), GOLDEN, str(tmp_path / "s.json")], capture_output=True,
                        text=True, timeout=60)
     assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stderr)
+
+
+def test_noalloc_entry_point_is_bound_and_checks_on_the_host():
+    lib = fv.lib()
+    dummy = ctypes.c_void_p(0x10000)  # never dereferenced: the checks return first
+    f = lib.fp8_amax_ring_update_noalloc
+    assert f.argtypes is not None and len(f.argtypes) == 7
+    assert f(None, dummy, dummy, 8, dummy, dummy, None) == fv.EINVAL
+    assert f(dummy, dummy, dummy, -1, dummy, dummy, None) == fv.EINVAL
+    assert f(ctypes.c_void_p(0x10002), dummy, dummy, 8, dummy, dummy, None) == fv.EINVAL
+    assert callable(fv.fp8_amax_ring_update_noalloc)
