@@ -859,9 +859,29 @@ def main():
     ap.add_argument("--group-quant-table", action="store_true",
                     help="also time the group quantizer on the shapes of the pages' table")
     args = ap.parse_args()
+    ws = int(os.environ.get("WORLD_SIZE", "0"))
+    if args.gpus > 1 and ws == 0:
+        # not launched by torch.distributed.run: start one rank per GPU here
+        return _launch_ranks(args.gpus)
+    if ws and ws != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={ws}", file=sys.stderr)
+        return 2
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
+
+
+def _launch_ranks(n: int) -> int:
+    """Re-run this command under torch.distributed.run with n ranks on this
+    node (rendezvous on 127.0.0.1); rank 0 prints the line."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
 
 
 if __name__ == "__main__":

@@ -59,6 +59,7 @@ _SIGNATURES = {
     "fp8_static_scales_save": (_I32, [ctypes.c_char_p, _I32, ctypes.POINTER(ctypes.c_char_p),
                                       _P, _F32]),
     "fp8_descale_from_amax": (_F32, [_F32]),
+    "fp8_descale_from_amax_margin": (_F32, [_F32, _F32]),
 }
 
 _lib = None
@@ -362,6 +363,10 @@ def fp8_descale_from_amax(v: float) -> float:
     return float(lib().fp8_descale_from_amax(float(v)))
 
 
+def fp8_descale_from_amax_margin(amax: float, margin: float) -> float:
+    return float(lib().fp8_descale_from_amax_margin(float(amax), float(margin)))
+
+
 # ---- one attention layer ---------------------------------------------------------------
 
 class FP8EncoderAttention:
@@ -407,11 +412,10 @@ class FP8EncoderAttention:
         """Use static scales.  ``values`` are in the amax domain (already
         including the save margin, as stored in a scale file); pass ``margin``
         to apply one here instead."""
-        import numpy as np
-        v = np.asarray(values, dtype=np.float32)
-        if margin is not None:
-            v = (v * np.float32(margin)).astype(np.float32)
-        d = [fp8_descale_from_amax(float(x)) for x in v]
+        if margin is None:
+            d = [fp8_descale_from_amax(float(x)) for x in values]
+        else:
+            d = [fp8_descale_from_amax_margin(float(x), float(margin)) for x in values]
         self.descale.copy_(torch.tensor(d, dtype=torch.float32))
         self.ring = None
 

@@ -34,14 +34,15 @@
 #include <atomic>
 #include <type_traits>
 
-#include "fp8vit_internal.cuh"
+#include "attn_common.cuh"
 
 namespace {
+
+using namespace fp8vit_attn;
 
 constexpr int kBM = 128;          // query rows per CTA (MMA M)
 constexpr int kThreads = 192;     // 6 warps
 constexpr int kTmemCols = 256;
-constexpr int kBox = 32;          // bytes per TMA box row (one SW32 atom row)
 constexpr int kQTileBytes = kBox * kBM;   // one [128 rows x 32 B] Q box
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 // P is stored as 2^(x - m_ref + kPLog2); a tile max up to kSlackLog2 above the
@@ -114,30 +115,6 @@ using Smem = SmemOf<Cfg<D>>;
 template <int D, bool BF>
 using CfgOf = std::conditional_t<BF, CfgB<D>, Cfg<D>>;
 
-// Shared-memory matrix descriptors (tcgen05 "version 1" format), 32-byte
-// swizzle.  K-major: rows of 32 bytes, 8-row groups 256 bytes apart (SBO).
-// MN-major (V): 32-byte atoms along N, one [64 keys x 32 B] box apart (LBO);
-// 8-key groups 256 bytes apart (SBO).
-__device__ __forceinline__ uint64_t desc_k_sw32(uint32_t addr) {
-    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(256 >> 4) << 32) |
-           ((uint64_t)1 << 46) | ((uint64_t)6 << 61);
-}
-template <int KVT>
-__device__ __forceinline__ uint64_t desc_mn_sw32(uint32_t addr) {
-    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)(KVT >> 4) << 16) |
-           ((uint64_t)(256 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)6 << 61);
-}
-
-// Instruction descriptor, kind::f8f6f4: e4m3 x e4m3 -> f32, M = 128.
-__host__ __device__ constexpr uint32_t idesc_e4m3(int n, bool b_mn_major) {
-    return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(n >> 3) << 17) |
-           ((uint32_t)(128 >> 4) << 24);
-}
-// Instruction descriptor, kind::f16: bf16 x bf16 -> f32 (A and B format
-// fields = 1), M = 128.
-__host__ __device__ constexpr uint32_t idesc_bf16(int n, bool b_mn_major) {
-    return idesc_e4m3(n, b_mn_major) | (1u << 7) | (1u << 10);
-}
 
 // D[tmem] (+)= A * B, kind::f16 (both operands bf16), issued by one thread;
 // A from shared memory (descriptor) or from TMEM.
@@ -160,147 +137,7 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, u
         : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld8_sync(uint32_t taddr, uint32_t (&r)[8]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7])
-        : "r"(taddr)
-        : "memory");
-}
 
-// 64 consecutive columns of this thread's lane into a[0..31], b[0..31], then wait.
-__device__ __forceinline__ void tmem_ld64_sync(uint32_t taddr, uint32_t (&a)[32], uint32_t (&b)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]), "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15]), "=r"(a[16]), "=r"(a[17]), "=r"(a[18]), "=r"(a[19]), "=r"(a[20]), "=r"(a[21]), "=r"(a[22]), "=r"(a[23]), "=r"(a[24]), "=r"(a[25]), "=r"(a[26]), "=r"(a[27]), "=r"(a[28]), "=r"(a[29]), "=r"(a[30]), "=r"(a[31]), "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7]), "=r"(b[8]), "=r"(b[9]), "=r"(b[10]), "=r"(b[11]), "=r"(b[12]), "=r"(b[13]), "=r"(b[14]), "=r"(b[15]), "=r"(b[16]), "=r"(b[17]), "=r"(b[18]), "=r"(b[19]), "=r"(b[20]), "=r"(b[21]), "=r"(b[22]), "=r"(b[23]), "=r"(b[24]), "=r"(b[25]), "=r"(b[26]), "=r"(b[27]), "=r"(b[28]), "=r"(b[29]), "=r"(b[30]), "=r"(b[31])
-        : "r"(taddr)
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
-        "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(
-            taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
-        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
-        "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
-
-// O *= alpha over columns [0, NPV) of this thread's lane, in 32-column steps
-// (one load wait per step); NPV = 80 ends with two 8-column pieces.
-template <int NPV>
-__device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
-#pragma unroll
-    for (int c = 0; c + 32 <= NPV; c += 32) {
-        uint32_t r[32];
-        tmem_ld32(tO + c, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-        tmem_st32(tO + c, r);
-    }
-    if constexpr (NPV % 32 != 0) {
-        static_assert(NPV % 32 == 16, "O tail is one 16-column piece");
-        constexpr int c = NPV - 16;
-        uint32_t r[8], s[8];
-        tmem_ld8(tO + c, r);
-        tmem_ld8(tO + c + 8, s);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            s[i] = __float_as_uint(__uint_as_float(s[i]) * alpha);
-        }
-        tmem_st8(tO + c, r);
-        tmem_st8(tO + c + 8, s);
-    }
-}
-
-// One arrival per warp: every lane's prior memory and tcgen05 operations
-// (each lane has executed its own fences) are ordered before lane 0's arrive
-// by the warp barrier.
-__device__ __forceinline__ void warp_arrive(uint32_t bar, int lane) {
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar);
-}
-
-// ---- packed arithmetic used by the softmax --------------------------------
-
-__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-    float d;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
-// f32 pair -> f16x2 (lo in bits 0..15)
-__device__ __forceinline__ uint32_t cvt_f16x2(float lo, float hi) {
-    uint32_t d;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
-    return d;
-}
-// f16x2 -> two e4m3 codes in bits 0..15 (RNE, satfinite; bits 0..15 of the
-// source -> byte 0), returned zero-extended
-__device__ __forceinline__ uint32_t e4m3x2_of_f16x2(uint32_t h) {
-    uint16_t d;
-    asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(d) : "r"(h));
-    return d;
-}
-// two e4m3 codes (bits 0..15) -> f16x2 (exact)
-__device__ __forceinline__ uint32_t f16x2_of_e4m3x2(uint32_t e) {
-    uint32_t d;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"((uint16_t)e));
-    return d;
-}
-__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-
-// Row max of one S tile of NCH 32-key chunks held in registers; keys past the
-// segment end already hold -inf.
-template <int NCH>
-__device__ __forceinline__ float tile_row_max(const uint32_t (&r)[NCH][32]) {
-    float m[NCH];
-#pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-        float a = -INFINITY, b = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-            a = fmax3(a, __uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1]));
-            b = fmax3(b, __uint_as_float(r[c][i + 2]), __uint_as_float(r[c][i + 3]));
-        }
-        m[c] = fmaxf(a, b);
-    }
-    float mx = m[0];
-#pragma unroll
-    for (int c = 1; c < NCH; ++c) mx = fmaxf(mx, m[c]);
-    return mx;
-}
 
 // Probabilities of one 32-key chunk: p = 2^(s * c - bias) (a score of -inf
 // gives 0), summed into the two packed accumulators, then split into 8 hi and
@@ -425,28 +262,6 @@ __device__ __forceinline__ void tmem_st_p_any(uint32_t taddr, const uint32_t (&p
     else tmem_st_p<PLO>(taddr, pk);
 }
 
-// Eight O columns of this thread's lane times inv, rounded to bf16 (RNE) and
-// packed two per word: the values the bf16 epilogue stores.
-__device__ __forceinline__ uint4 bf16x8_of_o(uint32_t taddr, float inv) {
-    uint32_t r[8];
-    tmem_ld8_sync(taddr, r);
-    uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float(r[2 * i]) * inv,
-                                                 __uint_as_float(r[2 * i + 1]) * inv);
-        w[i] = *reinterpret_cast<uint32_t*>(&b);
-    }
-    return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
-// Output modes, one epilogue per kernel instance.
-enum : int {
-    kOutBf16 = 0,     // o as bf16
-    kOutE4m3 = 1,     // e4m3(o / output_scale)
-    kOutGroupQ = 2,   // the bf16 o of each head quantized as one 128-wide group:
-                      // e4m3 codes + one fp32 scale per (token, head); head_dim 128
-};
 
 // OUT selects the epilogue at compile time; PLO keeps P as two e4m3 terms
 // (hi + lo, two PV MMAs) or, when false, as one.  BF: the inputs are BF16
@@ -567,12 +382,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                 ++issued;
             }
             // Drain: every issued copy must land before the CTA may exit.
-            mbar_wait_bounded(b_q_full, 0, abort_flag, scr, SITE_ATTN_DRAIN, kTimeoutNs);
-            for (int j = issued - 1; j >= 0 && j >= issued - NS; --j) {
-                const int s = j % NS;
-                mbar_wait_bounded(b_kv_full(s), (j / NS) & 1, abort_flag, scr, SITE_ATTN_DRAIN,
-                                  kTimeoutNs);
-            }
+            mbar_wait_drain(b_q_full, 0, scr);
+            for (int j = issued - 1; j >= 0 && j >= issued - NS; --j)
+                mbar_wait_drain(b_kv_full(j % NS), (j / NS) & 1, scr);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
@@ -650,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             // Never leave MMAs in flight: one more commit tracks all of them.
             if (issued_any) {
                 umma_commit(b_drain);
-                mbar_wait_bounded(b_drain, 0, abort_flag, scr, SITE_ATTN_DRAIN, kTimeoutNs);
+                mbar_wait_drain(b_drain, 0, scr);
             }
         }
     } else {
@@ -863,19 +675,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 }
 
-bool encode_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_bytes,
-                int box_rows) {
-    fp8vit_encode_tiled_fn enc = fp8vit_get_encode_tiled();
-    if (!enc) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-    const cuuint32_t box[2] = {(cuuint32_t)kBox, (cuuint32_t)box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 template <int D, int OUT>
 fp8vit_status launch(fp8vit_ctx* ctx, const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
@@ -939,9 +738,6 @@ fp8vit_status launch_bf16(fp8vit_ctx* ctx, const uint16_t* q, const uint16_t* k,
     return cudaGetLastError() == cudaSuccess ? FP8VIT_OK : FP8VIT_ECUDA;
 }
 
-inline bool misaligned(const void* p, uintptr_t a) {
-    return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0;
-}
 
 }  // namespace
 

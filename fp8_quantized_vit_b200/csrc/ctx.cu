@@ -135,6 +135,11 @@ float fp8_descale_from_amax(float v) {
     return d > 1e-10f ? d : 1e-10f;
 }
 
+float fp8_descale_from_amax_margin(float amax, float margin) {
+    volatile float prod = margin * amax;  // the fp32 product fp8_static_scales_save writes
+    return fp8_descale_from_amax(prod);
+}
+
 }  // extern "C"
 
 fp8vit_encode_tiled_fn fp8vit_get_encode_tiled() {

@@ -189,8 +189,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Bounded wait on phase `parity` of an mbarrier.  Gives up when *abort is set
-// by another thread of the CTA or after timeout_ns; on a timeout it sets
-// *abort and records FP8VIT_ETIMEOUT with `site`.  Returns false on give-up.
+// by another thread of the CTA (abort may be null: then only the time limit
+// ends the wait) or after timeout_ns; on a timeout it sets *abort and records
+// FP8VIT_ETIMEOUT with `site`.  Returns false on give-up.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   volatile int32_t* abort, fp8vit_scratch* scr,
                                                   int32_t site, uint64_t timeout_ns) {
@@ -199,9 +200,9 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 63u) == 0) {
-            if (*abort) return false;
+            if (abort && *abort) return false;
             if (globaltimer_ns() - t0 > timeout_ns) {
-                *abort = 1;
+                if (abort) *abort = 1;
                 fp8vit_report(scr, FP8VIT_ETIMEOUT, site);
                 return false;
             }

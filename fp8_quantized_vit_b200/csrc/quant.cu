@@ -621,9 +621,9 @@ fp8vit_status per_token_group_quant_fp8(fp8vit_ctx* ctx, const uint16_t* d_x, in
 // Scratch: sizeof(fp8vit_scratch) = 128 bytes (three running |x| maxima, an
 // arrival counter, status words), taken from a 256-byte array.  The amount
 // does not grow with n_elems, so any size the context entry point accepts is
-// accepted here; a scratch need above the array's capacity is rejected with
-// FP8VIT_EUNSUPPORTED.  Every GPU that loads the library holds the array
-// until the process exits.
+// accepted here; that the need fits the array is checked when the library is
+// compiled.  Every GPU that loads the library holds the array until the
+// process exits.
 // ---------------------------------------------------------------------------
 namespace {
 
@@ -633,6 +633,8 @@ constexpr int kNoAllocMaxDevices = 64;
 }  // namespace
 
 static __device__ __align__(256) unsigned char g_amax_noalloc_scratch[kNoAllocScratchBytes];
+static_assert(sizeof(fp8vit_scratch) <= kNoAllocScratchBytes,
+              "the amax scratch must fit the library's fixed array");
 
 namespace {
 
@@ -679,7 +681,6 @@ extern "C" fp8vit_status fp8_amax_ring_update_noalloc(const uint16_t* d_q, const
     if (misaligned(d_q, 16) || misaligned(d_k, 16) || misaligned(d_v, 16) ||
         misaligned(d_ring, 16) || misaligned(d_descale3, 4))
         return FP8VIT_EINVAL;
-    if (sizeof(fp8vit_scratch) > kNoAllocScratchBytes) return FP8VIT_EUNSUPPORTED;
     void* scratch = nullptr;
     int num_sms = 0;
     fp8vit_status st = noalloc_scratch(&scratch, &num_sms);

@@ -93,8 +93,9 @@ fp8vit_status fp8vit_inject_lost_arrival(fp8vit_ctx* ctx, void* stream);
  * the kernel then stops its other roles, drains its copies and MMAs, frees
  * TMEM and returns.  The injection stays set until fp8vit_check returns the
  * fault it causes: FP8VIT_ETIMEOUT (site 113, the softmax wait for the
- * scores, or 119, the issuer's wait for their buffer to be released,
- * whichever gives up first); that check clears it together with the status
+ * scores, or the issuer's wait that starves with it: 114, the FP8 kernel's
+ * wait for the first tile's P, 119, the BF16 kernel's wait for the score
+ * buffer to be released; whichever gives up first); that check clears it together with the status
  * word.  A check with no attention launch in between leaves it set.  No GPU
  * fault is involved.  Synchronizes `stream`.  Not for production use. */
 fp8vit_status fp8vit_inject_attn_timeout(fp8vit_ctx* ctx, void* stream);
@@ -162,11 +163,16 @@ fp8vit_status fp8_ring_push(const float* d_amax3, void* d_ring, float* d_descale
  *   - Takes no context and allocates nothing: its 128 bytes of scratch come
  *     from a 256-byte array built into the library's device image, which
  *     every GPU that loads the library keeps until the process exits.  The
- *     scratch need does not grow with n_elems; a need above the array's
- *     capacity would be refused with FP8VIT_EUNSUPPORTED.
+ *     scratch need does not grow with n_elems; that it fits the array is
+ *     checked when the library is compiled.
  *   - The first call on a device looks up the array's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture on the device.
+ *     that device current) and caches it for the life of the process; make
+ *     that first call before any stream capture on the device.  The cached
+ *     address must not outlive the device's primary context: after
+ *     cudaDeviceReset on a device, do not call this entry point on it again
+ *     in the same process.
+ *   - Devices numbered 64 or above are refused with FP8VIT_EUNSUPPORTED (the
+ *     per-device address cache has 64 slots).
  *   - Every call on a device shares the one array: each call clears it with
  *     a 128-byte memset on `stream` before its kernel.  Calls whose work
  *     overlaps on the GPU (different streams, no ordering) race on it and
@@ -313,6 +319,13 @@ fp8vit_status fp8_static_scales_save(const char* path, int32_t n_layers,
 
 /* max(v / 448, 1e-10) in fp32: the descale for a value v of the amax domain. */
 float fp8_descale_from_amax(float v);
+
+/* The descale of an observed amax with the save margin applied here
+ * (vLLM "FP8 ViT Encoder Attention": the margin multiplies the calibrated
+ * amax when the scales are saved): fp8_descale_from_amax(fp32(margin *
+ * amax)), the same fp32 product fp8_static_scales_save writes, so that
+ * scales taken this way equal those of a saved and reloaded file. */
+float fp8_descale_from_amax_margin(float amax, float margin);
 
 #ifdef __cplusplus
 }

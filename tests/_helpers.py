@@ -45,9 +45,11 @@ def assert_attn_close(got, ref, what=""):
     return e
 
 
-def sample_pairs(cu: np.ndarray, heads: int, per_seg: int, seed: int):
-    """(token, head) pairs per segment: first/last rows, rows around the
-    128-row tile edges, and random rows; heads cycle so all are covered."""
+def sample_pairs(cu: np.ndarray, heads: int, per_seg: int, seed: int, tile: int = 128):
+    """(token, head) pairs per segment: its first, middle and last rows, both
+    rows on every `tile`-row query-tile edge, and seeded random rows up to
+    per_seg; the heads cycle through all of them (each segment starts at a
+    different head), so every head and every tile edge is covered."""
     rng = np.random.default_rng(seed)
     toks, hs = [], []
     for i in range(len(cu) - 1):
@@ -55,12 +57,46 @@ def sample_pairs(cu: np.ndarray, heads: int, per_seg: int, seed: int):
         L = b - a
         if L <= 0:
             continue
-        fixed = {0, L - 1, min(127, L - 1), min(128, L - 1), L // 2, max(0, L - 129)}
-        rows = sorted(fixed) + list(rng.integers(0, L, size=max(0, per_seg - len(fixed))))
+        fixed = {0, L - 1, L // 2, max(0, L - 129)}
+        for k in range(1, (L - 1) // tile + 1):
+            fixed |= {k * tile - 1, k * tile}
+        fixed = sorted(r for r in fixed if r < L)
+        rows = fixed + [int(r) for r in rng.integers(0, L, size=max(0, per_seg - len(fixed)))]
         for n, r in enumerate(rows):
             toks.append(a + int(r))
-            hs.append(int((n + i) % heads) if n < heads else int(rng.integers(0, heads)))
+            hs.append(int((n + i) % heads))
     return np.array(toks, dtype=np.int64), np.array(hs, dtype=np.int32)
+
+
+def complete_tile_pairs(cu: np.ndarray, heads: int, seed: int, tile: int = 128):
+    """Every (token, head) pair of one full `tile`-row query tile per segment
+    (a seeded choice among the segment's full tiles)."""
+    rng = np.random.default_rng(seed)
+    toks, hs = [], []
+    for i in range(len(cu) - 1):
+        a, L = int(cu[i]), int(cu[i + 1] - cu[i])
+        if L < tile:
+            continue
+        t0 = int(rng.integers(0, L // tile)) * tile
+        rows = np.arange(a + t0, a + t0 + tile, dtype=np.int64)
+        toks.append(np.repeat(rows, heads))
+        hs.append(np.tile(np.arange(heads, dtype=np.int32), tile))
+    return np.concatenate(toks), np.concatenate(hs)
+
+
+def oracle_pairs_threaded(fn, args, toks, hs, threads: int = 0):
+    """Runs the oracle's per-pair attention (fn(*args, toks, hs)) over chunks
+    of the pairs on several host threads (the C call releases the GIL) and
+    concatenates the rows in order."""
+    import concurrent.futures as cf
+    import os
+    n = len(toks)
+    threads = threads or max(1, min(32, len(os.sched_getaffinity(0))))
+    bounds = np.linspace(0, n, threads + 1).astype(int)
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        parts = list(ex.map(lambda k: fn(*args, toks[bounds[k]:bounds[k + 1]],
+                                         hs[bounds[k]:bounds[k + 1]]), range(threads)))
+    return np.concatenate(parts, axis=0)
 
 
 def e4m3_half_step(y: np.ndarray) -> np.ndarray:

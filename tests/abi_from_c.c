@@ -26,6 +26,7 @@ int main(int argc, char** argv) {
     CHECK(2, strcmp(fp8vit_status_string(FP8VIT_OK), "ok") == 0);
     CHECK(3, fp8_descale_from_amax(224.0f) == 0.5f);
     CHECK(4, fp8_descale_from_amax(0.0f) == 1e-10f);
+    CHECK(41, fp8_descale_from_amax_margin(224.0f, 1.5f) == 0.75f);
 
     float v[3] = {0, 0, 0};
     CHECK(5, fp8_static_scales_load(golden, "visual.blocks.0.attn.attn", v) == FP8VIT_OK);

@@ -118,6 +118,22 @@ def test_scale_file_round_trip_with_margin(tmp_path):
         assert got == want
 
 
+def test_descale_with_margin_equals_a_saved_and_reloaded_file(tmp_path):
+    """The margin applied in C (fp8_descale_from_amax_margin) gives the same
+    descales as saving the amax with that margin and loading the file back."""
+    rng = np.random.default_rng(2)
+    amax = (rng.random((4, 3)) * 60).astype(np.float32)
+    amax[0, 0] = 0.0
+    layers = [f"l{i}" for i in range(4)]
+    p = str(tmp_path / "m.json")
+    for margin in (1.5, 1.25, 2.0):
+        fv.fp8_static_scales_save(p, layers, amax, margin=margin)
+        for i, name in enumerate(layers):
+            via_file = [fv.fp8_descale_from_amax(x) for x in fv.fp8_static_scales_load(p, name)]
+            direct = [fv.fp8_descale_from_amax_margin(float(a), margin) for a in amax[i]]
+            assert direct == via_file, (margin, i)
+
+
 def test_attn_p_terms_setting_is_checked_on_the_host():
     lib = fv.lib()
     fake_ctx = ctypes.create_string_buffer(64)  # host-only call: the struct is never on the GPU

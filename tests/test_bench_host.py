@@ -279,3 +279,23 @@ def test_output_modes_leg_calls_the_binding_as_declared(monkeypatch):
         assert all(r["ms"] == 0.5 and r["tflops"] > 0 for r in res.values())
         assert seen[:2] == ["fp8_amax3", "fp8_quantize_qkv_per_tensor"]
         assert ("fp8_varlen_attn_fwd_group_quant" in seen) == (D == 128)
+
+
+def test_gpus_flag_launches_one_rank_per_gpu(monkeypatch):
+    """`bench.py --gpus N` started without torch.distributed.run re-runs
+    itself under it with N ranks on 127.0.0.1 (it never times one GPU and
+    reports N); under a launcher whose WORLD_SIZE disagrees with --gpus it
+    exits non-zero."""
+    import sys as _sys
+    calls = []
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.setattr(bench.subprocess, "call", lambda cmd: calls.append(cmd) or 0)
+    monkeypatch.setattr(_sys, "argv", ["bench.py", "--gpus", "4", "--steps", "3"])
+    assert bench.main() == 0
+    cmd = calls[0]
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "127.0.0.1" in cmd
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "3"]
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setattr(_sys, "argv", ["bench.py", "--gpus", "4"])
+    assert bench.main() == 2

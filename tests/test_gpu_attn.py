@@ -19,7 +19,8 @@ import torch
 import oracle
 import synth
 from _helpers import (ATTN_COS, ATTN_MEAN_ABS, assert_attn_close, assert_fp8_out_close,
-                      attn_errors, bf16_bits_to_f64, code_step_distance, sample_pairs)
+                      attn_errors, bf16_bits_to_f64, code_step_distance, complete_tile_pairs,
+                      oracle_pairs_threaded, sample_pairs)
 
 pytestmark = pytest.mark.gpu
 
@@ -108,11 +109,11 @@ def test_1024_tokens_full_oracle(ctx):
     print("1024 tokens errors", e)
 
 
-@pytest.mark.parametrize("name", ["1x8192_d128", "1x2304_d72", "1x4096_d72", "1x8192_d72", "1x16384_d72",
-                                  "3x14400_d72", "3x32400_d72"])
-def test_workload_sampled_rows(ctx, name):
-    w = synth.WORKLOADS[name]
-    q, k, v = w.qkv(0)
+def _workload_codes(w, slot=0):
+    """The oracle's e4m3 codes and descales of forward/layer `slot` of a
+    workload (static: 1.5 x the exact amax; dynamic: a fresh ring's first
+    update, i.e. the layer's own ring)."""
+    q, k, v = w.qkv(slot)
     amax = [oracle.amax_bf16(x) for x in (q, k, v)]
     if w.mode == "static":
         desc = [oracle.descale_from_amax(np.float32(1.5) * np.float32(a)) for a in amax]
@@ -120,15 +121,82 @@ def test_workload_sampled_rows(ctx, name):
         desc = list(oracle.Ring().update(amax))
     codes = [oracle.quantize_per_tensor(x, d).reshape(w.tokens, w.heads, w.head_dim)
              for x, d in zip((q, k, v), desc)]
+    return (q, k, v), codes, desc
+
+
+def _oracle_rows(w, codes, desc, cu, toks, hs):
+    return oracle_pairs_threaded(oracle.attn_pairs, (*codes, *desc, cu, w.heads, w.head_dim,
+                                                     w.softmax_scale), toks, hs)
+
+
+@pytest.mark.parametrize("name", ["1x8192_d128", "1x2304_d72", "1x4096_d72", "1x8192_d72", "1x16384_d72",
+                                  "3x14400_d72", "3x32400_d72"])
+def test_workload_sampled_rows(ctx, name):
+    """At least 256 (token, head) rows per image: every 128-row query-tile
+    edge (both sides), first, middle and last rows, seeded random rows, all
+    heads."""
+    w = synth.WORKLOADS[name]
+    _, codes, desc = _workload_codes(w)
     cu = synth.cu_seqlens(w.seg_lens)
-    toks, hs = sample_pairs(cu, w.heads, per_seg=24, seed=len(name))
-    ref = oracle.attn_pairs(*codes, *desc, cu, w.heads, w.head_dim, w.softmax_scale, toks, hs)
+    toks, hs = sample_pairs(cu, w.heads, per_seg=256, seed=len(name))
+    ref = _oracle_rows(w, codes, desc, cu, toks, hs)
     out = _run_gpu(ctx, cu, codes, desc, w.heads, w.head_dim, max(w.seg_lens))
     got = _gpu_bf16_to_f64(out)[toks, hs]
     e = assert_attn_close(got, ref, name)
-    print(name, "errors", e)
+    print(name, len(toks), "rows, errors", e)
     # every row was written (no NaN left from the fill)
     assert not torch.isnan(out.float()).any().item()
+
+
+@pytest.mark.parametrize("name", ["1x8192_d128", "3x32400_d72"])
+def test_workload_complete_query_tile(ctx, name):
+    """One complete 128-row query tile per image (every row, every head)."""
+    w = synth.WORKLOADS[name]
+    _, codes, desc = _workload_codes(w)
+    cu = synth.cu_seqlens(w.seg_lens)
+    toks, hs = complete_tile_pairs(cu, w.heads, seed=7)
+    ref = _oracle_rows(w, codes, desc, cu, toks, hs)
+    out = _run_gpu(ctx, cu, codes, desc, w.heads, w.head_dim, max(w.seg_lens))
+    e = assert_attn_close(_gpu_bf16_to_f64(out)[toks, hs], ref, name)
+    print(name, len(toks), "rows of complete tiles, errors", e)
+
+
+@pytest.mark.parametrize("layer", [0, 13, 26])
+def test_27_layer_workload_layers_with_own_rings(ctx, layer):
+    """Layers 0, 13 and 26 of the 3x32400-token, 27-layer workload, each
+    with its own amax ring: the device ring update and quantizer give the
+    oracle's descales and codes bit for bit, the attention meets the gate on
+    sampled rows, and the group-128 quantizer of the kernel's BF16 output
+    equals the oracle's group quantizer of that output byte for byte."""
+    w = synth.WORKLOADS["3x32400_d72"]
+    T, H, D = w.tokens, w.heads, w.head_dim
+    bf, codes, desc = _workload_codes(w, layer)
+    dev = [_dev(x.view(np.int16), torch.bfloat16).reshape(T, H, D) for x in bf]
+    ring = fv.new_ring()
+    d = torch.zeros(3, dtype=torch.float32, device="cuda")
+    q8, k8, v8 = (torch.empty((T, H, D), dtype=torch.uint8, device="cuda") for _ in range(3))
+    fv.fp8_amax_ring_quantize_qkv(*dev, ring, d, q8, k8, v8, ctx=ctx)
+    assert (d.cpu().numpy().view(np.uint32) ==
+            np.asarray(desc, np.float32).view(np.uint32)).all()
+    for got, want in zip((q8, k8, v8), codes):
+        assert np.array_equal(got.cpu().numpy(), want)
+    cu = synth.cu_seqlens(w.seg_lens)
+    out = torch.empty((T, H, D), dtype=torch.bfloat16, device="cuda")
+    fv.fp8_varlen_attn_fwd(q8, k8, v8, d[0:1], d[1:2], d[2:3], _dev(cu), max(w.seg_lens),
+                           w.softmax_scale, out, ctx=ctx)
+    xq = torch.empty((T, H * D), dtype=torch.uint8, device="cuda")
+    xs = torch.empty((T, H * D // 128), dtype=torch.float32, device="cuda")
+    fv.per_token_group_quant_fp8(out.view(T, H * D), 128, xq, xs, ctx=ctx)
+    st, site = ctx.check()
+    assert st == fv.OK, (fv.status_string(st), site)
+    toks, hs = sample_pairs(cu, H, per_seg=256, seed=100 + layer)
+    ref = _oracle_rows(w, codes, desc, cu, toks, hs)
+    e = assert_attn_close(_gpu_bf16_to_f64(out)[toks, hs], ref, f"layer {layer}")
+    print("layer", layer, "errors", e)
+    bits = out.view(torch.int16).cpu().numpy().view(np.uint16).reshape(T, H * D)
+    gq, gs = oracle.group_quant(bits, 128)
+    assert np.array_equal(xq.cpu().numpy(), gq)
+    assert np.array_equal(xs.cpu().numpy().view(np.uint32), gs.view(np.uint32))
 
 
 def test_fp8_output_small_full(ctx):
@@ -397,9 +465,10 @@ def test_attention_timeout_is_reported_and_recovered():
     fv.fp8_varlen_attn_fwd(q8, k8, v8, d[0], d[1], d[2], _dev(cu), max(lens),
                            np.float32(1.0 / math.sqrt(D)), out, ctx=c)
     st, site = c.check()
-    # the softmax warps wait for S(0) (site 113) while the issuer waits for
-    # the S buffer to be released (site 119): the first to give up records it
-    assert st == fv.ETIMEOUT and site in (113, 119), (fv.status_string(st), site)
+    # the softmax warps of the first query tile wait for S(0) (site 113)
+    # while the issuer waits for that tile's P (114) or for the score buffer
+    # to be released (119): the first to give up records it
+    assert st == fv.ETIMEOUT and site in (113, 114, 119), (fv.status_string(st), site)
     assert c.check() == (fv.OK, 0)
     got = _gpu_bf16_to_f64(_run_gpu(c, cu, codes, desc, H, D, max(lens)))
     ref = oracle.attn_full(*codes, *desc, cu, H, D, np.float32(1.0 / math.sqrt(D)))
