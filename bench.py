@@ -179,9 +179,15 @@ def _oracle_rows_time(w, codes, desc, rows_budget_s: float, seed: int):
 
 
 def _oracle_inputs(w):
+    """The oracle's e4m3 codes and descales of forward 0: static scales from
+    the margin x the exact amax, or a fresh ring's first update."""
     import oracle
     q, k, v = w.qkv(0)
-    desc = list(oracle.Ring().update([oracle.amax_bf16(x) for x in (q, k, v)]))
+    amax = [oracle.amax_bf16(x) for x in (q, k, v)]
+    if w.mode == "static":
+        desc = [oracle.descale_from_amax(np.float32(w.margin) * np.float32(a)) for a in amax]
+    else:
+        desc = list(oracle.Ring().update(amax))
     codes = [oracle.quantize_per_tensor(x, d).reshape(w.tokens, w.heads, w.head_dim)
              for x, d in zip((q, k, v), desc)]
     return codes, desc
@@ -257,14 +263,19 @@ def _parity_field(w, codes, desc, fwd0) -> dict:
         return {"error": repr(exc)}
 
 
-def _forward0_outputs(fv, ctx, w, qkv0, cu_d, max_s, q8, k8, v8, out, dev):
-    """Runs forward 0 again from a fresh ring (after the timed region) and
-    returns what the kernels produced: descales, e4m3 codes, BF16 output bits
-    (host arrays; compared with the oracle by the CPU-baseline leg)."""
+def _forward0_outputs(fv, ctx, w, qkv0, cu_d, max_s, q8, k8, v8, out, dev, static_desc=None):
+    """Runs forward 0 again (after the timed region; dynamic workloads from a
+    fresh ring, static ones with their calibrated descales) and returns what
+    the kernels produced: descales, e4m3 codes, BF16 output bits (host arrays;
+    compared with the oracle by the CPU-baseline leg)."""
     import torch
-    ring0 = fv.new_ring(dev)
-    desc0 = torch.zeros(3, dtype=torch.float32, device=dev)
-    fv.fp8_amax_ring_quantize_qkv(*qkv0, ring0, desc0, q8, k8, v8, ctx=ctx)
+    if static_desc is not None:
+        desc0 = static_desc
+        fv.fp8_quantize_qkv_per_tensor(*qkv0, desc0, q8, k8, v8, ctx=ctx)
+    else:
+        ring0 = fv.new_ring(dev)
+        desc0 = torch.zeros(3, dtype=torch.float32, device=dev)
+        fv.fp8_amax_ring_quantize_qkv(*qkv0, ring0, desc0, q8, k8, v8, ctx=ctx)
     fv.fp8_varlen_attn_fwd(q8, k8, v8, desc0[0:1], desc0[1:2], desc0[2:3], cu_d, max_s,
                            w.softmax_scale, out, ctx=ctx)
     st, site = ctx.check()
@@ -594,16 +605,172 @@ def _quant_rooflines(fv, ctx, src, dev, hbm_gbs, reps=10):
             "bound": "hbm", "kernels": out}
 
 
+def _step_description(w) -> str:
+    """What one timed step of workload w runs (the configuration's own path)."""
+    if w.mode == "static":
+        quant = "per-tensor quantize q/k/v with static scales (1.5 x the calibrated amax)"
+    else:
+        quant = "amax ring update + per-tensor quantize q/k/v (one launch)"
+    out = ("attention (fp8 out, output_scale = amax(bf16 out)/448 from a calibration pass on "
+           "the device)" if w.fp8_out else "attention (bf16 out)")
+    tail = " + group quant (128)" if w.group_quant else ""
+    return f"{quant} + {out}{tail}"
+
+
+def _launches_per_step(w, l2_bytes: int) -> int:
+    """Kernels one step launches: the quantizer (the dynamic entry point takes
+    two kernels once the BF16 inputs exceed twice the L2), attention, and the
+    group quantizer where the workload has it."""
+    quant = 1
+    if w.mode != "static" and 3 * w.tokens * w.hd * 2 > 2 * l2_bytes:
+        quant = 2
+    return quant + 1 + (1 if w.group_quant else 0)
+
+
 def _config(w, n_fwd=None):
     n_fwd = len(w.seeds) if n_fwd is None else n_fwd
     gb = n_fwd * 3 * w.tokens * w.hd * 2 / 1e9
     return {"workload": w.name, "seq_lens": list(w.seg_lens), "heads": w.heads,
             "head_dim": w.head_dim, "forwards": n_fwd,
-            "step": "amax ring + quantize q/k/v (one launch) + attention (bf16 out) + group quant (128)",
+            "step": _step_description(w),
             "l2": f"inputs rotate over {n_fwd} forwards ({gb:.2f} GB; L2 is 126 MB)",
             "rings": (f"one amax ring per layer ({n_fwd} layers)" if w.per_layer_rings
-                      else "one amax ring over the rotation"),
+                      else ("no ring (static scales)" if w.mode == "static"
+                            else "one amax ring over the rotation")),
             "parallelism": "replicas"}
+
+
+class _Path:
+    """One workload's own step on the device: the scale state (static
+    descales, or dynamic rings) and the buffers, built once; step(i) runs
+    forward i on the current stream through the library's entry points."""
+
+    def __init__(self, fv, ctx, w, inputs, dev):
+        import torch
+        import synth
+        self.fv, self.ctx, self.w = fv, ctx, w
+        T, H, D = w.tokens, w.heads, w.head_dim
+        self.inputs = inputs
+        self.cu = torch.from_numpy(synth.cu_seqlens(w.seg_lens)).to(dev)
+        self.max_s = max(w.seg_lens)
+        self.q8, self.k8, self.v8 = (torch.empty((T, H, D), dtype=torch.uint8, device=dev)
+                                     for _ in range(3))
+        self.out = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+        self.out8 = torch.empty((T, H, D), dtype=torch.uint8, device=dev) if w.fp8_out else None
+        self.xq = torch.empty((T, H * D), dtype=torch.uint8, device=dev)
+        self.xs = torch.empty((T, H * D // 128), dtype=torch.float32, device=dev)
+        self.desc = torch.zeros(3, dtype=torch.float32, device=dev)
+        self.oscale = None
+        if w.mode == "static":
+            # calibration (untimed): exact amax of forward 0 on the device,
+            # saved with the margin; the static descales then stay fixed
+            amax3 = torch.zeros(3, dtype=torch.float32, device=dev)
+            fv.fp8_amax3(*inputs[0], amax3, ctx=ctx)
+            self.desc.copy_(torch.tensor([fv.fp8_descale_from_amax_margin(float(a), w.margin)
+                                          for a in amax3.cpu().numpy()], dtype=torch.float32))
+            self.rings = []
+        else:
+            self.rings = [fv.new_ring(dev) for _ in range(len(inputs) if w.per_layer_rings
+                                                             else 1)]
+        if w.fp8_out:
+            # output_scale = amax(bf16 output of forward 0) / 448, formed on the
+            # device: the amax kernel on the output, then the ring rule of a
+            # fresh ring (max over one entry / 448, floored at 1e-10)
+            self._quantize(0)
+            self._attend(self.out, None)
+            amax3 = torch.zeros(3, dtype=torch.float32, device=dev)
+            fv.fp8_amax3(self.out, self.out, self.out, amax3, ctx=ctx)
+            os3 = torch.zeros(3, dtype=torch.float32, device=dev)
+            fv.fp8_ring_push(amax3, fv.new_ring(dev), os3)
+            self.oscale = os3[0:1].clone()
+            for r in self.rings:
+                fv.ring_init(r)
+
+    def _quantize(self, i):
+        fv, q, k, v = self.fv, *self.inputs[i % len(self.inputs)]
+        if self.w.mode == "static":
+            fv.fp8_quantize_qkv_per_tensor(q, k, v, self.desc, self.q8, self.k8, self.v8,
+                                           ctx=self.ctx)
+        else:
+            fv.fp8_amax_ring_quantize_qkv(q, k, v, self.rings[i % len(self.rings)], self.desc,
+                                          self.q8, self.k8, self.v8, ctx=self.ctx)
+
+    def _attend(self, out, oscale):
+        d = self.desc
+        self.fv.fp8_varlen_attn_fwd(self.q8, self.k8, self.v8, d[0:1], d[1:2], d[2:3], self.cu,
+                                    self.max_s, self.w.softmax_scale, out, output_scale=oscale,
+                                    ctx=self.ctx)
+
+    def step(self, i, ev_a=None, ev_b=None, stream=None):
+        w = self.w
+        self._quantize(i)
+        if ev_a is not None:
+            ev_a.record(stream)
+        if w.fp8_out:
+            self._attend(self.out8, self.oscale)
+        else:
+            self._attend(self.out, None)
+        if ev_b is not None:
+            ev_b.record(stream)
+        if w.group_quant:
+            T, HD = w.tokens, w.heads * w.head_dim
+            self.fv.per_token_group_quant_fp8(self.out.view(T, HD), 128, self.xq, self.xs,
+                                              ctx=self.ctx)
+
+
+def _time_path(path, steps, warmup, stream):
+    """(ms per step, attention ms per launch) of a workload's own step, CUDA
+    events on the launching stream."""
+    import torch
+    for i in range(warmup):
+        path.step(i)
+    torch.cuda.synchronize()
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        path.step(i, ev_a[i], ev_b[i], stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    attn = statistics.mean(a.elapsed_time(b) for a, b in zip(ev_a, ev_b))
+    return t0.elapsed_time(t1) / steps, attn
+
+
+def _config_records(fv, ctx, dev, peaks, stream, steps=5, warmup=3):
+    """Every target workload's own step, timed in the same run as the headline
+    (attention TFLOP/s and its fraction of the FP8 denominator, step time), with
+    torch's BF16 SDPA on the same inputs beside the single-image workloads."""
+    import torch
+    import synth
+    fp8_peak = 2.0 * peaks["bf16"]
+    recs = {}
+    for name in ("1x1024_d72", "1x2304_d72", "1x4096_d72", "1x8192_d72", "1x16384_d72",
+                 "3x14400_d72", "3x32400_d72"):
+        w = synth.WORKLOADS[name]
+        T, H, D = w.tokens, w.heads, w.head_dim
+        n_in = len(w.seeds) if w.per_layer_rings else min(2, len(w.seeds))
+        inputs = [[torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).reshape(T, H, D)
+                   .to(dev) for x in w.qkv(f)] for f in range(n_in)]
+        path = _Path(fv, ctx, w, inputs, dev)
+        n_steps = n_in if w.per_layer_rings else steps  # one pass over all 27 layers
+        ms, attn_ms = _time_path(path, n_steps, min(warmup, n_steps), stream)
+        st, site = ctx.check()
+        if st != fv.OK:
+            raise RuntimeError(f"device fault in {name}: {fv.status_string(st)} site {site}")
+        tf = w.attn_flops() / (attn_ms * 1e-3) / 1e12
+        rec = {"workload": w.name, "step": _step_description(w), "ms_per_step": ms,
+               "steps_timed": n_steps, "attn_ms": attn_ms, "attn_tflops": tf,
+               "attn_frac_of_fp8_peak": tf / fp8_peak,
+               "step_tflops": w.attn_flops() / (ms * 1e-3) / 1e12}
+        if len(w.seg_lens) == 1:
+            rec["torch_bf16_sdpa"] = _sdpa_comparator(w, inputs, dev)
+        recs[name] = rec
+        del path, inputs
+        torch.cuda.empty_cache()
+    return {"fp8_peak_tflops": fp8_peak, "peak_source": f"{peaks['source']} bf16 burst x 2",
+            "records": recs}
 
 
 def run_ours(args):
@@ -632,30 +799,22 @@ def run_ours(args):
         qkv = w.qkv(f)
         inputs.append([torch.from_numpy(x.view(np.int16)).view(torch.bfloat16)
                        .reshape(T, H, D).to(dev) for x in qkv])
-    cu = torch.from_numpy(synth.cu_seqlens(w.seg_lens)).to(dev)
-    max_s = max(w.seg_lens)
-    # one ring for a rotation of forwards; one per layer when the seeds are the
-    # layers of one encoder forward (each layer keeps its own amax history)
-    rings = [fv.new_ring(dev) for _ in range(n_fwd if w.per_layer_rings else 1)]
-    desc = torch.zeros(3, dtype=torch.float32, device=dev)
-    q8, k8, v8 = (torch.empty((T, H, D), dtype=torch.uint8, device=dev) for _ in range(3))
-    out = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
-    xq = torch.empty((T, H * D), dtype=torch.uint8, device=dev)
-    xs = torch.empty((T, H * D // 128), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    # the workload's own step: static or dynamic scales (one ring per layer
+    # when the seeds are the layers of one encoder forward), BF16 or FP8
+    # output, group quantization of the output where the workload has it
+    path = _Path(fv, ctx, w, inputs, dev)
+    cu, max_s = path.cu, path.max_s
+    q8, k8, v8, out, xq, xs = path.q8, path.k8, path.v8, path.out, path.xq, path.xs
+    rings = path.rings
     ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
 
     def step(i, timed=False):
-        q, k, v = inputs[i % n_fwd]
-        fv.fp8_amax_ring_quantize_qkv(q, k, v, rings[i % len(rings)], desc, q8, k8, v8, ctx=ctx)
         if timed:
-            ev_a[i].record(stream)
-        fv.fp8_varlen_attn_fwd(q8, k8, v8, desc[0:1], desc[1:2], desc[2:3], cu, max_s,
-                               w.softmax_scale, out, ctx=ctx)
-        if timed:
-            ev_b[i].record(stream)
-        fv.per_token_group_quant_fp8(out.view(T, H * D), 128, xq, xs, ctx=ctx)
+            path.step(i, ev_a[i], ev_b[i], stream)
+        else:
+            path.step(i)
 
     for i in range(args.warmup):
         step(i)
@@ -704,12 +863,18 @@ def run_ours(args):
     # buffers are double-buffered and events order every reuse.
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     host_in = [[t.cpu().pin_memory() for t in inputs[f]] for f in range(min(n_fwd, e2e_steps))]
-    host_xq = [torch.empty(xq.shape, dtype=xq.dtype).pin_memory() for _ in range(2)]
-    host_xs = [torch.empty(xs.shape, dtype=xs.dtype).pin_memory() for _ in range(2)]
     dbuf = [[torch.empty((T, H, D), dtype=torch.bfloat16, device=dev) for _ in range(3)]
             for _ in range(2)]
-    dxq = [xq, torch.empty_like(xq)]
-    dxs = [xs, torch.empty_like(xs)]
+    # the step's result, double-buffered on the device and in pinned host
+    # memory: the group-quantized output (codes + scales), else the FP8 or
+    # BF16 attention output
+    if w.group_quant:
+        dres = [[xq, xs], [torch.empty_like(xq), torch.empty_like(xs)]]
+    elif w.fp8_out:
+        dres = [[path.out8], [torch.empty_like(path.out8)]]
+    else:
+        dres = [[out], [torch.empty_like(out)]]
+    hres = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in dres[0]] for _ in range(2)]
     up = torch.cuda.Stream(dev)
     down = torch.cuda.Stream(dev)
     ev_up = [torch.cuda.Event() for _ in range(e2e_steps)]
@@ -724,6 +889,18 @@ def run_ours(args):
                 d_t.copy_(h_t, non_blocking=True)
             ev_up[i].record(up)
 
+    def e2e_compute(i):
+        r = dres[i % 2]
+        path.inputs = [dbuf[i % 2]]
+        path._quantize(i)
+        if w.group_quant:
+            path._attend(out, None)
+            fv.per_token_group_quant_fp8(out.view(T, H * D), 128, r[0], r[1], ctx=ctx)
+        elif w.fp8_out:
+            path._attend(r[0], path.oscale)
+        else:
+            path._attend(r[0], None)
+
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
@@ -737,23 +914,19 @@ def run_ours(args):
             upload(i + 1)
         stream.wait_event(ev_up[i])
         if i >= 2:
-            stream.wait_event(ev_down[i - 2])  # dxq/dxs[i % 2] have been read back
-        dq, dk, dv = dbuf[i % 2]
-        fv.fp8_amax_ring_quantize_qkv(dq, dk, dv, rings[i % len(rings)], desc, q8, k8, v8,
-                                      ctx=ctx)
-        fv.fp8_varlen_attn_fwd(q8, k8, v8, desc[0:1], desc[1:2], desc[2:3], cu, max_s,
-                               w.softmax_scale, out, ctx=ctx)
-        fv.per_token_group_quant_fp8(out.view(T, H * D), 128, dxq[i % 2], dxs[i % 2], ctx=ctx)
+            stream.wait_event(ev_down[i - 2])  # result buffers [i % 2] have been read back
+        e2e_compute(i)
         ev_done[i].record(stream)
         with torch.cuda.stream(down):
             down.wait_event(ev_done[i])
-            host_xq[i % 2].copy_(dxq[i % 2], non_blocking=True)
-            host_xs[i % 2].copy_(dxs[i % 2], non_blocking=True)
+            for h_t, d_t in zip(hres[i % 2], dres[i % 2]):
+                h_t.copy_(d_t, non_blocking=True)
             ev_down[i].record(down)
     stream.wait_stream(up)
     stream.wait_stream(down)
     e1.record(stream)
     torch.cuda.synchronize()
+    path.inputs = inputs
     e2e_ms = e0.elapsed_time(e1)
     if dist:
         t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
@@ -761,7 +934,7 @@ def run_ours(args):
         e2e_ms = float(t.item())
     e2e_value = ws * flops_step * e2e_steps / (e2e_ms * 1e-3) / 1e12
     h2d = 3 * T * H * D * 2
-    d2h = xq.numel() + xs.numel() * 4
+    d2h = sum(t.numel() * t.element_size() for t in dres[0])
 
     # forward 0 once more from a fresh ring (untimed), for the CPU-baseline
     # leg's full-size parity check
@@ -769,7 +942,8 @@ def run_ours(args):
     fwd0 = None
     if cpu_leg:
         try:
-            fwd0 = _forward0_outputs(fv, ctx, w, inputs[0], cu, max_s, q8, k8, v8, out, dev)
+            fwd0 = _forward0_outputs(fv, ctx, w, inputs[0], cu, max_s, q8, k8, v8, out, dev,
+                                     static_desc=path.desc if w.mode == "static" else None)
         except Exception as exc:  # reported in the line's parity field, not dropped
             fwd0 = exc
 
@@ -793,7 +967,8 @@ def run_ours(args):
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "copies": "pinned host buffers; uploads, compute and read-backs on three "
                           "streams, double-buffered, overlapping across steps"},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": _launches_per_step(
+            w, torch.cuda.get_device_properties(dev).L2_cache_size) * args.steps,
         "clocks": clk,
         "quantizers": quant,
     }
@@ -807,6 +982,10 @@ def run_ours(args):
         line["attn_sweep"] = _attn_sweep(fv, ctx, dev)
     if args.output_modes:
         line["output_modes"] = _output_modes(fv, ctx, w, inputs, dev)
+    if rank == 0 and ws == 1 and not args.no_configs:
+        del path, inputs
+        torch.cuda.empty_cache()
+        line["configs"] = _config_records(fv, ctx, dev, peaks, stream)
     if cpu_leg:
         codes, dsc = _oracle_inputs(w)
         threads = _host_threads()
@@ -843,6 +1022,9 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=1.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-quant-roofline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-workload records (each target workload's own step "
+                         "timed in the same run)")
     ap.add_argument("--p-terms", type=int, choices=[1, 2], default=2,
                     help="e4m3 terms of P in the PV product (2: hi + lo, the default that meets "
                          "the attention tolerance; 1: a single term, faster, less accurate)")

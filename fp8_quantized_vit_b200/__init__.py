@@ -37,6 +37,8 @@ _SIGNATURES = {
     "fp8vit_check": (_I32, [_P, _P, ctypes.POINTER(_I32)]),
     "fp8vit_status_string": (ctypes.c_char_p, [_I32]),
     "fp8vit_set_attn_p_terms": (_I32, [_P, _I32]),
+    "fp8vit_tmap_cache_stats": (_I32, [_P, ctypes.POINTER(ctypes.c_uint64),
+                                       ctypes.POINTER(ctypes.c_uint64)]),
     "fp8vit_inject_lost_arrival": (_I32, [_P, _P]),
     "fp8vit_inject_attn_timeout": (_I32, [_P, _P]),
     "fp8vit_version": (_I32, []),
@@ -52,6 +54,8 @@ _SIGNATURES = {
                                    _F32, _P, _I32, _P, _P]),
     "bf16_varlen_attn_fwd": (_I32, [_P, _P, _P, _P, _P, _I32, _I32, _I64, _I32, _I32, _F32, _P,
                                     _P]),
+    "fp8_varlen_attn_fwd_qbf16": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I64, _I32,
+                                         _I32, _F32, _P, _I32, _P, _P]),
     "fp8_varlen_attn_fwd_group_quant": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I64,
                                                _I32, _I32, _F32, _P, _P, _P]),
     "per_token_group_quant_fp8": (_I32, [_P, _P, _I64, _I64, _I32, _P, _P, _P]),
@@ -136,6 +140,13 @@ class Context:
         site = _I32(0)
         st = lib().fp8vit_check(self.handle, _stream(stream), ctypes.byref(site))
         return st, site.value
+
+    def tmap_cache_stats(self) -> tuple[int, int]:
+        """(hits, misses) of the context's tensor-map cache."""
+        h, m = ctypes.c_uint64(0), ctypes.c_uint64(0)
+        _check(lib().fp8vit_tmap_cache_stats(self.handle, ctypes.byref(h), ctypes.byref(m)),
+               "fp8vit_tmap_cache_stats")
+        return h.value, m.value
 
     def set_attn_p_terms(self, terms: int):
         """P of the attention's PV product as 2 e4m3 terms (hi + lo, the
@@ -242,8 +253,10 @@ def fp8_ring_read_amax(ring, stream=None) -> list[float]:
 # ---- quantizers ----------------------------------------------------------------------
 
 def fp8_quantize_qkv_per_tensor(q, k, v, descale3, q8, k8, v8, ctx=None, stream=None):
+    """Per-tensor e4m3 codes of q, k, v with the device descales; q8=None
+    leaves Q to fp8_varlen_attn_fwd_qbf16, which quantizes it itself."""
     n = q.numel()
-    for t in (k, v, q8, k8, v8):
+    for t in (k, v, k8, v8) + ((q8,) if q8 is not None else ()):
         if t.numel() != n:
             raise ValueError("all tensors must have the same number of elements")
     _check(lib().fp8_quantize_qkv_per_tensor(
@@ -256,9 +269,10 @@ def fp8_quantize_qkv_per_tensor(q, k, v, descale3, q8, k8, v8, ctx=None, stream=
 
 def fp8_amax_ring_quantize_qkv(q, k, v, ring, descale3, q8, k8, v8, ctx=None, stream=None):
     """fp8_amax_ring_update followed by fp8_quantize_qkv_per_tensor in one
-    cooperative launch (same ring state, descales and codes)."""
+    cooperative launch (same ring state, descales and codes); q8=None leaves
+    Q's codes to fp8_varlen_attn_fwd_qbf16 (the amax still covers Q)."""
     n = q.numel()
-    for t in (k, v, q8, k8, v8):
+    for t in (k, v, k8, v8) + ((q8,) if q8 is not None else ()):
         if t.numel() != n:
             raise ValueError("all tensors must have the same number of elements")
     _check(lib().fp8_amax_ring_quantize_qkv(
@@ -300,6 +314,29 @@ def fp8_varlen_attn_fwd(q8, k8, v8, q_descale, k_descale, v_descale, cu_seqlens,
         _ptr(out, _FP8 if fp8_out else torch.bfloat16, "out"), 1 if fp8_out else 0,
         _ptr(output_scale, torch.float32, "output_scale"), _stream(stream)),
         "fp8_varlen_attn_fwd")
+    return out
+
+
+def fp8_varlen_attn_fwd_qbf16(q, k8, v8, q_descale, k_descale, v_descale, cu_seqlens,
+                              max_seqlen, softmax_scale, out, output_scale=None, ctx=None,
+                              stream=None):
+    """fp8_varlen_attn_fwd with Q given in BF16 [T, H, D]: the kernel divides
+    it by q_descale and rounds it to e4m3 in its prologue (the same bytes the
+    per-tensor quantizer writes), so Q's codes never go through memory."""
+    if q.dim() != 3:
+        raise ValueError("q must be [T, H, D]")
+    T, H, D = q.shape
+    if k8.shape != q.shape or v8.shape != q.shape or out.shape != q.shape:
+        raise ValueError("q, k8, v8 and out must have the same [T, H, D] shape")
+    fp8_out = output_scale is not None
+    _check(lib().fp8_varlen_attn_fwd_qbf16(
+        _ctx(ctx), _ptr(q, torch.bfloat16, "q"), _ptr(k8, _FP8, "k8"), _ptr(v8, _FP8, "v8"),
+        _ptr(q_descale, torch.float32, "q_descale"), _ptr(k_descale, torch.float32, "k_descale"),
+        _ptr(v_descale, torch.float32, "v_descale"), _ptr(cu_seqlens, torch.int32, "cu_seqlens"),
+        cu_seqlens.numel() - 1, int(max_seqlen), T, H, D, float(softmax_scale),
+        _ptr(out, _FP8 if fp8_out else torch.bfloat16, "out"), 1 if fp8_out else 0,
+        _ptr(output_scale, torch.float32, "output_scale"), _stream(stream)),
+        "fp8_varlen_attn_fwd_qbf16")
     return out
 
 
@@ -386,8 +423,11 @@ class FP8EncoderAttention:
 
     def __init__(self, num_heads: int, head_dim: int, softmax_scale: float | None = None,
                  static_amax=None, margin: float = 1.5, device=None, ctx: Context | None = None,
-                 process_group=None):
+                 process_group=None, fold_q: bool = False):
         self.H, self.D = num_heads, head_dim
+        # fold_q: the attention kernel quantizes Q in its prologue
+        # (fp8_varlen_attn_fwd_qbf16); the quantizer writes only K and V codes
+        self.fold_q = fold_q
         self.softmax_scale = (float(torch.tensor(head_dim ** -0.5, dtype=torch.float32))
                               if softmax_scale is None else softmax_scale)
         self.device = torch.device(device or "cuda")
@@ -450,6 +490,8 @@ class FP8EncoderAttention:
         if group_quant and (self.H * self.D) % 128 != 0:
             raise ValueError("group_quant needs num_heads * head_dim to be a multiple of 128")
         b = self._buffers(T, output_scale is not None, group_quant)
+        fold = self.fold_q and not (group_quant and self.D == 128)
+        q8 = None if fold else b["q8"]
         if self.ring is not None and self.process_group is not None:
             # this rank holds some of the batch's images: agree on the
             # per-tensor amax with the other ranks before the ring update
@@ -459,11 +501,13 @@ class FP8EncoderAttention:
             fp8_ring_push(self._amax3, self.ring, self.descale)
         if self.ring is not None and self.process_group is None:
             # amax, ring rule and quantization in one cooperative launch
-            fp8_amax_ring_quantize_qkv(q, k, v, self.ring, self.descale, b["q8"], b["k8"],
+            fp8_amax_ring_quantize_qkv(q, k, v, self.ring, self.descale, q8, b["k8"],
                                        b["v8"], ctx=self.ctx)
         else:
-            fp8_quantize_qkv_per_tensor(q, k, v, self.descale, b["q8"], b["k8"], b["v8"],
+            fp8_quantize_qkv_per_tensor(q, k, v, self.descale, q8, b["k8"], b["v8"],
                                         ctx=self.ctx)
+        attn = fp8_varlen_attn_fwd_qbf16 if fold else fp8_varlen_attn_fwd
+        qa = q if fold else b["q8"]
         if group_quant:
             hd = self.H * self.D
             xq, xs = b["xq"], b["xs"]
@@ -474,15 +518,15 @@ class FP8EncoderAttention:
                                                 ctx=self.ctx)
             else:
                 o = b["out"]
-                fp8_varlen_attn_fwd(b["q8"], b["k8"], b["v8"], self.descale[0:1],
-                                    self.descale[1:2], self.descale[2:3], cu_seqlens, max_seqlen,
-                                    self.softmax_scale, o, ctx=self.ctx)
+                attn(qa, b["k8"], b["v8"], self.descale[0:1], self.descale[1:2],
+                     self.descale[2:3], cu_seqlens, max_seqlen, self.softmax_scale, o,
+                     ctx=self.ctx)
                 per_token_group_quant_fp8(o.view(T, hd), 128, xq, xs, ctx=self.ctx)
             return xq, xs
         o = b["out"] if out is None else out
-        fp8_varlen_attn_fwd(b["q8"], b["k8"], b["v8"], self.descale[0:1], self.descale[1:2],
-                            self.descale[2:3], cu_seqlens, max_seqlen, self.softmax_scale, o,
-                            output_scale=output_scale, ctx=self.ctx)
+        attn(qa, b["k8"], b["v8"], self.descale[0:1], self.descale[1:2], self.descale[2:3],
+             cu_seqlens, max_seqlen, self.softmax_scale, o, output_scale=output_scale,
+             ctx=self.ctx)
         return o
 
     __call__ = forward

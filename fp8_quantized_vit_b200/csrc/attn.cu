@@ -139,27 +139,42 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, u
 
 
 
+// Four fp32 values that are exact in e4m3 -> their four codes in one word
+// (first value in byte 0), by the 4-wide conversion; its rounding (rbits = 0:
+// toward zero) never applies to exact values.
+__device__ __forceinline__ uint32_t e4m3x4_exact(float a, float b, float c, float d) {
+    uint32_t r;
+    asm("cvt.rs.satfinite.e4m3x4.f32 %0, {%4, %3, %2, %1}, %5;"
+        : "=r"(r)
+        : "f"(a), "f"(b), "f"(c), "f"(d), "r"(0u));
+    return r;
+}
+
+// Four fp32 -> four e4m3 codes (RNE, satfinite), first value in byte 0.
+__device__ __forceinline__ uint32_t e4m3x4_rn(float a, float b, float c, float d) {
+    return (uint32_t)f32x2_to_e4m3x2(a, b) | ((uint32_t)f32x2_to_e4m3x2(c, d) << 16);
+}
+
 // Probabilities of one 32-key chunk: p = 2^(s * c - bias) (a score of -inf
-// gives 0), summed into the two packed accumulators, then split into 8 hi and
-// 8 lo words of e4m3 codes with hi + lo ~= p to ~8 significant bits, so that
-// the PV product on FP8 tensor cores keeps about a BF16-width P: p is rounded
-// to f16 (11 bits); hi = e4m3(p16); the residual p16 - hi is exact in f16
-// (both share the exponent range of p16); lo = e4m3(residual).  Five
-// conversions/subtracts per pair, written stage by stage over the chunk.  The
-// words are combined from zero-extended halves with shifts (packing two
-// 16-bit asm results with mov.b32 {a, b} was miscompiled here).
+// gives 0), summed into the two packed accumulators, then written as e4m3
+// words pk[0..7] (hi) and pk[8..15] (lo), key 4i+k in byte k of word i, with
+// hi + lo ~= p to ~8 significant bits, so that the PV product on FP8 tensor
+// cores keeps about a BF16-width P.  hi = p with its fp32 mantissa cut to 3
+// bits (a mask; exact in e4m3 wherever p is e4m3-normal, and the P scaling
+// keeps the significant probabilities there), lo = RN_e4m3(p - hi) with
+// p - hi exact in fp32: the only rounding, of lo, is to nearest, so the pair
+// carries no bias and its error is below 2^-7 p.  Per four probabilities:
+// four masks, two packed subtracts, one 4-wide conversion for hi and two
+// 2-wide conversions for lo (no f16 round trip).
 template <bool PLO>
 __device__ __forceinline__ void p_chunk(const uint32_t (&r)[32], uint64_t c2, uint64_t nb2,
                                         uint64_t& l0, uint64_t& l1, uint32_t (&pk)[16]) {
     float p[32];
-    uint64_t x[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-        x[i] = ffma2(f2pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), c2, nb2);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         float x0, x1;
-        f2unpack(x[i], x0, x1);
+        f2unpack(ffma2(f2pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), c2, nb2),
+                 x0, x1);
         p[2 * i] = ex2_approx(x0);
         p[2 * i + 1] = ex2_approx(x1);
     }
@@ -172,22 +187,20 @@ __device__ __forceinline__ void p_chunk(const uint32_t (&r)[32], uint64_t c2, ui
         // single e4m3 term: P rounded once, straight from fp32
 #pragma unroll
         for (int w = 0; w < 8; ++w)
-            pk[w] = (uint32_t)f32x2_to_e4m3x2(p[4 * w], p[4 * w + 1]) |
-                    ((uint32_t)f32x2_to_e4m3x2(p[4 * w + 2], p[4 * w + 3]) << 16);
+            pk[w] = e4m3x4_rn(p[4 * w], p[4 * w + 1], p[4 * w + 2], p[4 * w + 3]);
     } else {
-        uint32_t h[16], e[16], d[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) h[i] = cvt_f16x2(p[2 * i], p[2 * i + 1]);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) e[i] = e4m3x2_of_f16x2(h[i]);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) d[i] = hsub2(h[i], f16x2_of_e4m3x2(e[i]));
-#pragma unroll
-        for (int i = 0; i < 16; ++i) d[i] = e4m3x2_of_f16x2(d[i]);
+        const uint64_t m1 = f2pack(-1.0f, -1.0f);
 #pragma unroll
         for (int w = 0; w < 8; ++w) {
-            pk[w] = e[2 * w] | (e[2 * w + 1] << 16);
-            pk[8 + w] = d[2 * w] | (d[2 * w + 1] << 16);
+            float hf[4], lf[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                hf[i] = __uint_as_float(__float_as_uint(p[4 * w + i]) & 0xFFF00000u);
+            f2unpack(ffma2(f2pack(hf[0], hf[1]), m1, f2pack(p[4 * w], p[4 * w + 1])), lf[0], lf[1]);
+            f2unpack(ffma2(f2pack(hf[2], hf[3]), m1, f2pack(p[4 * w + 2], p[4 * w + 3])), lf[2],
+                     lf[3]);
+            pk[w] = e4m3x4_exact(hf[0], hf[1], hf[2], hf[3]);
+            pk[8 + w] = e4m3x4_rn(lf[0], lf[1], lf[2], lf[3]);
         }
     }
 }
@@ -266,7 +279,10 @@ __device__ __forceinline__ void tmem_st_p_any(uint32_t taddr, const uint32_t (&p
 // OUT selects the epilogue at compile time; PLO keeps P as two e4m3 terms
 // (hi + lo, two PV MMAs) or, when false, as one.  BF: the inputs are BF16
 // (no descales) and both products run as kind::f16 MMAs with P in BF16.
-template <int D, int OUT, bool PLO, bool BF = false>
+// QB: Q arrives as BF16 (qbf) and the prologue quantizes it with the Q
+// descale into the e4m3 Q tile (each softmax thread its own row), so the
+// per-tensor quantizer need not write or read Q's codes.
+template <int D, int OUT, bool PLO, bool BF = false, bool QB = false>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ dq_p,
@@ -274,9 +290,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                     const int32_t* __restrict__ cu, int32_t max_seqlen, int64_t total_tokens,
                     int32_t num_heads, float sm_scale, void* __restrict__ out,
                     const float* __restrict__ out_scale_p, float* __restrict__ gscales,
-                    fp8vit_scratch* __restrict__ scr) {
+                    fp8vit_scratch* __restrict__ scr, const uint16_t* __restrict__ qbf) {
     static_assert(OUT != kOutGroupQ || D == 128, "a 128-wide group is one head at head_dim 128");
     static_assert(!BF || OUT == kOutBf16, "bf16 inputs: bf16 output");
+    static_assert(!(BF && QB), "BF16 Q is quantized only on the FP8 path");
     using C = CfgOf<D, BF>;
     using L = SmemOf<C>;
     constexpr int E = BF ? 2 : 1;  // bytes per element
@@ -360,10 +377,12 @@ __global__ void __launch_bounds__(kThreads, 2)
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
-            mbar_arrive_expect_tx(b_q_full, C::KB * kQTileBytes);
-            for (int kb = 0; kb < C::KB; ++kb)
-                tma_load_2d(sQ + kb * kQTileBytes, &tm_q, x0 + kBox * kb, seg_start + q0,
-                            b_q_full);
+            if constexpr (!QB) {
+                mbar_arrive_expect_tx(b_q_full, C::KB * kQTileBytes);
+                for (int kb = 0; kb < C::KB; ++kb)
+                    tma_load_2d(sQ + kb * kQTileBytes, &tm_q, x0 + kBox * kb, seg_start + q0,
+                                b_q_full);
+            }
             int issued = 0;
             for (int j = 0; j < n_kv; ++j) {
                 const int s = j % NS;
@@ -382,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 ++issued;
             }
             // Drain: every issued copy must land before the CTA may exit.
-            mbar_wait_drain(b_q_full, 0, scr);
+            if constexpr (!QB) mbar_wait_drain(b_q_full, 0, scr);
             for (int j = issued - 1; j >= 0 && j >= issued - NS; --j)
                 mbar_wait_drain(b_kv_full(j % NS), (j / NS) & 1, scr);
         }
@@ -395,21 +414,23 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (lane == 0) {
             constexpr uint32_t idesc_qk = BF ? idesc_bf16(C::BN, false) : idesc_e4m3(C::BN, false);
             constexpr uint32_t idesc_pv = BF ? idesc_bf16(C::NPV, true) : idesc_e4m3(C::NPV, true);
-            const uint32_t tO = tmem + C::TO;
+            // The issue loop is on the tensor core's critical path: a single
+            // thread's scalar work between MMAs is comparable to an MMA, so
+            // descriptors are formed once and advanced by constants (one box
+            // is KVT >> 4 descriptor address units), and stages and phases
+            // are counters instead of divisions.
+            constexpr uint64_t kQBox = kQTileBytes >> 4, kKVBox = L::KVT >> 4;
+            const uint32_t tO = tmem + C::TO, tS = tmem + C::TS;
+            const uint64_t qd = desc_k_sw32(sQ), kd0 = desc_k_sw32(sK);
+            const uint64_t vd0 = desc_mn_sw32<L::KVT>(sV);
             const bool skip_first_s = *reinterpret_cast<volatile uint32_t*>(&scr->inject_attn) != 0;
-            auto issue_qk = [&](int j) {
-                const int s = j % NS;
-                const uint32_t tSb = tmem + C::TS;
+            auto issue_qk = [&](int s) {
+                const uint64_t kd = kd0 + (uint64_t)(s * C::KB) * kKVBox;
 #pragma unroll
                 for (int kb = 0; kb < C::KB; ++kb) {
-                    const uint64_t ad = desc_k_sw32(sQ + kb * kQTileBytes);
-                    const uint64_t bd = desc_k_sw32(sK + (s * C::KB + kb) * L::KVT);
-                    if constexpr (BF) umma_bf16_ss(tSb, ad, bd, idesc_qk, kb > 0 ? 1u : 0u);
-                    else umma_f8_ss(tSb, ad, bd, idesc_qk, kb > 0 ? 1u : 0u);
+                    if constexpr (BF) umma_bf16_ss(tS, qd + kb * kQBox, kd + kb * kKVBox, idesc_qk, kb > 0 ? 1u : 0u);
+                    else umma_f8_ss(tS, qd + kb * kQBox, kd + kb * kKVBox, idesc_qk, kb > 0 ? 1u : 0u);
                 }
-                // test hook (fp8vit_inject_attn_timeout): S(0) is never
-                // announced, so the softmax warps' bounded wait runs out
-                if (j > 0 || !skip_first_s) umma_commit(b_s_full);
             };
             bool ok = mbar_wait_bounded(b_q_ready, 0, abort_flag, scr, SITE_ATTN_WAIT_QREADY,
                                         kTimeoutNs);
@@ -420,35 +441,43 @@ __global__ void __launch_bounds__(kThreads, 2)
                 if (ok) {
                     tc_fence_after();
                     issue_qk(0);
+                    // test hook (fp8vit_inject_attn_timeout): S(0) is never
+                    // announced, so the softmax warps' bounded wait runs out
+                    if (!skip_first_s) umma_commit(b_s_full);
                     issued_any = true;
                 }
             }
+            int sk = NS > 1 ? 1 : 0, sv = 0;  // stages of the next QK and of the next PV
+            uint32_t phk = NS > 1 ? 0u : 1u;   // fill phase of stage sk
             for (int j = 0; ok && j < n_kv; ++j) {
                 if (j + 1 < n_kv) {
-                    const int s1 = (j + 1) % NS;
-                    if (!mbar_wait_bounded(b_kv_full(s1), ((j + 1) / NS) & 1, abort_flag, scr,
-                                           SITE_ATTN_WAIT_K, kTimeoutNs))
+                    if (!mbar_wait_bounded(b_kv_full(sk), phk, abort_flag, scr, SITE_ATTN_WAIT_K,
+                                           kTimeoutNs))
                         break;
                     if (!mbar_wait_bounded(b_s_free, j & 1, abort_flag, scr, SITE_ATTN_WAIT_SFREE,
                                            kTimeoutNs))
                         break;
                     tc_fence_after();
-                    issue_qk(j + 1);
+                    issue_qk(sk);
+                    umma_commit(b_s_full);
+                    if (++sk == NS) {
+                        sk = 0;
+                        phk ^= 1u;
+                    }
                 }
                 // V(j) landed with K(j), which QK(j) waited for.
-                const int s = j % NS;
                 if (!mbar_wait_bounded(b_p_full(j & 1), (j >> 1) & 1, abort_flag, scr,
                                        SITE_ATTN_WAIT_P, kTimeoutNs))
                     break;
                 tc_fence_after();
                 const uint32_t tPb = tmem + C::TP + (C::PSLOTS == 2 ? 32 * (j & 1) : 0);
-                const uint32_t vbase = sV + s * C::VA * L::KVT;
+                const uint64_t vd = vd0 + (uint64_t)(sv * C::VA) * kKVBox;
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 32; ++kk) {
-                    const uint64_t bdesc = desc_mn_sw32<L::KVT>(vbase + kk * 32 * kBox);
+                    const uint64_t bdesc = vd + (uint64_t)((kk * 32 * kBox) >> 4);
                     if constexpr (BF) {
                         // keys 32kk..32kk+15 at P columns +0, the next 16 keys at +8
-                        const uint64_t bdesc2 = desc_mn_sw32<L::KVT>(vbase + (kk * 32 + 16) * kBox);
+                        const uint64_t bdesc2 = vd + (uint64_t)(((kk * 32 + 16) * kBox) >> 4);
                         umma_bf16_ts(tO, tPb + 16 * kk, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
                         umma_bf16_ts(tO, tPb + 16 * kk + 8, bdesc2, idesc_pv, 1u);
                     } else {
@@ -457,7 +486,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                     }
                 }
                 umma_commit(b_o_ready(j & 1));
-                umma_commit(b_kv_empty(s));
+                umma_commit(b_kv_empty(sv));
+                if (++sv == NS) sv = 0;
             }
             // Never leave MMAs in flight: one more commit tracks all of them.
             if (issued_any) {
@@ -474,9 +504,49 @@ __global__ void __launch_bounds__(kThreads, 2)
         const float dq = BF ? 1.0f : *dq_p, dk = BF ? 1.0f : *dk_p, dv = BF ? 1.0f : *dv_p;
         const float scale_log2 = sm_scale * dq * dk * 1.4426950408889634f;
 
-        bool ok = mbar_wait_bounded(b_q_full, 0, abort_flag, scr, SITE_ATTN_WAIT_Q, kTimeoutNs);
-        ok = __all_sync(0xFFFFFFFFu, ok);
-        if (ok && D == 72 && BF) {
+        bool ok = true;
+        if constexpr (QB) {
+            // This row's BF16 Q of the head, divided by the Q descale (IEEE
+            // fp32, as the per-tensor quantizer) and rounded to e4m3, into the
+            // QK window of KB x 32 bytes: the head at col_off, zeros around
+            // it (so the neighbouring head's K bytes contribute exactly 0), and
+            // zeros for rows past the image.  SW32 layout as the TMA writes it:
+            // row r of k-block kb at kb*4096 + r*32, 16-byte chunk c at c ^ ((r>>2)&1).
+            uint32_t wq[C::KB * 8];
+#pragma unroll
+            for (int i = 0; i < C::KB * 8; ++i) wq[i] = 0;
+            if (q0 + row < seg_len) {
+                const uint4* src = reinterpret_cast<const uint4*>(
+                    qbf + ((int64_t)(seg_start + q0 + row) * num_heads + h) * D);
+                const float rq = __frcp_rn(dq);
+#pragma unroll
+                for (int v = 0; v < D / 8; ++v) {
+                    const uint2 c = quant8(__ldg(src + v), dq, rq);
+                    if (col_off == 0) {
+                        wq[2 * v] = c.x;
+                        wq[2 * v + 1] = c.y;
+                    } else {
+                        wq[2 * v + 2] = c.x;
+                        wq[2 * v + 3] = c.y;
+                    }
+                }
+            }
+            const int sw = (row >> 2) & 1;
+#pragma unroll
+            for (int kb = 0; kb < C::KB; ++kb)
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+                    *reinterpret_cast<uint4*>(sm + L::Q + kb * kQTileBytes + row * kBox +
+                                              ((c ^ sw) << 4)) =
+                        make_uint4(wq[8 * kb + 4 * c], wq[8 * kb + 4 * c + 1],
+                                   wq[8 * kb + 4 * c + 2], wq[8 * kb + 4 * c + 3]);
+        } else {
+            ok = mbar_wait_bounded(b_q_full, 0, abort_flag, scr, SITE_ATTN_WAIT_Q, kTimeoutNs);
+            ok = __all_sync(0xFFFFFFFFu, ok);
+        }
+        if (QB) {
+            // the Q tile is complete as written above
+        } else if (ok && D == 72 && BF) {
             // BF16: the 160-byte window's last 16 bytes (chunk 1 of k-block 4)
             // belong to the next head.
             const int sw = (row >> 2) & 1;
@@ -676,23 +746,29 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 
+// qbf non-null: Q is BF16 (the kernel quantizes it with dq in its prologue)
+// and q8 is ignored.
 template <int D, int OUT>
 fp8vit_status launch(fp8vit_ctx* ctx, const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
                      const float* dq, const float* dk, const float* dv, const int32_t* cu,
                      int32_t num_seqs, int32_t max_seqlen, int64_t T, int32_t H, float sm_scale,
-                     void* out, const float* out_scale, float* gscales, cudaStream_t st) {
+                     void* out, const float* out_scale, float* gscales, cudaStream_t st,
+                     const uint16_t* qbf = nullptr) {
     CUtensorMap mq, mk, mv;
     const int64_t row_bytes = (int64_t)H * D;
-    if (!encode_map(&mq, q8, T, row_bytes, kBM) ||
-        !encode_map(&mk, k8, T, row_bytes, Cfg<D>::BN) ||
-        !encode_map(&mv, v8, T, row_bytes, Cfg<D>::BN))
+    if (!cached_map(ctx, &mk, k8, T, row_bytes, Cfg<D>::BN) ||
+        !cached_map(ctx, &mv, v8, T, row_bytes, Cfg<D>::BN))
         return FP8VIT_ECUDA;
+    if (qbf) mq = mk;  // not read by the kernel
+    else if (!cached_map(ctx, &mq, q8, T, row_bytes, kBM)) return FP8VIT_ECUDA;
     // The dynamic shared-memory limit is a per-device setting of each kernel
     // instance: raise it once per (device, instance).
-    static std::atomic<uint64_t> attr_set[2];
+    static std::atomic<uint64_t> attr_set[4];
     const bool two_terms = ctx->attn_p_terms != 1;
-    const int inst = two_terms ? 1 : 0;
-    auto kern = two_terms ? attn_fwd_kernel<D, OUT, true> : attn_fwd_kernel<D, OUT, false>;
+    const int inst = (two_terms ? 1 : 0) + (qbf ? 2 : 0);
+    auto kern = qbf ? (two_terms ? attn_fwd_kernel<D, OUT, true, false, true>
+                                 : attn_fwd_kernel<D, OUT, false, false, true>)
+                    : (two_terms ? attn_fwd_kernel<D, OUT, true> : attn_fwd_kernel<D, OUT, false>);
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FP8VIT_ECUDA;
     const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
@@ -705,7 +781,7 @@ fp8vit_status launch(fp8vit_ctx* ctx, const uint8_t* q8, const uint8_t* k8, cons
     dim3 grid((unsigned)((max_seqlen + kBM - 1) / kBM), (unsigned)H, (unsigned)num_seqs);
     kern<<<grid, kThreads, Smem<D>::ALLOC, st>>>(mq, mk, mv, dq, dk, dv, cu, max_seqlen, T, H,
                                                  sm_scale, out, out_scale, gscales,
-                                                 ctx->d_scratch);
+                                                 ctx->d_scratch, qbf);
     return cudaGetLastError() == cudaSuccess ? FP8VIT_OK : FP8VIT_ECUDA;
 }
 
@@ -718,8 +794,8 @@ fp8vit_status launch_bf16(fp8vit_ctx* ctx, const uint16_t* q, const uint16_t* k,
     using L = SmemOf<C>;
     CUtensorMap mq, mk, mv;
     const int64_t row_bytes = (int64_t)H * D * 2;
-    if (!encode_map(&mq, q, T, row_bytes, kBM) || !encode_map(&mk, k, T, row_bytes, C::BN) ||
-        !encode_map(&mv, v, T, row_bytes, C::BN))
+    if (!cached_map(ctx, &mq, q, T, row_bytes, kBM) || !cached_map(ctx, &mk, k, T, row_bytes, C::BN) ||
+        !cached_map(ctx, &mv, v, T, row_bytes, C::BN))
         return FP8VIT_ECUDA;
     static std::atomic<uint64_t> attr_set;
     auto kern = attn_fwd_kernel<D, kOutBf16, true, true>;
@@ -734,7 +810,8 @@ fp8vit_status launch_bf16(fp8vit_ctx* ctx, const uint16_t* q, const uint16_t* k,
     }
     dim3 grid((unsigned)((max_seqlen + kBM - 1) / kBM), (unsigned)H, (unsigned)num_seqs);
     kern<<<grid, kThreads, L::ALLOC, st>>>(mq, mk, mv, nullptr, nullptr, nullptr, cu, max_seqlen, T,
-                                           H, sm_scale, out, nullptr, nullptr, ctx->d_scratch);
+                                           H, sm_scale, out, nullptr, nullptr, ctx->d_scratch,
+                                           nullptr);
     return cudaGetLastError() == cudaSuccess ? FP8VIT_OK : FP8VIT_ECUDA;
 }
 
@@ -783,6 +860,50 @@ extern "C" fp8vit_status fp8_varlen_attn_fwd(
                                        d_v_descale, d_cu_seqlens, num_seqs, max_seqlen,
                                        total_tokens, num_heads, softmax_scale, d_out,
                                        d_output_scale, nullptr, st);
+}
+
+extern "C" fp8vit_status fp8_varlen_attn_fwd_qbf16(
+    fp8vit_ctx* ctx, const uint16_t* d_q, const uint8_t* d_k8, const uint8_t* d_v8,
+    const float* d_q_descale, const float* d_k_descale, const float* d_v_descale,
+    const int32_t* d_cu_seqlens, int32_t num_seqs, int32_t max_seqlen, int64_t total_tokens,
+    int32_t num_heads, int32_t head_dim, float softmax_scale, void* d_out, int32_t out_dtype,
+    const float* d_output_scale, void* stream) {
+    if (!ctx || !d_q || !d_k8 || !d_v8 || !d_q_descale || !d_k_descale || !d_v_descale ||
+        !d_cu_seqlens || !d_out)
+        return FP8VIT_EINVAL;
+    if (num_seqs < 0 || max_seqlen < 0 || total_tokens < 0 || total_tokens > INT32_MAX ||
+        num_heads < 1)
+        return FP8VIT_EINVAL;
+    if (!(softmax_scale > 0.0f) || !isfinite(softmax_scale)) return FP8VIT_EINVAL;
+    if (out_dtype != 0 && out_dtype != 1) return FP8VIT_EINVAL;
+    if ((out_dtype == 1) != (d_output_scale != nullptr)) return FP8VIT_EINVAL;
+    if (head_dim != 72 && head_dim != 128) return FP8VIT_EUNSUPPORTED;
+    if (((int64_t)num_heads * head_dim) % 16 != 0) return FP8VIT_EUNSUPPORTED;
+    if (misaligned(d_q, 16) || misaligned(d_k8, 16) || misaligned(d_v8, 16) ||
+        misaligned(d_out, out_dtype == 0 ? 16 : 8) || misaligned(d_cu_seqlens, 4))
+        return FP8VIT_EINVAL;
+    if (num_heads > 65535 || num_seqs > 65535) return FP8VIT_EUNSUPPORTED;
+    if (num_seqs == 0 || max_seqlen == 0 || total_tokens == 0) return FP8VIT_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (head_dim == 72)
+        return out_dtype == 0
+                   ? launch<72, kOutBf16>(ctx, nullptr, d_k8, d_v8, d_q_descale, d_k_descale,
+                                          d_v_descale, d_cu_seqlens, num_seqs, max_seqlen,
+                                          total_tokens, num_heads, softmax_scale, d_out, nullptr,
+                                          nullptr, st, d_q)
+                   : launch<72, kOutE4m3>(ctx, nullptr, d_k8, d_v8, d_q_descale, d_k_descale,
+                                          d_v_descale, d_cu_seqlens, num_seqs, max_seqlen,
+                                          total_tokens, num_heads, softmax_scale, d_out,
+                                          d_output_scale, nullptr, st, d_q);
+    return out_dtype == 0
+               ? launch<128, kOutBf16>(ctx, nullptr, d_k8, d_v8, d_q_descale, d_k_descale,
+                                       d_v_descale, d_cu_seqlens, num_seqs, max_seqlen,
+                                       total_tokens, num_heads, softmax_scale, d_out, nullptr,
+                                       nullptr, st, d_q)
+               : launch<128, kOutE4m3>(ctx, nullptr, d_k8, d_v8, d_q_descale, d_k_descale,
+                                       d_v_descale, d_cu_seqlens, num_seqs, max_seqlen,
+                                       total_tokens, num_heads, softmax_scale, d_out,
+                                       d_output_scale, nullptr, st, d_q);
 }
 
 extern "C" fp8vit_status fp8_varlen_attn_fwd_group_quant(

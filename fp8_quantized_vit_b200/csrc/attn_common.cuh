@@ -223,6 +223,33 @@ inline bool encode_map(CUtensorMap* map, const void* base, int64_t rows, int64_t
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The 2-D uint8 tensor map of encode_map, from the context's cache when the
+// same (base, rows, row_bytes, box_rows) was encoded before; encodes and
+// stores it otherwise.
+inline bool cached_map(fp8vit_ctx* ctx, CUtensorMap* map, const void* base, int64_t rows,
+                       int64_t row_bytes, int box_rows) {
+    std::lock_guard<std::mutex> lock(ctx->tmap_mu);
+    for (fp8vit_tmap_entry& e : ctx->tmaps) {
+        if (e.valid && e.base == base && e.rows == rows && e.row_bytes == row_bytes &&
+            e.box_rows == box_rows) {
+            *map = e.map;
+            ++ctx->tmap_hits;
+            return true;
+        }
+    }
+    if (!encode_map(map, base, rows, row_bytes, box_rows)) return false;
+    fp8vit_tmap_entry& e = ctx->tmaps[ctx->tmap_next];
+    ctx->tmap_next = (ctx->tmap_next + 1) % kTmapCacheSize;
+    e.base = base;
+    e.rows = rows;
+    e.row_bytes = row_bytes;
+    e.box_rows = box_rows;
+    e.map = *map;
+    e.valid = true;
+    ++ctx->tmap_misses;
+    return true;
+}
+
 inline bool misaligned(const void* p, uintptr_t a) {
     return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0;
 }

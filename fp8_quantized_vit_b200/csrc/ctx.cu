@@ -54,6 +54,14 @@ fp8vit_status fp8vit_destroy(fp8vit_ctx* ctx) {
     return e == cudaSuccess ? FP8VIT_OK : FP8VIT_ECUDA;
 }
 
+fp8vit_status fp8vit_tmap_cache_stats(fp8vit_ctx* ctx, uint64_t* hits, uint64_t* misses) {
+    if (!ctx || !hits || !misses) return FP8VIT_EINVAL;
+    std::lock_guard<std::mutex> lock(ctx->tmap_mu);
+    *hits = ctx->tmap_hits;
+    *misses = ctx->tmap_misses;
+    return FP8VIT_OK;
+}
+
 fp8vit_status fp8vit_set_attn_p_terms(fp8vit_ctx* ctx, int32_t terms) {
     if (!ctx || (terms != 1 && terms != 2)) return FP8VIT_EINVAL;
     ctx->attn_p_terms = terms;

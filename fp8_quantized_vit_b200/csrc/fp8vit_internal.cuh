@@ -9,6 +9,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "fp8vit.h"
 
 // Device scratch owned by a context (one cudaMalloc in fp8vit_create).
@@ -23,12 +25,28 @@ struct fp8vit_scratch {
     uint32_t pad[21];      // to 128 bytes
 };
 
+// Tensor maps the attention launches encode, kept per context: a layer
+// reuses its buffers from call to call, so the maps of (base, shape, box)
+// repeat and need not be encoded again on every launch.
+struct fp8vit_tmap_entry {
+    const void* base;
+    int64_t rows, row_bytes;
+    int32_t box_rows;
+    bool valid;
+    CUtensorMap map;
+};
+constexpr int kTmapCacheSize = 12;
+
 struct fp8vit_ctx {
     int32_t device;
     int32_t num_sms;
     fp8vit_scratch* d_scratch;
     int32_t attn_p_terms;  // 2 = P as e4m3 hi + lo (default), 1 = single e4m3 term
     int64_t l2_bytes;      // the device's L2 size
+    std::mutex tmap_mu;    // guards the cache below (calls may come from several threads)
+    fp8vit_tmap_entry tmaps[kTmapCacheSize] = {};
+    int32_t tmap_next = 0;  // round-robin replacement
+    uint64_t tmap_hits = 0, tmap_misses = 0;
 };
 
 // Ring state layout (FP8VIT_RING_BYTES == 256).
@@ -141,6 +159,40 @@ __device__ __forceinline__ uint2 quant8_small(const uint4& x, uint64_t s2, uint6
         float qlo, qhi;
         f2_unpack(f2_fma(e, nr2, q0), qlo, qhi);
         c[i] = f32x2_to_e4m3x2(qlo, qhi);
+    }
+    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+// Per-tensor quantization arithmetic (vLLM docs "FP8 ViT Encoder Attention":
+// x8 = e4m3(fp32(x) / descale)), shared by the per-tensor quantizers and the
+// attention prologue that quantizes Q itself, so both produce the same bytes.
+
+// x / s rounded to nearest fp32, given r = RN(1/s) (s > 0, finite).
+// Markstein's correction (IBM J. Res. Dev. 34(1), 1990): with an exactly
+// rounded reciprocal, q0 = RN(x r) is within one ulp of x / s, the
+// remainder x - s q0 is exact in one FMA, and RN(q0 + rem r) is the
+// correctly rounded quotient -- the IEEE division the quantizers are defined
+// with, without a divide per element.  Quotients of magnitude >= 1024
+// saturate to +-448 in e4m3 whatever their last bits, so they skip the
+// correction (which would turn an overflowed q0 into NaN); the sign of a
+// zero quotient is the sign of x.  Checked bit for bit against IEEE division
+// on every finite BF16 value at 96 scales.
+__device__ __forceinline__ float div_by_scale(float x, float s, float r) {
+    const float q0 = __fmul_rn(x, r);
+    const float rem = __fmaf_rn(-q0, s, x);
+    const float q1 = __fmaf_rn(rem, r, q0);
+    return copysignf(fabsf(q0) < 1024.0f ? q1 : q0, x);
+}
+
+// 8 bf16 (one 16-byte vector) / scale -> 8 e4m3 codes (8 bytes); r = RN(1/s).
+__device__ __forceinline__ uint2 quant8(const uint4& x, float s, float r) {
+    uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t c[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float lo = div_by_scale(__uint_as_float(w[i] << 16), s, r);
+        float hi = div_by_scale(__uint_as_float(w[i] & 0xFFFF0000u), s, r);
+        c[i] = f32x2_to_e4m3x2(lo, hi);
     }
     return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }

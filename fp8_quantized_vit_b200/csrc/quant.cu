@@ -152,36 +152,6 @@ __global__ void ring_push_kernel(const float* __restrict__ amax3, fp8vit_ring* _
     ring_rule(ring, a, descale3);
 }
 
-// x / s rounded to nearest fp32, given r = RN(1/s) (s > 0, finite).
-// Markstein's correction (IBM J. Res. Dev. 34(1), 1990): with an exactly
-// rounded reciprocal, q0 = RN(x r) is within one ulp of x / s, the
-// remainder x - s q0 is exact in one FMA, and RN(q0 + rem r) is the
-// correctly rounded quotient -- the IEEE division the quantizers are defined
-// with, without a divide per element.  Quotients of magnitude >= 1024
-// saturate to +-448 in e4m3 whatever their last bits, so they skip the
-// correction (which would turn an overflowed q0 into NaN); the sign of a
-// zero quotient is the sign of x.  Checked bit for bit against IEEE division
-// on every finite BF16 value at 96 scales.
-__device__ __forceinline__ float div_by_scale(float x, float s, float r) {
-    const float q0 = __fmul_rn(x, r);
-    const float rem = __fmaf_rn(-q0, s, x);
-    const float q1 = __fmaf_rn(rem, r, q0);
-    return copysignf(fabsf(q0) < 1024.0f ? q1 : q0, x);
-}
-
-// 8 bf16 (one 16-byte vector) / scale -> 8 e4m3 codes (8 bytes); r = RN(1/s).
-__device__ __forceinline__ uint2 quant8(const uint4& x, float s, float r) {
-    uint32_t w[4] = {x.x, x.y, x.z, x.w};
-    uint32_t c[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float lo = div_by_scale(__uint_as_float(w[i] << 16), s, r);
-        float hi = div_by_scale(__uint_as_float(w[i] & 0xFFFF0000u), s, r);
-        c[i] = f32x2_to_e4m3x2(lo, hi);
-    }
-    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
-}
-
 // One tensor's grid-stride share: four 16-byte loads in flight per thread.
 __device__ __forceinline__ void quant_share(const uint4* __restrict__ p, uint2* __restrict__ o,
                                             int64_t n_elems, float s) {
@@ -210,7 +180,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quant3_kernel(
     const uint4* __restrict__ q, const uint4* __restrict__ k, const uint4* __restrict__ v,
     int64_t n_elems, const float* __restrict__ descale3, uint2* __restrict__ q8,
     uint2* __restrict__ k8, uint2* __restrict__ v8) {
-    quant_share(q, q8, n_elems, descale3[0]);
+    if (q8) quant_share(q, q8, n_elems, descale3[0]);  // null: Q is quantized by the attention
     quant_share(k, k8, n_elems, descale3[1]);
     quant_share(v, v8, n_elems, descale3[2]);
 }
@@ -282,22 +252,34 @@ __device__ __forceinline__ void quant3_share(const uint4* __restrict__ q,
     const float rq = __frcp_rn(s[0]), rk = __frcp_rn(s[1]), rv = __frcp_rn(s[2]);
     const int64_t nvec = n_elems >> 3;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const bool wq = q8 != nullptr;  // null: Q is quantized by the attention kernel
     int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    for (; i + stride < nvec; i += 2 * stride) {
-        const uint4 v0 = __ldcs(v + i), k0 = __ldcs(k + i), q0 = __ldcs(q + i);
-        const uint4 v1 = __ldcs(v + i + stride), k1 = __ldcs(k + i + stride);
-        const uint4 q1 = __ldcs(q + i + stride);
-        __stcs(v8 + i, quant8(v0, s[2], rv));
-        __stcs(k8 + i, quant8(k0, s[1], rk));
-        __stcs(q8 + i, quant8(q0, s[0], rq));
-        __stcs(v8 + i + stride, quant8(v1, s[2], rv));
-        __stcs(k8 + i + stride, quant8(k1, s[1], rk));
-        __stcs(q8 + i + stride, quant8(q1, s[0], rq));
+    if (wq) {
+        for (; i + stride < nvec; i += 2 * stride) {
+            const uint4 v0 = __ldcs(v + i), k0 = __ldcs(k + i), q0 = __ldcs(q + i);
+            const uint4 v1 = __ldcs(v + i + stride), k1 = __ldcs(k + i + stride);
+            const uint4 q1 = __ldcs(q + i + stride);
+            __stcs(v8 + i, quant8(v0, s[2], rv));
+            __stcs(k8 + i, quant8(k0, s[1], rk));
+            __stcs(q8 + i, quant8(q0, s[0], rq));
+            __stcs(v8 + i + stride, quant8(v1, s[2], rv));
+            __stcs(k8 + i + stride, quant8(k1, s[1], rk));
+            __stcs(q8 + i + stride, quant8(q1, s[0], rq));
+        }
+    } else {
+        for (; i + stride < nvec; i += 2 * stride) {
+            const uint4 v0 = __ldcs(v + i), k0 = __ldcs(k + i);
+            const uint4 v1 = __ldcs(v + i + stride), k1 = __ldcs(k + i + stride);
+            __stcs(v8 + i, quant8(v0, s[2], rv));
+            __stcs(k8 + i, quant8(k0, s[1], rk));
+            __stcs(v8 + i + stride, quant8(v1, s[2], rv));
+            __stcs(k8 + i + stride, quant8(k1, s[1], rk));
+        }
     }
     if (i < nvec) {
         __stcs(v8 + i, quant8(__ldcs(v + i), s[2], rv));
         __stcs(k8 + i, quant8(__ldcs(k + i), s[1], rk));
-        __stcs(q8 + i, quant8(__ldcs(q + i), s[0], rq));
+        if (wq) __stcs(q8 + i, quant8(__ldcs(q + i), s[0], rq));
     }
     const int tail = (int)(n_elems & 7);
     if (blockIdx.x == 0 && (int)threadIdx.x < tail) {
@@ -306,7 +288,7 @@ __device__ __forceinline__ void quant3_share(const uint4* __restrict__ q,
         uint2* dst[3] = {q8, k8, v8};
         const float r[3] = {rq, rk, rv};
 #pragma unroll
-        for (int t = 0; t < 3; ++t) {
+        for (int t = wq ? 0 : 1; t < 3; ++t) {
             const float y = div_by_scale(
                 bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(src[t])[e]), s[t], r[t]);
             reinterpret_cast<uint8_t*>(dst[t])[e] = (uint8_t)(f32x2_to_e4m3x2(y, 0.0f) & 0xFF);
@@ -505,7 +487,7 @@ fp8vit_status fp8_quantize_qkv_per_tensor(fp8vit_ctx* ctx, const uint16_t* d_q,
                                           const uint16_t* d_k, const uint16_t* d_v,
                                           int64_t n_elems, const float* d_descale3, uint8_t* d_q8,
                                           uint8_t* d_k8, uint8_t* d_v8, void* stream) {
-    if (!ctx || !d_q || !d_k || !d_v || !d_descale3 || !d_q8 || !d_k8 || !d_v8 || n_elems < 0)
+    if (!ctx || !d_q || !d_k || !d_v || !d_descale3 || !d_k8 || !d_v8 || n_elems < 0)
         return FP8VIT_EINVAL;
     if (misaligned(d_q, 16) || misaligned(d_k, 16) || misaligned(d_v, 16) ||
         misaligned(d_q8, 8) || misaligned(d_k8, 8) || misaligned(d_v8, 8) ||
@@ -526,7 +508,7 @@ fp8vit_status fp8_amax_ring_quantize_qkv(fp8vit_ctx* ctx, const uint16_t* d_q,
                                          int64_t n_elems, void* d_ring, float* d_descale3,
                                          uint8_t* d_q8, uint8_t* d_k8, uint8_t* d_v8,
                                          void* stream) {
-    if (!ctx || !d_q || !d_k || !d_v || !d_ring || !d_descale3 || !d_q8 || !d_k8 || !d_v8 ||
+    if (!ctx || !d_q || !d_k || !d_v || !d_ring || !d_descale3 || !d_k8 || !d_v8 ||
         n_elems < 0)
         return FP8VIT_EINVAL;
     if (misaligned(d_q, 16) || misaligned(d_k, 16) || misaligned(d_v, 16) ||

@@ -100,6 +100,13 @@ fp8vit_status fp8vit_inject_lost_arrival(fp8vit_ctx* ctx, void* stream);
  * fault is involved.  Synchronizes `stream`.  Not for production use. */
 fp8vit_status fp8vit_inject_attn_timeout(fp8vit_ctx* ctx, void* stream);
 
+/* The context keeps the TMA tensor maps its attention launches encode
+ * (keyed by base pointer, rows, row bytes and box rows; 12 entries, replaced
+ * round-robin), so a layer that reuses its buffers encodes them once.  The
+ * counts of launches' map lookups served from the cache and encoded anew.
+ * Host only. */
+fp8vit_status fp8vit_tmap_cache_stats(fp8vit_ctx* ctx, uint64_t* hits, uint64_t* misses);
+
 /* How many e4m3 terms the probabilities P of fp8_varlen_attn_fwd are kept in
  * for the PV product on this context (both run on the FP8 tensor cores):
  *   2 (the default): P = hi + lo, hi = e4m3(p), lo = e4m3(p - hi), two PV
@@ -193,7 +200,8 @@ fp8vit_status fp8_ring_read_amax(const void* d_ring, float out_amax3[3], void* s
  * fp32 division, round-to-nearest-even and saturation to +-448.  d_descale3:
  * float[3] (q, k, v) in device memory, e.g. from fp8_amax_ring_update or the
  * static scales.  Inputs BF16 [n_elems] 16-byte aligned; outputs e4m3 codes
- * [n_elems], 8-byte aligned. */
+ * [n_elems], 8-byte aligned.  d_q8 may be NULL: Q's codes are then not
+ * written (fp8_varlen_attn_fwd_qbf16 quantizes Q in its prologue). */
 fp8vit_status fp8_quantize_qkv_per_tensor(fp8vit_ctx* ctx, const uint16_t* d_q,
                                           const uint16_t* d_k, const uint16_t* d_v,
                                           int64_t n_elems, const float* d_descale3, uint8_t* d_q8,
@@ -212,7 +220,8 @@ fp8vit_status fp8_quantize_qkv_per_tensor(fp8vit_ctx* ctx, const uint16_t* d_q,
  * without the barrier.  A barrier wait that exceeds 2 s records
  * FP8VIT_ETIMEOUT (read it with fp8vit_check) and leaves the codes unwritten.
  * Alignment and ownership as the two calls; uses the context's scratch (one
- * stream per context at a time). */
+ * stream per context at a time).  d_q8 may be NULL (Q's amax still enters
+ * the ring; its codes are left to fp8_varlen_attn_fwd_qbf16). */
 fp8vit_status fp8_amax_ring_quantize_qkv(fp8vit_ctx* ctx, const uint16_t* d_q,
                                          const uint16_t* d_k, const uint16_t* d_v,
                                          int64_t n_elems, void* d_ring, float* d_descale3,
@@ -262,6 +271,26 @@ fp8vit_status bf16_varlen_attn_fwd(fp8vit_ctx* ctx, const uint16_t* d_q, const u
                                    int32_t num_seqs, int32_t max_seqlen, int64_t total_tokens,
                                    int32_t num_heads, int32_t head_dim, float softmax_scale,
                                    uint16_t* d_out, void* stream);
+
+/* fp8_varlen_attn_fwd with Q given as BF16 d_q [T, H, D] (16-byte aligned):
+ * the kernel's prologue divides each query row by *d_q_descale (IEEE fp32)
+ * and rounds it to e4m3 (RNE, satfinite) -- the same bytes
+ * fp8_quantize_qkv_per_tensor writes -- straight into its shared-memory Q
+ * tile, so Q's codes are neither written nor read through memory (vLLM docs
+ * "FP8 ViT Encoder Attention": Q/K/V are quantized right before attention;
+ * the small-image overhead of separate quantization passes).  Pair it with
+ * fp8_quantize_qkv_per_tensor or fp8_amax_ring_quantize_qkv called with
+ * d_q8 = NULL (K and V codes only; the amax still covers Q).  Other
+ * arguments, checks and faults as fp8_varlen_attn_fwd. */
+fp8vit_status fp8_varlen_attn_fwd_qbf16(fp8vit_ctx* ctx, const uint16_t* d_q,
+                                        const uint8_t* d_k8, const uint8_t* d_v8,
+                                        const float* d_q_descale, const float* d_k_descale,
+                                        const float* d_v_descale, const int32_t* d_cu_seqlens,
+                                        int32_t num_seqs, int32_t max_seqlen,
+                                        int64_t total_tokens, int32_t num_heads,
+                                        int32_t head_dim, float softmax_scale, void* d_out,
+                                        int32_t out_dtype, const float* d_output_scale,
+                                        void* stream);
 
 /* fp8_varlen_attn_fwd with the per-token-group quantizer fused into its
  * epilogue (vLLM issue "fused fp8 output for FlashAttention 3": the output

@@ -211,9 +211,10 @@ def test_host_argument_checks_need_no_gpu():
                                            dummy, dummy, None) == fv.EINVAL
     assert lib.fp8_amax_ring_update(fake_ctx, odd, dummy, dummy, 8, dummy, dummy,
                                     None) == fv.EINVAL
-    # fused amax + ring + quantize: null output, misaligned ring
-    assert lib.fp8_amax_ring_quantize_qkv(fake_ctx, dummy, dummy, dummy, 8, dummy, dummy, None,
-                                          dummy, dummy, None) == fv.EINVAL
+    # fused amax + ring + quantize: null K output (a null Q output is allowed:
+    # fp8_varlen_attn_fwd_qbf16 quantizes Q itself), misaligned ring
+    assert lib.fp8_amax_ring_quantize_qkv(fake_ctx, dummy, dummy, dummy, 8, dummy, dummy, dummy,
+                                          None, dummy, None) == fv.EINVAL
     assert lib.fp8_amax_ring_quantize_qkv(fake_ctx, dummy, dummy, dummy, 8, odd, dummy, dummy,
                                           dummy, dummy, None) == fv.EINVAL
 

@@ -474,3 +474,131 @@ def test_attention_timeout_is_reported_and_recovered():
     ref = oracle.attn_full(*codes, *desc, cu, H, D, np.float32(1.0 / math.sqrt(D)))
     assert_attn_close(got, ref, "after the injected timeout")
     c.close()
+
+
+def test_tensor_map_cache_reuses_maps_and_keeps_results():
+    """Calls on the same buffers take their three tensor maps from the
+    context's cache and give the same bytes as the first call; a buffer shape
+    seen for the first time is encoded anew."""
+    c = fv.Context()
+    lens, H, D = (300, 131), 2, 72
+    cu, codes, desc = _prepare(lens, H, D, seed=11)
+    T = codes[0].shape[0]
+    q8, k8, v8 = (_dev(x) for x in codes)
+    d = [torch.tensor([x], dtype=torch.float32, device="cuda") for x in desc]
+    cu_d = _dev(cu)
+    outs = []
+    stats = [c.tmap_cache_stats()]
+    for _ in range(3):
+        o = torch.empty((T, H, D), dtype=torch.bfloat16, device="cuda")
+        fv.fp8_varlen_attn_fwd(q8, k8, v8, d[0], d[1], d[2], cu_d, max(lens),
+                               np.float32(1.0 / math.sqrt(D)), o, ctx=c)
+        outs.append(o)
+        stats.append(c.tmap_cache_stats())
+    st, site = c.check()
+    assert st == fv.OK, (fv.status_string(st), site)
+    # a fresh context: the first call encodes its three maps, later calls hit
+    assert stats[1][1] - stats[0][1] == 3
+    for a, b in zip(stats[1:], stats[2:]):
+        assert b[0] - a[0] == 3 and b[1] == a[1]
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+    ref = oracle.attn_full(*codes, *desc, cu, H, D, np.float32(1.0 / math.sqrt(D)))
+    assert_attn_close(_gpu_bf16_to_f64(outs[0]), ref, "cached maps")
+
+
+@pytest.mark.parametrize("lens,H,D,mode", [((300, 1, 77), 2, 72, "static"),
+                                           ((513,), 2, 128, "dynamic"),
+                                           ((129, 255, 0, 64), 16, 72, "dynamic"),
+                                           ((1024,), 16, 72, "static"),
+                                           ((2304,), 16, 72, "dynamic")])
+def test_q_quantized_in_the_attention_prologue(ctx, lens, H, D, mode):
+    """fp8_varlen_attn_fwd_qbf16 (BF16 Q, quantized by the kernel's prologue)
+    gives the same bytes as fp8_varlen_attn_fwd on the oracle's Q codes, in
+    BF16 and FP8 output, so the prologue's Q codes equal the oracle's per-tensor
+    quantizer byte for byte; the output meets the gate against the oracle."""
+    cu = synth.cu_seqlens(lens)
+    T = int(cu[-1])
+    bf = [synth.bf16_tensor(synth.stream_key(77 + sum(lens), 0, t), T, H * D) for t in range(3)]
+    amax = [oracle.amax_bf16(x) for x in bf]
+    if mode == "static":
+        desc = [oracle.descale_from_amax(np.float32(1.5) * np.float32(a)) for a in amax]
+    else:
+        desc = list(oracle.Ring().update(amax))
+    codes = [oracle.quantize_per_tensor(x, d).reshape(T, H, D) for x, d in zip(bf, desc)]
+    q_bf = _dev(bf[0].view(np.int16), torch.bfloat16).reshape(T, H, D)
+    q8, k8, v8 = (_dev(c) for c in codes)
+    d = [torch.tensor([x], dtype=torch.float32, device="cuda") for x in desc]
+    cu_d = _dev(cu)
+    sm = np.float32(1.0 / math.sqrt(D))
+    osc = torch.tensor([0.02], dtype=torch.float32, device="cuda")
+    outs = {}
+    for name, fn, q in (("codes", fv.fp8_varlen_attn_fwd, q8),
+                        ("bf16q", fv.fp8_varlen_attn_fwd_qbf16, q_bf)):
+        o16 = torch.full((T, H, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+        o8 = torch.full((T, H, D), 0x7F, dtype=torch.uint8, device="cuda")
+        fn(q, k8, v8, d[0], d[1], d[2], cu_d, max(lens), sm, o16, ctx=ctx)
+        fn(q, k8, v8, d[0], d[1], d[2], cu_d, max(lens), sm, o8, output_scale=osc, ctx=ctx)
+        outs[name] = (o16, o8)
+    st, site = ctx.check()
+    assert st == fv.OK, (fv.status_string(st), site)
+    assert torch.equal(outs["codes"][0].view(torch.int16), outs["bf16q"][0].view(torch.int16))
+    assert torch.equal(outs["codes"][1], outs["bf16q"][1])
+    toks, hs = sample_pairs(cu, H, per_seg=64, seed=3)
+    ref = oracle.attn_pairs(*codes, *desc, cu, H, D, sm, toks, hs)
+    assert_attn_close(_gpu_bf16_to_f64(outs["bf16q"][0])[toks, hs], ref, (lens, H, D))
+
+
+@pytest.mark.parametrize("n", [1 << 20, 3 * 1152 * 41 + 5, 45_000_000])
+def test_quantizers_leave_q_codes_to_the_attention(ctx, n):
+    """With d_q8 NULL the static and the dynamic quantizers write K and V codes
+    equal to the oracle's and no Q codes; the dynamic ring still takes Q's
+    amax (descales bit-exact).  45 M elements per tensor exceed twice the L2
+    (the dynamic entry point then takes its two-kernel form)."""
+    x = [synth.bf16_tensor(synth.stream_key(31, n % 97, t), 1, n).ravel() for t in range(3)]
+    dev = [_dev(a.view(np.int16), torch.bfloat16) for a in x]
+    amax = [oracle.amax_bf16(a) for a in x]
+    want_desc = np.asarray(oracle.Ring().update(amax), np.float32)
+    k8, v8 = (torch.zeros(n, dtype=torch.uint8, device="cuda") for _ in range(2))
+    ring = fv.new_ring()
+    desc = torch.zeros(3, dtype=torch.float32, device="cuda")
+    fv.fp8_amax_ring_quantize_qkv(*dev, ring, desc, None, k8, v8, ctx=ctx)
+    st, site = ctx.check()
+    assert st == fv.OK, (fv.status_string(st), site)
+    assert (desc.cpu().numpy().view(np.uint32) == want_desc.view(np.uint32)).all()
+    for got, a, dsc in zip((k8, v8), x[1:], want_desc[1:]):
+        assert np.array_equal(got.cpu().numpy(), oracle.quantize_per_tensor(a, dsc))
+    k8.zero_()
+    v8.zero_()
+    fv.fp8_quantize_qkv_per_tensor(*dev, desc, None, k8, v8, ctx=ctx)
+    st, site = ctx.check()
+    assert st == fv.OK, (fv.status_string(st), site)
+    for got, a, dsc in zip((k8, v8), x[1:], want_desc[1:]):
+        assert np.array_equal(got.cpu().numpy(), oracle.quantize_per_tensor(a, dsc))
+
+
+@pytest.mark.parametrize("H,D", [(16, 72), (4, 128)])
+def test_layer_fold_q_gives_the_same_bytes(H, D):
+    """FP8EncoderAttention(fold_q=True) (Q quantized in the attention prologue)
+    returns the same bytes as the default layer: dynamic scales with BF16 and
+    FP8 output, static scales, and the group-quantized output."""
+    lens = (333, 190)
+    cu = synth.cu_seqlens(lens)
+    T = int(cu[-1])
+    bf = [synth.bf16_tensor(synth.stream_key(5, 1, t), T, H * D) for t in range(3)]
+    q, k, v = (_dev(x.view(np.int16), torch.bfloat16).reshape(T, H, D) for x in bf)
+    cu_d = _dev(cu)
+    osc = torch.tensor([0.02], dtype=torch.float32, device="cuda")
+    got = {}
+    for fold in (False, True):
+        dyn = fv.FP8EncoderAttention(H, D, fold_q=fold)
+        sta = fv.FP8EncoderAttention(H, D, static_amax=[30.0, 31.0, 32.0], fold_q=fold)
+        got[fold] = [dyn(q, k, v, cu_d, max(lens)).clone(),
+                     dyn(q, k, v, cu_d, max(lens), output_scale=osc).clone(),
+                     sta(q, k, v, cu_d, max(lens)).clone()]
+        xq, xs = dyn(q, k, v, cu_d, max(lens), group_quant=True)
+        got[fold] += [xq.clone(), xs.clone()]
+        st, site = dyn.ctx.check()
+        assert st == fv.OK, (fv.status_string(st), site)
+    for a, b in zip(got[False], got[True]):
+        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
