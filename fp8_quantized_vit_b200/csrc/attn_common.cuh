@@ -138,31 +138,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
 }
-// f32 pair -> f16x2 (lo in bits 0..15)
-__device__ __forceinline__ uint32_t cvt_f16x2(float lo, float hi) {
-    uint32_t d;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
-    return d;
-}
-// f16x2 -> two e4m3 codes in bits 0..15 (RNE, satfinite; bits 0..15 of the
-// source -> byte 0), returned zero-extended
-__device__ __forceinline__ uint32_t e4m3x2_of_f16x2(uint32_t h) {
-    uint16_t d;
-    asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(d) : "r"(h));
-    return d;
-}
-// two e4m3 codes (bits 0..15) -> f16x2 (exact)
-__device__ __forceinline__ uint32_t f16x2_of_e4m3x2(uint32_t e) {
-    uint32_t d;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"((uint16_t)e));
-    return d;
-}
-__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-
 // Row max of one S tile of NCH 32-key chunks held in registers; keys past the
 // segment end already hold -inf.
 template <int NCH>

@@ -299,3 +299,81 @@ def test_gpus_flag_launches_one_rank_per_gpu(monkeypatch):
     monkeypatch.setenv("WORLD_SIZE", "2")
     monkeypatch.setattr(_sys, "argv", ["bench.py", "--gpus", "4"])
     assert bench.main() == 2
+
+
+def test_workload_paths_run_each_configurations_own_step(monkeypatch):
+    """bench._Path, run on the CPU with stand-ins for the library calls:
+    a static workload with FP8 output calibrates its descales from the exact
+    amax with the margin and forms output_scale on the device (amax of the BF16
+    output, then the ring rule) before any step, then each step quantizes with
+    the static descales and runs the FP8-output attention with that scale; a
+    27-layer dynamic workload gives each layer its own ring and adds the group
+    quantizer."""
+    import inspect
+    import types
+
+    import numpy as np
+    import torch
+
+    import fp8_quantized_vit_b200 as fv
+
+    seen = []
+
+    def stand_in(name, effect=None):
+        sig = inspect.signature(getattr(fv, name))
+
+        def f(*a, **k):
+            sig.bind(*a, **k)
+            seen.append((name, a, k))
+            if effect:
+                effect(*a, **k)
+        return f
+
+    def amax3(q, k, v, out, ctx=None):
+        out.copy_(torch.tensor([3.0, 4.0, 5.0]))
+
+    def push(amax3, ring, desc3, stream=None):
+        desc3.copy_(amax3 / 448.0)
+
+    fake = types.SimpleNamespace(
+        OK=0, status_string=str,
+        fp8_amax3=stand_in("fp8_amax3", amax3),
+        fp8_descale_from_amax_margin=lambda a, m: float(np.float32(np.float32(m) * np.float32(a))
+                                                        / np.float32(448.0)),
+        fp8_ring_push=stand_in("fp8_ring_push", push),
+        new_ring=lambda dev=None: torch.zeros(64),
+        ring_init=stand_in("ring_init"),
+        fp8_quantize_qkv_per_tensor=stand_in("fp8_quantize_qkv_per_tensor"),
+        fp8_amax_ring_quantize_qkv=stand_in("fp8_amax_ring_quantize_qkv"),
+        fp8_varlen_attn_fwd=stand_in("fp8_varlen_attn_fwd"),
+        per_token_group_quant_fp8=stand_in("per_token_group_quant_fp8"))
+    ctx = types.SimpleNamespace(check=lambda: (0, 0))
+    T, H, D = 40, 2, 72
+    w = synth.Workload("3 tiny images", (10, 10, 20), H, D, "static", (1,), fp8_out=True)
+    inputs = [[torch.zeros((T, H, D), dtype=torch.bfloat16) for _ in range(3)]]
+    path = bench._Path(fake, ctx, w, inputs, "cpu")
+    names = [s[0] for s in seen]
+    assert names == ["fp8_amax3", "fp8_quantize_qkv_per_tensor", "fp8_varlen_attn_fwd",
+                     "fp8_amax3", "fp8_ring_push"]
+    assert torch.equal(path.desc, torch.tensor([1.5 * 3, 1.5 * 4, 1.5 * 5]) / 448.0)
+    assert abs(float(path.oscale) - 3.0 / 448.0) < 1e-9
+    seen.clear()
+    path.step(0)
+    assert [s[0] for s in seen] == ["fp8_quantize_qkv_per_tensor", "fp8_varlen_attn_fwd"]
+    attn = seen[1]
+    assert attn[1][9].dtype == torch.uint8 and attn[2]["output_scale"] is path.oscale
+    assert bench._launches_per_step(w, 126 << 20) == 2
+
+    w27 = synth.WORKLOADS["3x32400_d72"]
+    small = synth.Workload("27 tiny layers", (10, 10, 20), H, D, "dynamic", w27.seeds,
+                           group_quant=True, per_layer_rings=True)
+    inputs = [[torch.zeros((T, H, D), dtype=torch.bfloat16) for _ in range(3)] for _ in range(27)]
+    seen.clear()
+    path = bench._Path(fake, ctx, small, inputs, "cpu")
+    assert len(path.rings) == 27 and seen == []
+    for i in range(3):
+        path.step(i)
+    quant = [s for s in seen if s[0] == "fp8_amax_ring_quantize_qkv"]
+    assert [q[1][3] is path.rings[i] for i, q in enumerate(quant)] == [True] * 3
+    assert [s[0] for s in seen].count("per_token_group_quant_fp8") == 3
+    assert bench._launches_per_step(w27, 126 << 20) == 4  # two quantizer kernels above 2 x L2
