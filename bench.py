@@ -645,10 +645,13 @@ class _Path:
     descales, or dynamic rings) and the buffers, built once; step(i) runs
     forward i on the current stream through the library's entry points."""
 
-    def __init__(self, fv, ctx, w, inputs, dev):
+    def __init__(self, fv, ctx, w, inputs, dev, group_tail=False):
         import torch
         import synth
         self.fv, self.ctx, self.w = fv, ctx, w
+        # group_tail: the group quantizer runs as the attention launch's tail
+        # (fp8_varlen_attn_fwd_bf16_group_quant), timed inside the attention events
+        self.group_tail = group_tail and w.group_quant
         T, H, D = w.tokens, w.heads, w.head_dim
         self.inputs = inputs
         self.cu = torch.from_numpy(synth.cu_seqlens(w.seg_lens)).to(dev)
@@ -660,6 +663,8 @@ class _Path:
         self.xq = torch.empty((T, H * D), dtype=torch.uint8, device=dev)
         self.xs = torch.empty((T, H * D // 128), dtype=torch.float32, device=dev)
         self.desc = torch.zeros(3, dtype=torch.float32, device=dev)
+        self.counters = (fv.new_tile_counters(T, len(w.seg_lens), dev) if self.group_tail
+                         else None)
         self.oscale = None
         if w.mode == "static":
             # calibration (untimed): exact amax of forward 0 on the device,
@@ -706,13 +711,18 @@ class _Path:
         self._quantize(i)
         if ev_a is not None:
             ev_a.record(stream)
-        if w.fp8_out:
+        if self.group_tail:
+            d = self.desc
+            self.fv.fp8_varlen_attn_fwd_bf16_group_quant(
+                self.q8, self.k8, self.v8, d[0:1], d[1:2], d[2:3], self.cu, self.max_s,
+                w.softmax_scale, self.out, self.xq, self.xs, self.counters, ctx=self.ctx)
+        elif w.fp8_out:
             self._attend(self.out8, self.oscale)
         else:
             self._attend(self.out, None)
         if ev_b is not None:
             ev_b.record(stream)
-        if w.group_quant:
+        if w.group_quant and not self.group_tail:
             T, HD = w.tokens, w.heads * w.head_dim
             self.fv.per_token_group_quant_fp8(self.out.view(T, HD), 128, self.xq, self.xs,
                                               ctx=self.ctx)
@@ -766,6 +776,18 @@ def _config_records(fv, ctx, dev, peaks, stream, steps=5, warmup=3):
                "step_tflops": w.attn_flops() / (ms * 1e-3) / 1e12}
         if len(w.seg_lens) == 1:
             rec["torch_bf16_sdpa"] = _sdpa_comparator(w, inputs, dev)
+        if w.group_quant and D != 128:
+            # the same step with the group quantizer as the attention launch's
+            # tail: one launch instead of attention + per_token_group_quant_fp8
+            del path
+            path = _Path(fv, ctx, w, inputs, dev, group_tail=True)
+            ms_t, attn_t = _time_path(path, n_steps, min(warmup, n_steps), stream)
+            st, site = ctx.check()
+            if st != fv.OK:
+                raise RuntimeError(f"device fault in {name} (group tail): "
+                                   f"{fv.status_string(st)} site {site}")
+            rec["group_tail"] = {"ms_per_step": ms_t, "attn_plus_tail_ms": attn_t,
+                                 "step_speedup_vs_two_launches": ms / ms_t}
         recs[name] = rec
         del path, inputs
         torch.cuda.empty_cache()

@@ -8,7 +8,8 @@ or ``python -m fp8_quantized_vit_b200._build``); there is no fallback.
 Entry points (same names as the C ABI):
   fp8_amax_ring_update, fp8_amax_ring_update_noalloc, fp8_amax3, fp8_ring_push,
   fp8_quantize_qkv_per_tensor,
-  fp8_varlen_attn_fwd, per_token_group_quant_fp8, fp8_static_scales_load,
+  fp8_varlen_attn_fwd, fp8_varlen_attn_fwd_bf16_group_quant (with new_tile_counters),
+  per_token_group_quant_fp8, fp8_static_scales_load,
   fp8_static_scales_save, fp8_descale_from_amax, fp8_ring_read_amax, ring_init
 and ``FP8EncoderAttention``, which chains them for one attention layer
 (dynamic ring or static scales, BF16 or FP8 output; with a process group, the
@@ -58,6 +59,9 @@ _SIGNATURES = {
                                          _I32, _F32, _P, _I32, _P, _P]),
     "fp8_varlen_attn_fwd_group_quant": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I64,
                                                _I32, _I32, _F32, _P, _P, _P]),
+    "fp8_varlen_attn_fwd_bf16_group_quant": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32,
+                                                    _I64, _I32, _I32, _F32, _P, _P, _P, _P,
+                                                    _P]),
     "per_token_group_quant_fp8": (_I32, [_P, _P, _I64, _I64, _I32, _P, _P, _P]),
     "fp8_static_scales_load": (_I32, [ctypes.c_char_p, ctypes.c_char_p, _P]),
     "fp8_static_scales_save": (_I32, [ctypes.c_char_p, _I32, ctypes.POINTER(ctypes.c_char_p),
@@ -379,6 +383,48 @@ def fp8_varlen_attn_fwd_group_quant(q8, k8, v8, q_descale, k_descale, v_descale,
     return xq, scales
 
 
+def tile_counters_size(total_tokens: int, num_seqs: int) -> int:
+    """Entries of the per-query-tile arrival counters that
+    fp8_varlen_attn_fwd_bf16_group_quant needs."""
+    return (int(total_tokens) + 127) // 128 + int(num_seqs)
+
+
+def new_tile_counters(total_tokens: int, num_seqs: int, device=None) -> torch.Tensor:
+    """Zeroed counters (uint32 bits held in an int32 tensor); a completed call
+    leaves them zero, so one buffer serves every later call of at most this
+    size on the same stream."""
+    return torch.zeros(tile_counters_size(total_tokens, num_seqs), dtype=torch.int32,
+                       device=device or "cuda")
+
+
+def fp8_varlen_attn_fwd_bf16_group_quant(q8, k8, v8, q_descale, k_descale, v_descale,
+                                         cu_seqlens, max_seqlen, softmax_scale, out, xq, scales,
+                                         tile_counters, ctx=None, stream=None):
+    """Attention with BF16 output ``out`` [T, H, D] and, in the same launch,
+    its per-token groups of 128 quantized: xq e4m3 [T, H * D], scales fp32
+    [T, H * D / 128] (head_dim 72 or 128, H * D a multiple of 128); the same
+    bytes as fp8_varlen_attn_fwd followed by per_token_group_quant_fp8.
+    ``tile_counters``: see new_tile_counters."""
+    if q8.dim() != 3:
+        raise ValueError("q8 must be [T, H, D]")
+    T, H, D = q8.shape
+    if k8.shape != q8.shape or v8.shape != q8.shape or out.shape != q8.shape:
+        raise ValueError("q8, k8, v8 and out must have the same [T, H, D] shape")
+    if xq.numel() != T * H * D or scales.numel() != T * H * D // 128:
+        raise ValueError("xq must hold T * H * D codes and scales T * H * D / 128 floats")
+    if tile_counters.numel() < tile_counters_size(T, cu_seqlens.numel() - 1):
+        raise ValueError("tile_counters is too small (see tile_counters_size)")
+    _check(lib().fp8_varlen_attn_fwd_bf16_group_quant(
+        _ctx(ctx), _ptr(q8, _FP8, "q8"), _ptr(k8, _FP8, "k8"), _ptr(v8, _FP8, "v8"),
+        _ptr(q_descale, torch.float32, "q_descale"), _ptr(k_descale, torch.float32, "k_descale"),
+        _ptr(v_descale, torch.float32, "v_descale"), _ptr(cu_seqlens, torch.int32, "cu_seqlens"),
+        cu_seqlens.numel() - 1, int(max_seqlen), T, H, D, float(softmax_scale),
+        _ptr(out, torch.bfloat16, "out"), _ptr(xq, _FP8, "xq"),
+        _ptr(scales, torch.float32, "scales"), _ptr(tile_counters, torch.int32, "tile_counters"),
+        _stream(stream)), "fp8_varlen_attn_fwd_bf16_group_quant")
+    return out, xq, scales
+
+
 # ---- static scales ------------------------------------------------------------------
 
 def fp8_static_scales_load(path: str, layer: str) -> tuple[float, float, float]:
@@ -413,7 +459,8 @@ class FP8EncoderAttention:
     static descales), and runs
         [amax ring update] -> per-tensor quantize -> varlen FP8 attention
     (the first two as one cooperative launch on one GPU)
-        [-> per-token-group quantize of the output, fused at head_dim 128]
+        [-> per-token-group quantize of the output: fused at head_dim 128,
+            the attention launch's tail at head_dim 72 with group_tail]
     on the current stream.  The intermediate FP8 buffers and the output are the
     layer's own: they grow to the largest token count seen and are reused, so
     a call allocates nothing once that size has been met, and the tensors a
@@ -423,8 +470,12 @@ class FP8EncoderAttention:
 
     def __init__(self, num_heads: int, head_dim: int, softmax_scale: float | None = None,
                  static_amax=None, margin: float = 1.5, device=None, ctx: Context | None = None,
-                 process_group=None, fold_q: bool = False):
+                 process_group=None, fold_q: bool = False, group_tail: bool = False):
         self.H, self.D = num_heads, head_dim
+        # group_tail: where a 128-column group spans heads (head_dim 72), the
+        # group quantizer runs as the attention launch's tail
+        # (fp8_varlen_attn_fwd_bf16_group_quant) instead of a separate launch
+        self.group_tail = group_tail
         # fold_q: the attention kernel quantizes Q in its prologue
         # (fp8_varlen_attn_fwd_qbf16); the quantizer writes only K and V codes
         self.fold_q = fold_q
@@ -476,6 +527,14 @@ class FP8EncoderAttention:
                                    device=self.device)
         return {k: v[:T] for k, v in st.items() if k != "cap"}
 
+    def _counters(self, T: int, num_seqs: int) -> torch.Tensor:
+        need = tile_counters_size(T, num_seqs)
+        c = self._bufs.get("tile_counters")
+        if c is None or c.numel() < need:
+            c = new_tile_counters(T, num_seqs, self.device)
+            self._bufs["tile_counters"] = c
+        return c
+
     def forward(self, q, k, v, cu_seqlens, max_seqlen: int, output_scale=None, out=None,
                 group_quant: bool = False):
         """q, k, v: BF16 [T, H, D] on the device; cu_seqlens: int32 [B+1].
@@ -490,7 +549,7 @@ class FP8EncoderAttention:
         if group_quant and (self.H * self.D) % 128 != 0:
             raise ValueError("group_quant needs num_heads * head_dim to be a multiple of 128")
         b = self._buffers(T, output_scale is not None, group_quant)
-        fold = self.fold_q and not (group_quant and self.D == 128)
+        fold = self.fold_q and not (group_quant and (self.D == 128 or self.group_tail))
         q8 = None if fold else b["q8"]
         if self.ring is not None and self.process_group is not None:
             # this rank holds some of the batch's images: agree on the
@@ -511,7 +570,12 @@ class FP8EncoderAttention:
         if group_quant:
             hd = self.H * self.D
             xq, xs = b["xq"], b["xs"]
-            if self.D == 128:
+            if self.D != 128 and self.group_tail and not fold:
+                fp8_varlen_attn_fwd_bf16_group_quant(
+                    b["q8"], b["k8"], b["v8"], self.descale[0:1], self.descale[1:2],
+                    self.descale[2:3], cu_seqlens, max_seqlen, self.softmax_scale, b["out"], xq,
+                    xs, self._counters(T, cu_seqlens.numel() - 1), ctx=self.ctx)
+            elif self.D == 128:
                 fp8_varlen_attn_fwd_group_quant(b["q8"], b["k8"], b["v8"], self.descale[0:1],
                                                 self.descale[1:2], self.descale[2:3], cu_seqlens,
                                                 max_seqlen, self.softmax_scale, xq, xs,

@@ -276,6 +276,112 @@ __device__ __forceinline__ void tmem_st_p_any(uint32_t taddr, const uint32_t (&p
 }
 
 
+// Group tail of kOutBf16GroupQ (atrex-bench "#025 per_token_group_quant_fp8":
+// 128-wide groups of a token row, fp32 scale = amax / 448, codes of x / scale;
+// vLLM issue "fused fp8 output for FlashAttention 3": the o-proj input is
+// produced by the attention call).  When a 128-column group spans several
+// heads (head_dim 72: 16 heads are 9 groups) no single head CTA holds a whole
+// group, so each CTA stores its bf16 head slice as usual and then counts
+// itself in on its query tile; the last of the num_heads CTAs to arrive
+// quantizes the tile's token rows across all heads.  Nobody waits on another
+// CTA: the counter only elects the one that runs the tail, then resets it
+// for the next launch.  The rows come back (L2-hot) through bulk copies into
+// two staging buffers over the CTA's now idle Q/K/V shared memory; each half
+// warp takes one group, 8 values a lane, with the arithmetic of
+// group_quant_kernel (same helpers), so codes and scales equal those of
+// per_token_group_quant_fp8 over the stored bf16 output.
+template <class L>
+__device__ __noinline__ void group_tail(uint8_t* sm, uint32_t bar_a, uint32_t bar_b,
+                                        volatile uint32_t* last_flag,
+                                        volatile int32_t* abort_flag, uint32_t* tile_cnt,
+                                        int seg, int32_t seg_start, int32_t seg_len, int qt,
+                                        int ncol, int num_heads, const uint16_t* out,
+                                        uint8_t* xq, float* gscales, fp8vit_scratch* scr) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        // Every CTA of the tile arrives exactly once per launch (the error
+        // paths too), so the count returns to zero with the last arrival.
+        // Tiles are numbered seg_start / 128 + qt + seg: distinct across
+        // segments because cu_seqlens is a cumulative sum.
+        uint32_t* cnt = tile_cnt + ((seg_start >> 7) + qt + seg);
+        __threadfence();  // this CTA's bf16 stores (ordered by the barrier above)
+        const bool last = atomicAdd(cnt, 1u) == (uint32_t)num_heads - 1;
+        if (last) {
+            atomicExch(cnt, 0u);
+            __threadfence();  // the other CTAs' stores, before the copies below
+            fence_proxy_async_global();
+        }
+        *last_flag = last && *abort_flag == 0;
+    }
+    __syncthreads();
+    if (!*last_flag) return;
+
+    const int q0 = qt * kBM;
+    const int rows = min(kBM, seg_len - q0);
+    const int64_t tok0 = (int64_t)seg_start + q0;
+    const uint32_t row_bytes = (uint32_t)ncol * 2;
+    const int ngr = ncol >> 7;  // groups per token row
+    // Rows per staging buffer: half of the Q/K/V area each (the host checks
+    // that one row fits).
+    const int R = min(rows, (int)((L::BAR / 2) / row_bytes));
+    const int nch = (rows + R - 1) / R;
+    const uint32_t buf0 = smem_u32(sm), buf1 = smem_u32(sm) + (uint32_t)(L::BAR / 2);
+    auto issue = [&](int c) {
+        const int r0 = c * R, nr = min(R, rows - r0);
+        const uint32_t bar = (c & 1) ? bar_b : bar_a;
+        mbar_arrive_expect_tx(bar, nr * row_bytes);
+        bulk_load((c & 1) ? buf1 : buf0, out + (tok0 + r0) * ncol, nr * row_bytes, bar);
+    };
+    if (tid == 0) {
+        issue(0);
+        if (nch > 1) issue(1);
+    }
+    const int half = lane >> 4, l16 = lane & 15;
+    const int nwarps = blockDim.x >> 5;
+    int c = 0;
+    bool ok = true;
+    for (; c < nch; ++c) {
+        ok = mbar_wait_bounded((c & 1) ? bar_b : bar_a, (c >> 1) & 1, abort_flag, scr,
+                               SITE_ATTN_WAIT_GROUP, kTimeoutNs);
+        if (!__syncthreads_and(ok)) break;
+        const int r0 = c * R, nr = min(R, rows - r0);
+        const uint8_t* buf = sm + ((c & 1) ? L::BAR / 2 : 0);
+        const int ngroups = nr * ngr;
+        for (int p = warp; 2 * p < ngroups; p += nwarps) {
+            const int g = 2 * p + half;
+            const bool active = g < ngroups;
+            const int r = active ? g / ngr : 0, cg = active ? g - r * ngr : 0;
+            const uint4 x = active ? *reinterpret_cast<const uint4*>(buf + r * row_bytes + cg * 256 +
+                                                                     l16 * 16)
+                                   : make_uint4(0, 0, 0, 0);
+            uint32_t a = __vmaxu2(__vmaxu2(x.x & 0x7FFF7FFFu, x.y & 0x7FFF7FFFu),
+                                  __vmaxu2(x.z & 0x7FFF7FFFu, x.w & 0x7FFF7FFFu));
+            a = max(a & 0xFFFFu, a >> 16);
+#pragma unroll
+            for (int off = 8; off > 0; off >>= 1) a = max(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+            const float sc = group_scale_of_amax(bf16_bits_to_f32(a));
+            const float nr2f = -__frcp_rn(sc);
+            const uint2 q = quant8_small(x, f2_pack(sc, sc), f2_pack(nr2f, nr2f));
+            if (active) {
+                const int64_t tok = tok0 + r0 + r;
+                *reinterpret_cast<uint2*>(xq + tok * ncol + cg * 128 + l16 * 8) = q;
+                if (l16 == 0) gscales[tok * ngr + cg] = sc;
+            }
+        }
+        __syncthreads();  // buffer (c & 1) read by all before it is refilled
+        if (tid == 0 && c + 2 < nch) {
+            fence_proxy_async_smem();
+            issue(c + 2);
+        }
+    }
+    if (c < nch && tid == 0) {
+        // Gave up: let the copies still in flight land before the CTA exits.
+        for (int k = c; k < min(c + 2, nch); ++k)
+            mbar_wait_drain((k & 1) ? bar_b : bar_a, (k >> 1) & 1, scr);
+    }
+}
+
+
 // OUT selects the epilogue at compile time; PLO keeps P as two e4m3 terms
 // (hi + lo, two PV MMAs) or, when false, as one.  BF: the inputs are BF16
 // (no descales) and both products run as kind::f16 MMAs with P in BF16.
@@ -290,8 +396,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                     const int32_t* __restrict__ cu, int32_t max_seqlen, int64_t total_tokens,
                     int32_t num_heads, float sm_scale, void* __restrict__ out,
                     const float* __restrict__ out_scale_p, float* __restrict__ gscales,
-                    fp8vit_scratch* __restrict__ scr, const uint16_t* __restrict__ qbf) {
+                    fp8vit_scratch* __restrict__ scr, const uint16_t* __restrict__ qbf,
+                    uint8_t* __restrict__ xq, uint32_t* __restrict__ tile_cnt) {
     static_assert(OUT != kOutGroupQ || D == 128, "a 128-wide group is one head at head_dim 128");
+    static_assert(!BF || OUT != kOutBf16GroupQ, "the group tail runs on the FP8 path");
     static_assert(!BF || OUT == kOutBf16, "bf16 inputs: bf16 output");
     static_assert(!(BF && QB), "BF16 Q is quantized only on the FP8 path");
     using C = CfgOf<D, BF>;
@@ -340,6 +448,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     auto b_kv_empty = [&](int s) { return bar0 + 8 * (9 + NS + s); };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::BAR + 8 * (9 + 2 * NS));
     volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
+    // Group tail (kOutBf16GroupQ): two staging-buffer barriers and the
+    // "last CTA of the tile" word after the TMEM slot and the abort flag.
+    auto b_grp = [&](int b) { return bar0 + 8 * (10 + 2 * NS + b); };
+    volatile uint32_t* last_flag = reinterpret_cast<volatile uint32_t*>(sm + L::BAR + 8 * (12 + 2 * NS));
+    static_assert(8 * (12 + 2 * NS) + 4 <= L::TOTAL - L::BAR, "barrier area");
 
     if (threadIdx.x == 0) {
         mbar_init(b_q_full, 1);
@@ -356,6 +469,10 @@ __global__ void __launch_bounds__(kThreads, 2)
             mbar_init(b_kv_empty(s), 1);
         }
         *abort_flag = 0;
+        if constexpr (OUT == kOutBf16GroupQ) {
+            mbar_init(b_grp(0), 1);
+            mbar_init(b_grp(1), 1);
+        }
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -743,6 +860,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+    if constexpr (OUT == kOutBf16GroupQ)
+        group_tail<L>(sm, b_grp(0), b_grp(1), last_flag, abort_flag, tile_cnt, seg, seg_start,
+                      seg_len, qt, num_heads * D, num_heads, reinterpret_cast<const uint16_t*>(out),
+                      xq, gscales, scr);
 }
 
 
@@ -753,7 +874,8 @@ fp8vit_status launch(fp8vit_ctx* ctx, const uint8_t* q8, const uint8_t* k8, cons
                      const float* dq, const float* dk, const float* dv, const int32_t* cu,
                      int32_t num_seqs, int32_t max_seqlen, int64_t T, int32_t H, float sm_scale,
                      void* out, const float* out_scale, float* gscales, cudaStream_t st,
-                     const uint16_t* qbf = nullptr) {
+                     const uint16_t* qbf = nullptr, uint8_t* xq = nullptr,
+                     uint32_t* tile_cnt = nullptr) {
     CUtensorMap mq, mk, mv;
     const int64_t row_bytes = (int64_t)H * D;
     if (!cached_map(ctx, &mk, k8, T, row_bytes, Cfg<D>::BN) ||
@@ -766,9 +888,11 @@ fp8vit_status launch(fp8vit_ctx* ctx, const uint8_t* q8, const uint8_t* k8, cons
     static std::atomic<uint64_t> attr_set[4];
     const bool two_terms = ctx->attn_p_terms != 1;
     const int inst = (two_terms ? 1 : 0) + (qbf ? 2 : 0);
-    auto kern = qbf ? (two_terms ? attn_fwd_kernel<D, OUT, true, false, true>
-                                 : attn_fwd_kernel<D, OUT, false, false, true>)
-                    : (two_terms ? attn_fwd_kernel<D, OUT, true> : attn_fwd_kernel<D, OUT, false>);
+    auto kern = two_terms ? attn_fwd_kernel<D, OUT, true> : attn_fwd_kernel<D, OUT, false>;
+    if constexpr (OUT != kOutBf16GroupQ)  // the group tail has no BF16-Q instance
+        if (qbf)
+            kern = two_terms ? attn_fwd_kernel<D, OUT, true, false, true>
+                             : attn_fwd_kernel<D, OUT, false, false, true>;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FP8VIT_ECUDA;
     const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
@@ -781,7 +905,7 @@ fp8vit_status launch(fp8vit_ctx* ctx, const uint8_t* q8, const uint8_t* k8, cons
     dim3 grid((unsigned)((max_seqlen + kBM - 1) / kBM), (unsigned)H, (unsigned)num_seqs);
     kern<<<grid, kThreads, Smem<D>::ALLOC, st>>>(mq, mk, mv, dq, dk, dv, cu, max_seqlen, T, H,
                                                  sm_scale, out, out_scale, gscales,
-                                                 ctx->d_scratch, qbf);
+                                                 ctx->d_scratch, qbf, xq, tile_cnt);
     return cudaGetLastError() == cudaSuccess ? FP8VIT_OK : FP8VIT_ECUDA;
 }
 
@@ -811,7 +935,7 @@ fp8vit_status launch_bf16(fp8vit_ctx* ctx, const uint16_t* q, const uint16_t* k,
     dim3 grid((unsigned)((max_seqlen + kBM - 1) / kBM), (unsigned)H, (unsigned)num_seqs);
     kern<<<grid, kThreads, L::ALLOC, st>>>(mq, mk, mv, nullptr, nullptr, nullptr, cu, max_seqlen, T,
                                            H, sm_scale, out, nullptr, nullptr, ctx->d_scratch,
-                                           nullptr);
+                                           nullptr, nullptr, nullptr);
     return cudaGetLastError() == cudaSuccess ? FP8VIT_OK : FP8VIT_ECUDA;
 }
 
@@ -929,6 +1053,42 @@ extern "C" fp8vit_status fp8_varlen_attn_fwd_group_quant(
                                    d_cu_seqlens, num_seqs, max_seqlen, total_tokens, num_heads,
                                    softmax_scale, d_xq, nullptr, d_scales,
                                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" fp8vit_status fp8_varlen_attn_fwd_bf16_group_quant(
+    fp8vit_ctx* ctx, const uint8_t* d_q8, const uint8_t* d_k8, const uint8_t* d_v8,
+    const float* d_q_descale, const float* d_k_descale, const float* d_v_descale,
+    const int32_t* d_cu_seqlens, int32_t num_seqs, int32_t max_seqlen, int64_t total_tokens,
+    int32_t num_heads, int32_t head_dim, float softmax_scale, uint16_t* d_out, uint8_t* d_xq,
+    float* d_scales, uint32_t* d_tile_counters, void* stream) {
+    if (!ctx || !d_q8 || !d_k8 || !d_v8 || !d_q_descale || !d_k_descale || !d_v_descale ||
+        !d_cu_seqlens || !d_out || !d_xq || !d_scales || !d_tile_counters)
+        return FP8VIT_EINVAL;
+    if (num_seqs < 0 || max_seqlen < 0 || total_tokens < 0 || total_tokens > INT32_MAX ||
+        num_heads < 1)
+        return FP8VIT_EINVAL;
+    if (!(softmax_scale > 0.0f) || !isfinite(softmax_scale)) return FP8VIT_EINVAL;
+    if (head_dim != 72 && head_dim != 128) return FP8VIT_EUNSUPPORTED;
+    if (((int64_t)num_heads * head_dim) % 128 != 0) return FP8VIT_EINVAL;
+    if (misaligned(d_q8, 16) || misaligned(d_k8, 16) || misaligned(d_v8, 16) ||
+        misaligned(d_out, 16) || misaligned(d_xq, 16) || misaligned(d_scales, 4) ||
+        misaligned(d_tile_counters, 4) || misaligned(d_cu_seqlens, 4))
+        return FP8VIT_EINVAL;
+    if (num_heads > 65535 || num_seqs > 65535) return FP8VIT_EUNSUPPORTED;
+    // Two staging buffers of at least one token row each in the Q/K/V area.
+    const int64_t row_bytes = (int64_t)num_heads * head_dim * 2;
+    if (2 * row_bytes > (head_dim == 72 ? Smem<72>::BAR : Smem<128>::BAR)) return FP8VIT_EUNSUPPORTED;
+    if (num_seqs == 0 || max_seqlen == 0 || total_tokens == 0) return FP8VIT_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (head_dim == 72)
+        return launch<72, kOutBf16GroupQ>(ctx, d_q8, d_k8, d_v8, d_q_descale, d_k_descale,
+                                          d_v_descale, d_cu_seqlens, num_seqs, max_seqlen,
+                                          total_tokens, num_heads, softmax_scale, d_out, nullptr,
+                                          d_scales, st, nullptr, d_xq, d_tile_counters);
+    return launch<128, kOutBf16GroupQ>(ctx, d_q8, d_k8, d_v8, d_q_descale, d_k_descale,
+                                       d_v_descale, d_cu_seqlens, num_seqs, max_seqlen,
+                                       total_tokens, num_heads, softmax_scale, d_out, nullptr,
+                                       d_scales, st, nullptr, d_xq, d_tile_counters);
 }
 
 extern "C" fp8vit_status bf16_varlen_attn_fwd(fp8vit_ctx* ctx, const uint16_t* d_q,

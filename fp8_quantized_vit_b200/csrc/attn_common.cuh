@@ -180,6 +180,9 @@ enum : int {
     kOutE4m3 = 1,     // e4m3(o / output_scale)
     kOutGroupQ = 2,   // the bf16 o of each head quantized as one 128-wide group:
                       // e4m3 codes + one fp32 scale per (token, head); head_dim 128
+    kOutBf16GroupQ = 3,  // o as bf16, then the last of a query tile's head CTAs
+                         // quantizes the tile's token rows (all heads) in 128-wide
+                         // groups: any head_dim with num_heads * head_dim % 128 == 0
 };
 
 // Host: a 2-D uint8 tensor map over a [rows, row_bytes] matrix with

@@ -298,8 +298,8 @@ fp8vit_status fp8_varlen_attn_fwd_qbf16(fp8vit_ctx* ctx, const uint16_t* d_q,
  * per_token_group_quant_fp8": group 128, fp32 scales, the o-proj input).
  * head_dim must be 128, so that each 128-column group of a token row of
  * [total_tokens, num_heads * 128] is exactly one head (head_dim 72 groups
- * straddle heads: FP8VIT_EUNSUPPORTED; use fp8_varlen_attn_fwd plus
- * per_token_group_quant_fp8).  The attention output is rounded to BF16 as
+ * straddle heads: FP8VIT_EUNSUPPORTED; use
+ * fp8_varlen_attn_fwd_bf16_group_quant).  The attention output is rounded to BF16 as
  * fp8_varlen_attn_fwd's out_dtype 0 stores it, then quantized exactly as
  * per_token_group_quant_fp8(group = 128) does: the bytes of d_xq and the bits
  * of d_scales equal those two calls' results, and no BF16 output is written.
@@ -312,6 +312,40 @@ fp8vit_status fp8_varlen_attn_fwd_group_quant(
     const int32_t* d_cu_seqlens, int32_t num_seqs, int32_t max_seqlen, int64_t total_tokens,
     int32_t num_heads, int32_t head_dim, float softmax_scale, uint8_t* d_xq, float* d_scales,
     void* stream);
+
+/* fp8_varlen_attn_fwd (BF16 output) and per_token_group_quant_fp8(group =
+ * 128) of that output in one launch, for any supported head_dim (72 or 128)
+ * with num_heads * head_dim a multiple of 128 (vLLM issue "fused fp8 output
+ * for FlashAttention 3": the output quantization moves into the attention
+ * call; atrex-bench "#025 per_token_group_quant_fp8": 128-wide groups of a
+ * token row, fp32 scales, the o-proj input).  At head_dim 72 a group spans
+ * two or three heads, so no single head's CTA holds a group: every CTA
+ * stores its BF16 head slice to d_out, and the last of the num_heads CTAs of
+ * a query tile to finish quantizes that tile's token rows over all heads
+ * (an arrival counter per tile elects it; no CTA waits for another).
+ * d_out: BF16 [total_tokens, num_heads * head_dim], 16-byte aligned; holds
+ *   fp8_varlen_attn_fwd's out_dtype 0 result on return.
+ * d_xq: e4m3 [total_tokens, num_heads * head_dim], 16-byte aligned, and
+ * d_scales: fp32 [total_tokens, num_heads * head_dim / 128], 4-byte aligned:
+ *   byte for byte and bit for bit what per_token_group_quant_fp8(d_out, 128)
+ *   writes.
+ * d_tile_counters: uint32 workspace of at least
+ *   (total_tokens + 127) / 128 + num_seqs entries, all zero before the first
+ *   call; a completed call leaves them zero again (the caller zeroes it once,
+ *   e.g. with cudaMemsetAsync, and reuses it).  Calls that share a counter
+ *   buffer must not run concurrently.
+ * Returns FP8VIT_EINVAL when num_heads * head_dim is not a multiple of 128
+ * or a pointer is null or misaligned, FP8VIT_EUNSUPPORTED for another
+ * head_dim or for token rows too long for two staging rows in the
+ * kernel's Q/K/V shared memory (above 160 heads at head_dim 128, 352 at 72).  A timeout of the
+ * tail's staging copies records FP8VIT_ETIMEOUT at site 120.  Other
+ * arguments, checks and faults as fp8_varlen_attn_fwd. */
+fp8vit_status fp8_varlen_attn_fwd_bf16_group_quant(
+    fp8vit_ctx* ctx, const uint8_t* d_q8, const uint8_t* d_k8, const uint8_t* d_v8,
+    const float* d_q_descale, const float* d_k_descale, const float* d_v_descale,
+    const int32_t* d_cu_seqlens, int32_t num_seqs, int32_t max_seqlen, int64_t total_tokens,
+    int32_t num_heads, int32_t head_dim, float softmax_scale, uint16_t* d_out, uint8_t* d_xq,
+    float* d_scales, uint32_t* d_tile_counters, void* stream);
 
 /* ---- per-token-group quantizer (atrex-bench "#025 per_token_group_quant_fp8",
  *      Reference Implementation) --------------------------------------------- */

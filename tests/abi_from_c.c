@@ -49,6 +49,9 @@ int main(int argc, char** argv) {
                                   128, 0.088f, NULL, 0, NULL, NULL) == FP8VIT_EINVAL);
     CHECK(16, per_token_group_quant_fp8(NULL, NULL, 1, 128, 128, NULL, NULL, NULL) ==
                   FP8VIT_EINVAL);
+    CHECK(17, fp8_varlen_attn_fwd_bf16_group_quant(NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL,
+                                                   1, 64, 64, 16, 72, 0.118f, NULL, NULL, NULL,
+                                                   NULL, NULL) == FP8VIT_EINVAL);
     printf("ok\n");
     return 0;
 }

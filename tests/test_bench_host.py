@@ -346,7 +346,10 @@ def test_workload_paths_run_each_configurations_own_step(monkeypatch):
         fp8_quantize_qkv_per_tensor=stand_in("fp8_quantize_qkv_per_tensor"),
         fp8_amax_ring_quantize_qkv=stand_in("fp8_amax_ring_quantize_qkv"),
         fp8_varlen_attn_fwd=stand_in("fp8_varlen_attn_fwd"),
-        per_token_group_quant_fp8=stand_in("per_token_group_quant_fp8"))
+        per_token_group_quant_fp8=stand_in("per_token_group_quant_fp8"),
+        fp8_varlen_attn_fwd_bf16_group_quant=stand_in("fp8_varlen_attn_fwd_bf16_group_quant"),
+        new_tile_counters=lambda t, n, dev=None: torch.zeros(fv.tile_counters_size(t, n),
+                                                             dtype=torch.int32))
     ctx = types.SimpleNamespace(check=lambda: (0, 0))
     T, H, D = 40, 2, 72
     w = synth.Workload("3 tiny images", (10, 10, 20), H, D, "static", (1,), fp8_out=True)
@@ -377,3 +380,10 @@ def test_workload_paths_run_each_configurations_own_step(monkeypatch):
     assert [q[1][3] is path.rings[i] for i, q in enumerate(quant)] == [True] * 3
     assert [s[0] for s in seen].count("per_token_group_quant_fp8") == 3
     assert bench._launches_per_step(w27, 126 << 20) == 4  # two quantizer kernels above 2 x L2
+    # the same workload with the group quantizer as the attention launch's tail
+    seen.clear()
+    path = bench._Path(fake, ctx, small, inputs, "cpu", group_tail=True)
+    path.step(0)
+    assert [s[0] for s in seen] == ["fp8_amax_ring_quantize_qkv",
+                                    "fp8_varlen_attn_fwd_bf16_group_quant"]
+    assert seen[1][1][12] is path.counters and path.counters.numel() == (T + 127) // 128 + 3

@@ -387,17 +387,19 @@ def test_head_counts_and_slack_max_seqlen(ctx, lens, H, D, max_seqlen):
     assert_attn_close(got, ref, (lens, H, D, max_seqlen))
 
 
-@pytest.mark.parametrize("lens,H,D", [((333, 190), 4, 128), ((333, 190), 16, 72)])
-def test_layer_group_quant_output(lens, H, D):
+@pytest.mark.parametrize("lens,H,D,tail", [((333, 190), 4, 128, False), ((333, 190), 16, 72, False),
+                                           ((333, 190), 16, 72, True)])
+def test_layer_group_quant_output(lens, H, D, tail):
     """FP8EncoderAttention(group_quant=True) returns the o-proj input: the
     codes and scales of per_token_group_quant_fp8 applied to the layer's own
-    BF16 output (fused epilogue at head_dim 128, two calls at 72), bit for
-    bit, on two layers fed the same inputs."""
+    BF16 output (fused epilogue at head_dim 128; at 72 two calls, or the
+    attention launch's group tail), bit for bit, on two layers fed the same
+    inputs."""
     cu = synth.cu_seqlens(lens)
     T = int(cu[-1])
     bf = [synth.bf16_tensor(synth.stream_key(88, 0, t), T, H * D) for t in range(3)]
     dev = [_dev(x.view(np.int16)).view(torch.bfloat16).reshape(T, H, D) for x in bf]
-    a = fv.FP8EncoderAttention(H, D)
+    a = fv.FP8EncoderAttention(H, D, group_tail=tail)
     b = fv.FP8EncoderAttention(H, D)
     xq, xs = a(*dev, _dev(cu), max(lens), group_quant=True)
     o = b(*dev, _dev(cu), max(lens))
@@ -602,3 +604,85 @@ def test_layer_fold_q_gives_the_same_bytes(H, D):
         assert st == fv.OK, (fv.status_string(st), site)
     for a, b in zip(got[False], got[True]):
         assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+
+
+def _group_tail_call(ctx, cu, codes, desc, H, D, max_seqlen, sm, counters):
+    T = codes[0].shape[0]
+    q8, k8, v8 = (_dev(c) for c in codes)
+    d = [torch.tensor([x], dtype=torch.float32, device="cuda") for x in desc]
+    out = torch.full((T, H, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    xq = torch.full((T, H * D), 0x7F, dtype=torch.uint8, device="cuda")
+    xs = torch.full((T, H * D // 128), float("nan"), dtype=torch.float32, device="cuda")
+    fv.fp8_varlen_attn_fwd_bf16_group_quant(q8, k8, v8, d[0], d[1], d[2], _dev(cu), max_seqlen,
+                                            sm, out, xq, xs, counters, ctx=ctx)
+    st, site = ctx.check()
+    assert st == fv.OK, (fv.status_string(st), site)
+    return out, xq, xs
+
+
+def _oracle_group_quant_of(out: torch.Tensor):
+    T = out.shape[0]
+    return oracle.group_quant(out.view(torch.int16).cpu().numpy().view(np.uint16).reshape(T, -1),
+                              128)
+
+
+@pytest.mark.parametrize("lens,H,D,max_seqlen", [
+    ((513, 129, 0, 300, 1), 16, 72, 513),  # several tiles, ragged tails, empty and 1-token images
+    ((256, 5), 32, 72, 300),               # 12 staging chunks per tile; slack max_seqlen
+    ((200, 77), 2, 128, 200),              # head_dim 128: one group per head
+    ((1,), 16, 72, 1),
+])
+def test_group_quant_tail(ctx, lens, H, D, max_seqlen):
+    """fp8_varlen_attn_fwd_bf16_group_quant: its BF16 output is
+    fp8_varlen_attn_fwd's, byte for byte (and within the gate of the fp64
+    oracle attention); its codes and scales are the oracle group quantizer's
+    (group 128, groups spanning heads at head_dim 72) applied to that output,
+    byte for byte and bit for bit; the tile counters are zero again afterwards,
+    and a second call on the same counters repeats every byte."""
+    cu, codes, desc = _prepare(lens, H, D, seed=sum(lens) + 7 * H + D)
+    sm = np.float32(1.0 / math.sqrt(D))
+    T = codes[0].shape[0]
+    ref_out = _run_gpu(ctx, cu, codes, desc, H, D, max_seqlen)
+    counters = fv.new_tile_counters(T, len(lens))
+    out, xq, xs = _group_tail_call(ctx, cu, codes, desc, H, D, max_seqlen, sm, counters)
+    assert torch.equal(out.view(torch.int16), ref_out.view(torch.int16))
+    assert_attn_close(_gpu_bf16_to_f64(out), oracle.attn_full(*codes, *desc, cu, H, D, sm),
+                      (lens, H, D))
+    want_q, want_s = _oracle_group_quant_of(out)
+    assert np.array_equal(xq.cpu().numpy(), want_q)
+    assert np.array_equal(xs.cpu().numpy().view(np.uint32), want_s.view(np.uint32))
+    assert int(counters.abs().sum()) == 0
+    out2, xq2, xs2 = _group_tail_call(ctx, cu, codes, desc, H, D, max_seqlen, sm, counters)
+    assert torch.equal(out2.view(torch.int16), out.view(torch.int16))
+    assert torch.equal(xq2, xq) and torch.equal(xs2.view(torch.int32), xs.view(torch.int32))
+    assert int(counters.abs().sum()) == 0
+
+
+def test_group_quant_tail_27_layer_workload_size(ctx):
+    """The group tail at its own workload's size (3 images of 32400 tokens, 16
+    heads of 72, [97200, 1152]): BF16 output equal to fp8_varlen_attn_fwd's and
+    codes/scales equal to per_token_group_quant_fp8 of it over the whole
+    tensor, and equal to the oracle group quantizer on sampled token rows
+    (every tile edge of every image)."""
+    w = synth.WORKLOADS["3x32400_d72"]
+    H, D = w.heads, w.head_dim
+    q, k, v = w.qkv(0)
+    desc = list(oracle.Ring().update([oracle.amax_bf16(x) for x in (q, k, v)]))
+    codes = [oracle.quantize_per_tensor(x, d).reshape(w.tokens, H, D)
+             for x, d in zip((q, k, v), desc)]
+    cu = synth.cu_seqlens(w.seg_lens)
+    T, ms = w.tokens, max(w.seg_lens)
+    ref_out = _run_gpu(ctx, cu, codes, desc, H, D, ms)
+    counters = fv.new_tile_counters(T, len(w.seg_lens))
+    out, xq, xs = _group_tail_call(ctx, cu, codes, desc, H, D, ms, w.softmax_scale, counters)
+    assert torch.equal(out.view(torch.int16), ref_out.view(torch.int16))
+    yq, ys = torch.empty_like(xq), torch.empty_like(xs)
+    fv.per_token_group_quant_fp8(out.view(T, H * D), 128, yq, ys, ctx=ctx)
+    assert torch.equal(xq, yq) and torch.equal(xs.view(torch.int32), ys.view(torch.int32))
+    assert int(counters.abs().sum()) == 0
+    toks, _ = sample_pairs(cu, H, per_seg=64, seed=31)
+    toks = np.unique(toks)
+    bits = out.view(torch.int16).cpu().numpy().view(np.uint16).reshape(T, H * D)
+    want_q, want_s = oracle.group_quant(np.ascontiguousarray(bits[toks]), 128)
+    assert np.array_equal(xq.cpu().numpy()[toks], want_q)
+    assert np.array_equal(xs.cpu().numpy()[toks].view(np.uint32), want_s.view(np.uint32))
