@@ -617,14 +617,15 @@ def _step_description(w) -> str:
     return f"{quant} + {out}{tail}"
 
 
-def _launches_per_step(w, l2_bytes: int) -> int:
+def _launches_per_step(w, l2_bytes: int, group_tail: bool = False) -> int:
     """Kernels one step launches: the quantizer (the dynamic entry point takes
     two kernels once the BF16 inputs exceed twice the L2), attention, and the
-    group quantizer where the workload has it."""
+    group quantizer where the workload has it (none when it is the attention
+    launch's tail)."""
     quant = 1
     if w.mode != "static" and 3 * w.tokens * w.hd * 2 > 2 * l2_bytes:
         quant = 2
-    return quant + 1 + (1 if w.group_quant else 0)
+    return quant + 1 + (1 if w.group_quant and not group_tail else 0)
 
 
 def _config(w, n_fwd=None):
@@ -706,16 +707,19 @@ class _Path:
                                     self.max_s, self.w.softmax_scale, out, output_scale=oscale,
                                     ctx=self.ctx)
 
+    def attend_with_tail(self, xq, xs):
+        d = self.desc
+        self.fv.fp8_varlen_attn_fwd_bf16_group_quant(
+            self.q8, self.k8, self.v8, d[0:1], d[1:2], d[2:3], self.cu, self.max_s,
+            self.w.softmax_scale, self.out, xq, xs, self.counters, ctx=self.ctx)
+
     def step(self, i, ev_a=None, ev_b=None, stream=None):
         w = self.w
         self._quantize(i)
         if ev_a is not None:
             ev_a.record(stream)
         if self.group_tail:
-            d = self.desc
-            self.fv.fp8_varlen_attn_fwd_bf16_group_quant(
-                self.q8, self.k8, self.v8, d[0:1], d[1:2], d[2:3], self.cu, self.max_s,
-                w.softmax_scale, self.out, self.xq, self.xs, self.counters, ctx=self.ctx)
+            self.attend_with_tail(self.xq, self.xs)
         elif w.fp8_out:
             self._attend(self.out8, self.oscale)
         else:
@@ -825,7 +829,7 @@ def run_ours(args):
     # the workload's own step: static or dynamic scales (one ring per layer
     # when the seeds are the layers of one encoder forward), BF16 or FP8
     # output, group quantization of the output where the workload has it
-    path = _Path(fv, ctx, w, inputs, dev)
+    path = _Path(fv, ctx, w, inputs, dev, group_tail=args.group_tail)
     cu, max_s = path.cu, path.max_s
     q8, k8, v8, out, xq, xs = path.q8, path.k8, path.v8, path.out, path.xq, path.xs
     rings = path.rings
@@ -915,7 +919,9 @@ def run_ours(args):
         r = dres[i % 2]
         path.inputs = [dbuf[i % 2]]
         path._quantize(i)
-        if w.group_quant:
+        if path.group_tail:
+            path.attend_with_tail(r[0], r[1])
+        elif w.group_quant:
             path._attend(out, None)
             fv.per_token_group_quant_fp8(out.view(T, H * D), 128, r[0], r[1], ctx=ctx)
         elif w.fp8_out:
@@ -974,12 +980,13 @@ def run_ours(args):
     quant = None if args.no_quant_roofline else _quant_rooflines(fv, ctx, inputs[0], dev,
                                                                  peaks["hbm"])
     traffic = _traffic(os.path.join(ROOT, "fp8_quantized_vit_b200", "csrc", "attn.cu"),
-                       args.workload)
+                       args.workload + ("+group_tail" if path.group_tail else ""))
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3 (fp32 accumulate)",
-        "data": "synthetic", "config": dict(_config(w, n_fwd), p_terms=args.p_terms),
+        "data": "synthetic", "config": dict(_config(w, n_fwd), p_terms=args.p_terms,
+                                            **({"group_tail": True} if path.group_tail else {})),
         "roofline": {"bound": "tensor", "kernel": f"attn_fwd_kernel<{D}>",
                      "achieved": attn_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
                      "frac": attn_tflops / fp8_peak, "traffic": traffic,
@@ -990,7 +997,8 @@ def run_ours(args):
                 "copies": "pinned host buffers; uploads, compute and read-backs on three "
                           "streams, double-buffered, overlapping across steps"},
         "gpu_launches": _launches_per_step(
-            w, torch.cuda.get_device_properties(dev).L2_cache_size) * args.steps,
+            w, torch.cuda.get_device_properties(dev).L2_cache_size,
+            path.group_tail) * args.steps,
         "clocks": clk,
         "quantizers": quant,
     }
@@ -1043,6 +1051,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=1.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--group-tail", action="store_true",
+                    help="workloads with a group-quantized output at head_dim 72: run the "
+                         "group quantizer as the attention launch's tail")
     ap.add_argument("--no-quant-roofline", action="store_true")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the per-workload records (each target workload's own step "
