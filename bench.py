@@ -664,8 +664,8 @@ class _Path:
         self.xq = torch.empty((T, H * D), dtype=torch.uint8, device=dev)
         self.xs = torch.empty((T, H * D // 128), dtype=torch.float32, device=dev)
         self.desc = torch.zeros(3, dtype=torch.float32, device=dev)
-        self.counters = (fv.new_tile_counters(T, len(w.seg_lens), dev) if self.group_tail
-                         else None)
+        self.counters = (fv.new_tile_counters(T, len(w.seg_lens), H * D, dev)
+                         if self.group_tail else None)
         self.oscale = None
         if w.mode == "static":
             # calibration (untimed): exact amax of forward 0 on the device,

@@ -383,18 +383,20 @@ def fp8_varlen_attn_fwd_group_quant(q8, k8, v8, q_descale, k_descale, v_descale,
     return xq, scales
 
 
-def tile_counters_size(total_tokens: int, num_seqs: int) -> int:
-    """Entries of the per-query-tile arrival counters that
+def tile_counters_size(total_tokens: int, num_seqs: int, row_elems: int) -> int:
+    """Entries of the arrival counters (one per query tile and 128-column
+    group of a [total_tokens, row_elems] output) that
     fp8_varlen_attn_fwd_bf16_group_quant needs."""
-    return (int(total_tokens) + 127) // 128 + int(num_seqs)
+    return ((int(total_tokens) + 127) // 128 + int(num_seqs)) * (int(row_elems) // 128)
 
 
-def new_tile_counters(total_tokens: int, num_seqs: int, device=None) -> torch.Tensor:
+def new_tile_counters(total_tokens: int, num_seqs: int, row_elems: int,
+                      device=None) -> torch.Tensor:
     """Zeroed counters (uint32 bits held in an int32 tensor); a completed call
     leaves them zero, so one buffer serves every later call of at most this
     size on the same stream."""
-    return torch.zeros(tile_counters_size(total_tokens, num_seqs), dtype=torch.int32,
-                       device=device or "cuda")
+    return torch.zeros(tile_counters_size(total_tokens, num_seqs, row_elems),
+                       dtype=torch.int32, device=device or "cuda")
 
 
 def fp8_varlen_attn_fwd_bf16_group_quant(q8, k8, v8, q_descale, k_descale, v_descale,
@@ -412,7 +414,7 @@ def fp8_varlen_attn_fwd_bf16_group_quant(q8, k8, v8, q_descale, k_descale, v_des
         raise ValueError("q8, k8, v8 and out must have the same [T, H, D] shape")
     if xq.numel() != T * H * D or scales.numel() != T * H * D // 128:
         raise ValueError("xq must hold T * H * D codes and scales T * H * D / 128 floats")
-    if tile_counters.numel() < tile_counters_size(T, cu_seqlens.numel() - 1):
+    if tile_counters.numel() < tile_counters_size(T, cu_seqlens.numel() - 1, H * D):
         raise ValueError("tile_counters is too small (see tile_counters_size)")
     _check(lib().fp8_varlen_attn_fwd_bf16_group_quant(
         _ctx(ctx), _ptr(q8, _FP8, "q8"), _ptr(k8, _FP8, "k8"), _ptr(v8, _FP8, "v8"),
@@ -528,10 +530,11 @@ class FP8EncoderAttention:
         return {k: v[:T] for k, v in st.items() if k != "cap"}
 
     def _counters(self, T: int, num_seqs: int) -> torch.Tensor:
-        need = tile_counters_size(T, num_seqs)
+        hd = self.H * self.D
+        need = tile_counters_size(T, num_seqs, hd)
         c = self._bufs.get("tile_counters")
         if c is None or c.numel() < need:
-            c = new_tile_counters(T, num_seqs, self.device)
+            c = new_tile_counters(T, num_seqs, hd, self.device)
             self._bufs["tile_counters"] = c
         return c
 

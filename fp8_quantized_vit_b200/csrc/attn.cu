@@ -276,108 +276,86 @@ __device__ __forceinline__ void tmem_st_p_any(uint32_t taddr, const uint32_t (&p
 }
 
 
-// Group tail of kOutBf16GroupQ (atrex-bench "#025 per_token_group_quant_fp8":
+// Group tail of the bf16-output kernel, run when it is given tile counters (atrex-bench "#025 per_token_group_quant_fp8":
 // 128-wide groups of a token row, fp32 scale = amax / 448, codes of x / scale;
 // vLLM issue "fused fp8 output for FlashAttention 3": the o-proj input is
 // produced by the attention call).  When a 128-column group spans several
-// heads (head_dim 72: 16 heads are 9 groups) no single head CTA holds a whole
-// group, so each CTA stores its bf16 head slice as usual and then counts
-// itself in on its query tile; the last of the num_heads CTAs to arrive
-// quantizes the tile's token rows across all heads.  Nobody waits on another
-// CTA: the counter only elects the one that runs the tail, then resets it
-// for the next launch.  The rows come back (L2-hot) through bulk copies into
-// two staging buffers over the CTA's now idle Q/K/V shared memory; each half
-// warp takes one group, 8 values a lane, with the arithmetic of
-// group_quant_kernel (same helpers), so codes and scales equal those of
-// per_token_group_quant_fp8 over the stored bf16 output.
-template <class L>
-__device__ __noinline__ void group_tail(uint8_t* sm, uint32_t bar_a, uint32_t bar_b,
-                                        volatile uint32_t* last_flag,
-                                        volatile int32_t* abort_flag, uint32_t* tile_cnt,
-                                        int seg, int32_t seg_start, int32_t seg_len, int qt,
-                                        int ncol, int num_heads, const uint16_t* out,
-                                        uint8_t* xq, float* gscales, fp8vit_scratch* scr) {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+// heads (head_dim 72: 16 heads are 9 groups, each spanning 2 or 3 heads) no
+// single head CTA holds a whole group, so each CTA stores its bf16 head slice
+// as usual and then counts itself in on every group its columns touch; the
+// CTA whose arrival completes a group (its last head to finish) quantizes
+// that group's column block for the tile's token rows.  Nobody waits on
+// another CTA: the counters only elect who runs each group, then reset for
+// the next launch.  A block is 128 rows x 256 bytes, read back (L2-hot) with
+// all of its loads issued at once: each half warp takes a token row, 8 values
+// a lane, with the arithmetic of group_quant_kernel (same helpers), so codes
+// and scales equal those of per_token_group_quant_fp8 over the stored output.
+constexpr int kTailRowsPerPass = kThreads / 16;                          // half warps
+constexpr int kTailRowSlots = (kBM + kTailRowsPerPass - 1) / kTailRowsPerPass;
+
+template <int D>
+__device__ __noinline__ void group_tail(volatile uint32_t* elect, volatile int32_t* abort_flag,
+                                        uint32_t* tile_cnt, int seg, int32_t seg_start,
+                                        int32_t seg_len, int qt, int h, int num_heads,
+                                        const uint16_t* out, uint8_t* xq, float* gscales) {
+    const int tid = threadIdx.x;
+    const int ncol = num_heads * D, ngr = ncol >> 7;
+    // groups this head's columns [h*D, h*D + D) touch
+    const int g0 = (h * D) >> 7, g1 = (h * D + D - 1) >> 7;
     if (tid == 0) {
         // Every CTA of the tile arrives exactly once per launch (the error
-        // paths too), so the count returns to zero with the last arrival.
+        // paths too), so each count returns to zero with its last arrival.
         // Tiles are numbered seg_start / 128 + qt + seg: distinct across
         // segments because cu_seqlens is a cumulative sum.
-        uint32_t* cnt = tile_cnt + ((seg_start >> 7) + qt + seg);
+        uint32_t* cnt = tile_cnt + (int64_t)((seg_start >> 7) + qt + seg) * ngr;
         __threadfence();  // this CTA's bf16 stores (ordered by the barrier above)
-        const bool last = atomicAdd(cnt, 1u) == (uint32_t)num_heads - 1;
-        if (last) {
-            atomicExch(cnt, 0u);
-            __threadfence();  // the other CTAs' stores, before the copies below
-            fence_proxy_async_global();
+        uint32_t mine = 0;
+        for (int g = g0; g <= g1; ++g) {
+            // heads whose columns meet [128 g, 128 g + 128)
+            const uint32_t heads = (uint32_t)(min(128 * g + 127, ncol - 1) / D - (128 * g) / D + 1);
+            if (atomicAdd(cnt + g, 1u) == heads - 1) {
+                atomicExch(cnt + g, 0u);
+                mine |= 1u << (g - g0);
+            }
         }
-        *last_flag = last && *abort_flag == 0;
+        if (mine) __threadfence();  // the other heads' stores, before the reads below
+        *elect = *abort_flag == 0 ? mine : 0u;
     }
     __syncthreads();
-    if (!*last_flag) return;
+    const uint32_t mine = *elect;
+    if (!mine) return;
 
     const int q0 = qt * kBM;
     const int rows = min(kBM, seg_len - q0);
     const int64_t tok0 = (int64_t)seg_start + q0;
-    const uint32_t row_bytes = (uint32_t)ncol * 2;
-    const int ngr = ncol >> 7;  // groups per token row
-    // Rows per staging buffer: half of the Q/K/V area each (the host checks
-    // that one row fits).
-    const int R = min(rows, (int)((L::BAR / 2) / row_bytes));
-    const int nch = (rows + R - 1) / R;
-    const uint32_t buf0 = smem_u32(sm), buf1 = smem_u32(sm) + (uint32_t)(L::BAR / 2);
-    auto issue = [&](int c) {
-        const int r0 = c * R, nr = min(R, rows - r0);
-        const uint32_t bar = (c & 1) ? bar_b : bar_a;
-        mbar_arrive_expect_tx(bar, nr * row_bytes);
-        bulk_load((c & 1) ? buf1 : buf0, out + (tok0 + r0) * ncol, nr * row_bytes, bar);
-    };
-    if (tid == 0) {
-        issue(0);
-        if (nch > 1) issue(1);
-    }
-    const int half = lane >> 4, l16 = lane & 15;
-    const int nwarps = blockDim.x >> 5;
-    int c = 0;
-    bool ok = true;
-    for (; c < nch; ++c) {
-        ok = mbar_wait_bounded((c & 1) ? bar_b : bar_a, (c >> 1) & 1, abort_flag, scr,
-                               SITE_ATTN_WAIT_GROUP, kTimeoutNs);
-        if (!__syncthreads_and(ok)) break;
-        const int r0 = c * R, nr = min(R, rows - r0);
-        const uint8_t* buf = sm + ((c & 1) ? L::BAR / 2 : 0);
-        const int ngroups = nr * ngr;
-        for (int p = warp; 2 * p < ngroups; p += nwarps) {
-            const int g = 2 * p + half;
-            const bool active = g < ngroups;
-            const int r = active ? g / ngr : 0, cg = active ? g - r * ngr : 0;
-            const uint4 x = active ? *reinterpret_cast<const uint4*>(buf + r * row_bytes + cg * 256 +
-                                                                     l16 * 16)
-                                   : make_uint4(0, 0, 0, 0);
-            uint32_t a = __vmaxu2(__vmaxu2(x.x & 0x7FFF7FFFu, x.y & 0x7FFF7FFFu),
-                                  __vmaxu2(x.z & 0x7FFF7FFFu, x.w & 0x7FFF7FFFu));
+    const int hw = tid >> 4, l16 = tid & 15;
+    for (int g = g0; g <= g1; ++g) {
+        if (!((mine >> (g - g0)) & 1u)) continue;
+        uint4 x[kTailRowSlots];
+#pragma unroll
+        for (int u = 0; u < kTailRowSlots; ++u) {
+            const int r = u * kTailRowsPerPass + hw;
+            x[u] = r < rows ? __ldcg(reinterpret_cast<const uint4*>(out + (tok0 + r) * ncol +
+                                                                    g * 128) + l16)
+                            : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kTailRowSlots; ++u) {
+            const int r = u * kTailRowsPerPass + hw;
+            uint32_t a = __vmaxu2(__vmaxu2(x[u].x & 0x7FFF7FFFu, x[u].y & 0x7FFF7FFFu),
+                                  __vmaxu2(x[u].z & 0x7FFF7FFFu, x[u].w & 0x7FFF7FFFu));
             a = max(a & 0xFFFFu, a >> 16);
 #pragma unroll
             for (int off = 8; off > 0; off >>= 1) a = max(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
             const float sc = group_scale_of_amax(bf16_bits_to_f32(a));
-            const float nr2f = -__frcp_rn(sc);
-            const uint2 q = quant8_small(x, f2_pack(sc, sc), f2_pack(nr2f, nr2f));
-            if (active) {
-                const int64_t tok = tok0 + r0 + r;
-                *reinterpret_cast<uint2*>(xq + tok * ncol + cg * 128 + l16 * 8) = q;
-                if (l16 == 0) gscales[tok * ngr + cg] = sc;
+            const float nr = -__frcp_rn(sc);
+            const uint2 q = quant8_small(x[u], f2_pack(sc, sc), f2_pack(nr, nr));
+            if (r < rows) {
+                const int64_t tok = tok0 + r;
+                *reinterpret_cast<uint2*>(xq + tok * ncol + g * 128 + l16 * 8) = q;
+                if (l16 == 0) gscales[tok * ngr + g] = sc;
             }
         }
-        __syncthreads();  // buffer (c & 1) read by all before it is refilled
-        if (tid == 0 && c + 2 < nch) {
-            fence_proxy_async_smem();
-            issue(c + 2);
-        }
-    }
-    if (c < nch && tid == 0) {
-        // Gave up: let the copies still in flight land before the CTA exits.
-        for (int k = c; k < min(c + 2, nch); ++k)
-            mbar_wait_drain((k & 1) ? bar_b : bar_a, (k >> 1) & 1, scr);
     }
 }
 
@@ -399,7 +377,6 @@ __global__ void __launch_bounds__(kThreads, 2)
                     fp8vit_scratch* __restrict__ scr, const uint16_t* __restrict__ qbf,
                     uint8_t* __restrict__ xq, uint32_t* __restrict__ tile_cnt) {
     static_assert(OUT != kOutGroupQ || D == 128, "a 128-wide group is one head at head_dim 128");
-    static_assert(!BF || OUT != kOutBf16GroupQ, "the group tail runs on the FP8 path");
     static_assert(!BF || OUT == kOutBf16, "bf16 inputs: bf16 output");
     static_assert(!(BF && QB), "BF16 Q is quantized only on the FP8 path");
     using C = CfgOf<D, BF>;
@@ -448,11 +425,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     auto b_kv_empty = [&](int s) { return bar0 + 8 * (9 + NS + s); };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::BAR + 8 * (9 + 2 * NS));
     volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
-    // Group tail (kOutBf16GroupQ): two staging-buffer barriers and the
-    // "last CTA of the tile" word after the TMEM slot and the abort flag.
-    auto b_grp = [&](int b) { return bar0 + 8 * (10 + 2 * NS + b); };
-    volatile uint32_t* last_flag = reinterpret_cast<volatile uint32_t*>(sm + L::BAR + 8 * (12 + 2 * NS));
-    static_assert(8 * (12 + 2 * NS) + 4 <= L::TOTAL - L::BAR, "barrier area");
+    // Group tail (bf16 output with tile counters): the CTA's elected groups, after the TMEM
+    // slot and the abort flag.
+    volatile uint32_t* elect = reinterpret_cast<volatile uint32_t*>(tmem_slot + 2);
+    static_assert(8 * (9 + 2 * NS) + 12 <= L::TOTAL - L::BAR, "barrier area");
 
     if (threadIdx.x == 0) {
         mbar_init(b_q_full, 1);
@@ -469,10 +445,6 @@ __global__ void __launch_bounds__(kThreads, 2)
             mbar_init(b_kv_empty(s), 1);
         }
         *abort_flag = 0;
-        if constexpr (OUT == kOutBf16GroupQ) {
-            mbar_init(b_grp(0), 1);
-            mbar_init(b_grp(1), 1);
-        }
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -860,10 +832,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
-    if constexpr (OUT == kOutBf16GroupQ)
-        group_tail<L>(sm, b_grp(0), b_grp(1), last_flag, abort_flag, tile_cnt, seg, seg_start,
-                      seg_len, qt, num_heads * D, num_heads, reinterpret_cast<const uint16_t*>(out),
-                      xq, gscales, scr);
+    if constexpr (OUT == kOutBf16 && !BF)
+        if (tile_cnt)
+            group_tail<D>(elect, abort_flag, tile_cnt, seg, seg_start, seg_len, qt, h,
+                          num_heads, reinterpret_cast<const uint16_t*>(out), xq, gscales);
 }
 
 
@@ -889,10 +861,9 @@ fp8vit_status launch(fp8vit_ctx* ctx, const uint8_t* q8, const uint8_t* k8, cons
     const bool two_terms = ctx->attn_p_terms != 1;
     const int inst = (two_terms ? 1 : 0) + (qbf ? 2 : 0);
     auto kern = two_terms ? attn_fwd_kernel<D, OUT, true> : attn_fwd_kernel<D, OUT, false>;
-    if constexpr (OUT != kOutBf16GroupQ)  // the group tail has no BF16-Q instance
-        if (qbf)
-            kern = two_terms ? attn_fwd_kernel<D, OUT, true, false, true>
-                             : attn_fwd_kernel<D, OUT, false, false, true>;
+    if (qbf)
+        kern = two_terms ? attn_fwd_kernel<D, OUT, true, false, true>
+                         : attn_fwd_kernel<D, OUT, false, false, true>;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FP8VIT_ECUDA;
     const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
@@ -1075,17 +1046,14 @@ extern "C" fp8vit_status fp8_varlen_attn_fwd_bf16_group_quant(
         misaligned(d_tile_counters, 4) || misaligned(d_cu_seqlens, 4))
         return FP8VIT_EINVAL;
     if (num_heads > 65535 || num_seqs > 65535) return FP8VIT_EUNSUPPORTED;
-    // Two staging buffers of at least one token row each in the Q/K/V area.
-    const int64_t row_bytes = (int64_t)num_heads * head_dim * 2;
-    if (2 * row_bytes > (head_dim == 72 ? Smem<72>::BAR : Smem<128>::BAR)) return FP8VIT_EUNSUPPORTED;
     if (num_seqs == 0 || max_seqlen == 0 || total_tokens == 0) return FP8VIT_OK;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (head_dim == 72)
-        return launch<72, kOutBf16GroupQ>(ctx, d_q8, d_k8, d_v8, d_q_descale, d_k_descale,
+        return launch<72, kOutBf16>(ctx, d_q8, d_k8, d_v8, d_q_descale, d_k_descale,
                                           d_v_descale, d_cu_seqlens, num_seqs, max_seqlen,
                                           total_tokens, num_heads, softmax_scale, d_out, nullptr,
                                           d_scales, st, nullptr, d_xq, d_tile_counters);
-    return launch<128, kOutBf16GroupQ>(ctx, d_q8, d_k8, d_v8, d_q_descale, d_k_descale,
+    return launch<128, kOutBf16>(ctx, d_q8, d_k8, d_v8, d_q_descale, d_k_descale,
                                        d_v_descale, d_cu_seqlens, num_seqs, max_seqlen,
                                        total_tokens, num_heads, softmax_scale, d_out, nullptr,
                                        d_scales, st, nullptr, d_xq, d_tile_counters);

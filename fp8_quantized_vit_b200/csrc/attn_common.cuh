@@ -176,13 +176,12 @@ __device__ __forceinline__ uint4 bf16x8_of_o(uint32_t taddr, float inv) {
 
 // Output modes, one epilogue per kernel instance.
 enum : int {
-    kOutBf16 = 0,     // o as bf16
+    kOutBf16 = 0,     // o as bf16; with a tile-counter buffer, also its 128-wide
+                      // groups quantized by the launch's group tail (any head_dim
+                      // with num_heads * head_dim % 128 == 0)
     kOutE4m3 = 1,     // e4m3(o / output_scale)
     kOutGroupQ = 2,   // the bf16 o of each head quantized as one 128-wide group:
                       // e4m3 codes + one fp32 scale per (token, head); head_dim 128
-    kOutBf16GroupQ = 3,  // o as bf16, then the last of a query tile's head CTAs
-                         // quantizes the tile's token rows (all heads) in 128-wide
-                         // groups: any head_dim with num_heads * head_dim % 128 == 0
 };
 
 // Host: a 2-D uint8 tensor map over a [rows, row_bytes] matrix with

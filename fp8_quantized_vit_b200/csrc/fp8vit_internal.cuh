@@ -78,7 +78,6 @@ enum : int32_t {
     SITE_ATTN_WAIT_QREADY = 117,
     SITE_ATTN_DRAIN = 118,
     SITE_ATTN_WAIT_SFREE = 119,
-    SITE_ATTN_WAIT_GROUP = 120,
     SITE_QUANT_BARRIER = 200,
 };
 
@@ -265,21 +264,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_global() {
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-// Untiled bulk copy global -> shared of `bytes` (a multiple of 16; both
-// addresses 16-byte aligned), completion on an mbarrier.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            dst),
-        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-        : "memory");
 }
 
 // TMA: 2-D tiled load global -> shared, completion on an mbarrier.

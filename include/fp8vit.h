@@ -320,9 +320,10 @@ fp8vit_status fp8_varlen_attn_fwd_group_quant(
  * call; atrex-bench "#025 per_token_group_quant_fp8": 128-wide groups of a
  * token row, fp32 scales, the o-proj input).  At head_dim 72 a group spans
  * two or three heads, so no single head's CTA holds a group: every CTA
- * stores its BF16 head slice to d_out, and the last of the num_heads CTAs of
- * a query tile to finish quantizes that tile's token rows over all heads
- * (an arrival counter per tile elects it; no CTA waits for another).
+ * stores its BF16 head slice to d_out and counts itself in on the groups its
+ * columns touch; the CTA that completes a group (the last of its heads to
+ * finish on that query tile) quantizes it for the tile's token rows.  The
+ * counters only elect; no CTA waits for another.
  * d_out: BF16 [total_tokens, num_heads * head_dim], 16-byte aligned; holds
  *   fp8_varlen_attn_fwd's out_dtype 0 result on return.
  * d_xq: e4m3 [total_tokens, num_heads * head_dim], 16-byte aligned, and
@@ -330,16 +331,13 @@ fp8vit_status fp8_varlen_attn_fwd_group_quant(
  *   byte for byte and bit for bit what per_token_group_quant_fp8(d_out, 128)
  *   writes.
  * d_tile_counters: uint32 workspace of at least
- *   (total_tokens + 127) / 128 + num_seqs entries, all zero before the first
- *   call; a completed call leaves them zero again (the caller zeroes it once,
- *   e.g. with cudaMemsetAsync, and reuses it).  Calls that share a counter
- *   buffer must not run concurrently.
+ *   ((total_tokens + 127) / 128 + num_seqs) * (num_heads * head_dim / 128)
+ *   entries, all zero before the first call; a completed call leaves them
+ *   zero again (the caller zeroes it once, e.g. with cudaMemsetAsync, and
+ *   reuses it).  Calls that share a counter buffer must not run concurrently.
  * Returns FP8VIT_EINVAL when num_heads * head_dim is not a multiple of 128
  * or a pointer is null or misaligned, FP8VIT_EUNSUPPORTED for another
- * head_dim or for token rows too long for two staging rows in the
- * kernel's Q/K/V shared memory (above 160 heads at head_dim 128, 352 at 72).  A timeout of the
- * tail's staging copies records FP8VIT_ETIMEOUT at site 120.  Other
- * arguments, checks and faults as fp8_varlen_attn_fwd. */
+ * head_dim.  Other arguments, checks and faults as fp8_varlen_attn_fwd. */
 fp8vit_status fp8_varlen_attn_fwd_bf16_group_quant(
     fp8vit_ctx* ctx, const uint8_t* d_q8, const uint8_t* d_k8, const uint8_t* d_v8,
     const float* d_q_descale, const float* d_k_descale, const float* d_v_descale,

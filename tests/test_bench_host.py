@@ -348,8 +348,8 @@ def test_workload_paths_run_each_configurations_own_step(monkeypatch):
         fp8_varlen_attn_fwd=stand_in("fp8_varlen_attn_fwd"),
         per_token_group_quant_fp8=stand_in("per_token_group_quant_fp8"),
         fp8_varlen_attn_fwd_bf16_group_quant=stand_in("fp8_varlen_attn_fwd_bf16_group_quant"),
-        new_tile_counters=lambda t, n, dev=None: torch.zeros(fv.tile_counters_size(t, n),
-                                                             dtype=torch.int32))
+        new_tile_counters=lambda t, n, hd, dev=None: torch.zeros(
+            fv.tile_counters_size(t, n, hd), dtype=torch.int32))
     ctx = types.SimpleNamespace(check=lambda: (0, 0))
     T, H, D = 40, 2, 72
     w = synth.Workload("3 tiny images", (10, 10, 20), H, D, "static", (1,), fp8_out=True)
@@ -386,4 +386,5 @@ def test_workload_paths_run_each_configurations_own_step(monkeypatch):
     path.step(0)
     assert [s[0] for s in seen] == ["fp8_amax_ring_quantize_qkv",
                                     "fp8_varlen_attn_fwd_bf16_group_quant"]
-    assert seen[1][1][12] is path.counters and path.counters.numel() == (T + 127) // 128 + 3
+    assert seen[1][1][12] is path.counters
+    assert path.counters.numel() == ((T + 127) // 128 + 3) * (H * D // 128)

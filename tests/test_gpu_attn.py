@@ -628,7 +628,7 @@ def _oracle_group_quant_of(out: torch.Tensor):
 
 @pytest.mark.parametrize("lens,H,D,max_seqlen", [
     ((513, 129, 0, 300, 1), 16, 72, 513),  # several tiles, ragged tails, empty and 1-token images
-    ((256, 5), 32, 72, 300),               # 12 staging chunks per tile; slack max_seqlen
+    ((256, 5), 32, 72, 300),               # 18 groups per token row; slack max_seqlen
     ((200, 77), 2, 128, 200),              # head_dim 128: one group per head
     ((1,), 16, 72, 1),
 ])
@@ -643,7 +643,7 @@ def test_group_quant_tail(ctx, lens, H, D, max_seqlen):
     sm = np.float32(1.0 / math.sqrt(D))
     T = codes[0].shape[0]
     ref_out = _run_gpu(ctx, cu, codes, desc, H, D, max_seqlen)
-    counters = fv.new_tile_counters(T, len(lens))
+    counters = fv.new_tile_counters(T, len(lens), H * D)
     out, xq, xs = _group_tail_call(ctx, cu, codes, desc, H, D, max_seqlen, sm, counters)
     assert torch.equal(out.view(torch.int16), ref_out.view(torch.int16))
     assert_attn_close(_gpu_bf16_to_f64(out), oracle.attn_full(*codes, *desc, cu, H, D, sm),
@@ -673,7 +673,7 @@ def test_group_quant_tail_27_layer_workload_size(ctx):
     cu = synth.cu_seqlens(w.seg_lens)
     T, ms = w.tokens, max(w.seg_lens)
     ref_out = _run_gpu(ctx, cu, codes, desc, H, D, ms)
-    counters = fv.new_tile_counters(T, len(w.seg_lens))
+    counters = fv.new_tile_counters(T, len(w.seg_lens), H * D)
     out, xq, xs = _group_tail_call(ctx, cu, codes, desc, H, D, ms, w.softmax_scale, counters)
     assert torch.equal(out.view(torch.int16), ref_out.view(torch.int16))
     yq, ys = torch.empty_like(xq), torch.empty_like(xs)
