@@ -107,22 +107,34 @@ def _check(status: int, what: str):
         raise FP8VitError(status, what)
 
 
+# The current stream's raw handle: torch's direct accessor where it exists
+# (a tenth of the cost of building a torch.cuda.Stream object per call).
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+_cur_device = getattr(torch._C, "_cuda_getDevice", None)
+
+
 def _stream(stream=None) -> int:
     if stream is None:
+        if _raw_stream is not None and _cur_device is not None:
+            return _raw_stream(_cur_device())
         stream = torch.cuda.current_stream()
     return stream.cuda_stream
 
 
 def _ptr(t: torch.Tensor | None, dtype=None, name: str = "tensor") -> int | None:
+    """Device address of a contiguous CUDA tensor of one of the dtypes in
+    ``dtype`` (a dtype or a tuple of them); ValueError otherwise.  The common
+    case costs one combined test; the message is built only on failure."""
     if t is None:
         return None
+    if t.is_cuda and t.is_contiguous() and (
+            dtype is None or (t.dtype in dtype if type(dtype) is tuple else t.dtype is dtype)):
+        return t.data_ptr()
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
-    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
-        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
-    return t.data_ptr()
+    raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
 
 
 _FP8 = (torch.uint8, torch.float8_e4m3fn)
@@ -486,6 +498,7 @@ class FP8EncoderAttention:
         self.device = torch.device(device or "cuda")
         self.ctx = ctx or default_context()
         self.descale = torch.zeros(3, dtype=torch.float32, device=self.device)
+        self._dq, self._dk, self._dv = self._dq, self._dk, self._dv
         self.process_group = process_group
         self._amax3 = torch.zeros(3, dtype=torch.float32, device=self.device)
         self.ring = None
@@ -575,23 +588,23 @@ class FP8EncoderAttention:
             xq, xs = b["xq"], b["xs"]
             if self.D != 128 and self.group_tail and not fold:
                 fp8_varlen_attn_fwd_bf16_group_quant(
-                    b["q8"], b["k8"], b["v8"], self.descale[0:1], self.descale[1:2],
-                    self.descale[2:3], cu_seqlens, max_seqlen, self.softmax_scale, b["out"], xq,
+                    b["q8"], b["k8"], b["v8"], self._dq, self._dk,
+                    self._dv, cu_seqlens, max_seqlen, self.softmax_scale, b["out"], xq,
                     xs, self._counters(T, cu_seqlens.numel() - 1), ctx=self.ctx)
             elif self.D == 128:
-                fp8_varlen_attn_fwd_group_quant(b["q8"], b["k8"], b["v8"], self.descale[0:1],
-                                                self.descale[1:2], self.descale[2:3], cu_seqlens,
+                fp8_varlen_attn_fwd_group_quant(b["q8"], b["k8"], b["v8"], self._dq,
+                                                self._dk, self._dv, cu_seqlens,
                                                 max_seqlen, self.softmax_scale, xq, xs,
                                                 ctx=self.ctx)
             else:
                 o = b["out"]
-                attn(qa, b["k8"], b["v8"], self.descale[0:1], self.descale[1:2],
-                     self.descale[2:3], cu_seqlens, max_seqlen, self.softmax_scale, o,
+                attn(qa, b["k8"], b["v8"], self._dq, self._dk,
+                     self._dv, cu_seqlens, max_seqlen, self.softmax_scale, o,
                      ctx=self.ctx)
                 per_token_group_quant_fp8(o.view(T, hd), 128, xq, xs, ctx=self.ctx)
             return xq, xs
         o = b["out"] if out is None else out
-        attn(qa, b["k8"], b["v8"], self.descale[0:1], self.descale[1:2], self.descale[2:3],
+        attn(qa, b["k8"], b["v8"], self._dq, self._dk, self._dv,
              cu_seqlens, max_seqlen, self.softmax_scale, o, output_scale=output_scale,
              ctx=self.ctx)
         return o

@@ -323,3 +323,16 @@ def test_noalloc_entry_point_is_bound_and_checks_on_the_host():
     assert f(dummy, dummy, dummy, -1, dummy, dummy, None) == fv.EINVAL
     assert f(ctypes.c_void_p(0x10002), dummy, dummy, 8, dummy, dummy, None) == fv.EINVAL
     assert callable(fv.fp8_amax_ring_update_noalloc)
+
+
+def test_pointer_checks_refuse_host_tensors_without_a_gpu():
+    """The binding's argument check refuses a host tensor (and, on the same
+    path, reports non-contiguous tensors and wrong dtypes) before any call
+    into the library; the current-stream accessor it uses exists in torch."""
+    t = torch.zeros(4, 4, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        fv._ptr(t, fv._FP8, "x")
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        fv._ptr(t.t(), torch.uint8, "x")
+    assert fv._ptr(None, torch.float32) is None
+    assert fv._raw_stream is not None and fv._cur_device is not None
