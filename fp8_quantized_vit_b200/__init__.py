@@ -498,7 +498,7 @@ class FP8EncoderAttention:
         self.device = torch.device(device or "cuda")
         self.ctx = ctx or default_context()
         self.descale = torch.zeros(3, dtype=torch.float32, device=self.device)
-        self._dq, self._dk, self._dv = self._dq, self._dk, self._dv
+        self._dq, self._dk, self._dv = self.descale[0:1], self.descale[1:2], self.descale[2:3]
         self.process_group = process_group
         self._amax3 = torch.zeros(3, dtype=torch.float32, device=self.device)
         self.ring = None

@@ -336,3 +336,23 @@ def test_pointer_checks_refuse_host_tensors_without_a_gpu():
         fv._ptr(t.t(), torch.uint8, "x")
     assert fv._ptr(None, torch.float32) is None
     assert fv._raw_stream is not None and fv._cur_device is not None
+
+
+def test_layer_constructor_runs_without_a_gpu(monkeypatch):
+    """FP8EncoderAttention's constructor on host memory with a stand-in
+    context: the descale views alias the descale vector (a static-scale
+    update through copy_ reaches them), a dynamic layer gets a ring, and the
+    default softmax scale is the fp32 rounding of head_dim ** -0.5."""
+    import types
+    ctx = types.SimpleNamespace(handle=None)
+    layer = fv.FP8EncoderAttention(16, 72, device="cpu", ctx=ctx, static_amax=[448.0, 896.0, 1.5])
+    assert layer.ring is None and layer.group_tail is False and layer.fold_q is False
+    for view, i in zip((layer._dq, layer._dk, layer._dv), range(3)):
+        assert view.data_ptr() == layer.descale[i:i + 1].data_ptr()
+    assert float(layer._dq) == 1.0 and float(layer._dk) == 2.0
+    assert layer.softmax_scale == float(np.float32(72 ** -0.5))
+    # a dynamic layer asks for a device ring (ring_init refuses host memory)
+    monkeypatch.setattr(fv, "new_ring", lambda device=None: torch.zeros(fv.RING_BYTES // 4))
+    dyn = fv.FP8EncoderAttention(4, 128, device="cpu", ctx=ctx, group_tail=True)
+    assert dyn.ring is not None and dyn.ring.numel() * dyn.ring.element_size() == fv.RING_BYTES
+    assert dyn.group_tail and float(dyn.descale.abs().sum()) == 0.0
