@@ -686,3 +686,37 @@ def test_group_quant_tail_27_layer_workload_size(ctx):
     want_q, want_s = oracle.group_quant(np.ascontiguousarray(bits[toks]), 128)
     assert np.array_equal(xq.cpu().numpy()[toks], want_q)
     assert np.array_equal(xs.cpu().numpy()[toks].view(np.uint32), want_s.view(np.uint32))
+
+
+def test_group_tail_counters_survive_an_attention_timeout():
+    """The group tail's arrival counters return to zero when the attention
+    gives up: with the S-ready commit skipped (injected on the host), every
+    CTA's bounded wait runs out, every CTA still counts itself in on its
+    groups, and a CTA that aborted quantizes nothing.  fp8vit_check reports
+    the timeout; the next call on the same counters gives the oracle group
+    quantizer's bytes of its own BF16 output.  No GPU fault is involved."""
+    c = fv.Context()
+    lens, H, D = (129, 40), 16, 72
+    cu, codes, desc = _prepare(lens, H, D, seed=23)
+    sm = np.float32(1.0 / math.sqrt(D))
+    T = codes[0].shape[0]
+    counters = fv.new_tile_counters(T, len(lens), H * D)
+    q8, k8, v8 = (_dev(x) for x in codes)
+    d = [torch.tensor([x], dtype=torch.float32, device="cuda") for x in desc]
+    out = torch.empty((T, H, D), dtype=torch.bfloat16, device="cuda")
+    xq = torch.empty((T, H * D), dtype=torch.uint8, device="cuda")
+    xs = torch.empty((T, H * D // 128), dtype=torch.float32, device="cuda")
+    assert fv.lib().fp8vit_inject_attn_timeout(c.handle, fv._stream()) == fv.OK
+    fv.fp8_varlen_attn_fwd_bf16_group_quant(q8, k8, v8, d[0], d[1], d[2], _dev(cu), max(lens), sm,
+                                            out, xq, xs, counters, ctx=c)
+    st, site = c.check()
+    assert st == fv.ETIMEOUT and site in (113, 114, 119), (fv.status_string(st), site)
+    assert int(counters.abs().sum()) == 0
+    out, xq, xs = _group_tail_call(c, cu, codes, desc, H, D, max(lens), sm, counters)
+    assert_attn_close(_gpu_bf16_to_f64(out), oracle.attn_full(*codes, *desc, cu, H, D, sm),
+                      "after the injected timeout")
+    want_q, want_s = _oracle_group_quant_of(out)
+    assert np.array_equal(xq.cpu().numpy(), want_q)
+    assert np.array_equal(xs.cpu().numpy().view(np.uint32), want_s.view(np.uint32))
+    assert int(counters.abs().sum()) == 0
+    c.close()
