@@ -786,9 +786,27 @@ def _graph_times(path, w, inputs, reps=20, rounds=5):
     return rec
 
 
+def _events_median(fn, reps, stream, warmup=3):
+    """Median over reps of one call's device time (CUDA events on the stream)."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    per = []
+    for _ in range(reps):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        per.append((a, b))
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in per)
+
+
 def _time_path(path, steps, warmup, stream):
-    """(ms per step, attention ms per launch) of a workload's own step, CUDA
-    events on the launching stream."""
+    """(ms per step, median and mean attention ms per launch) of a workload's
+    own step, CUDA events on the launching stream."""
     import torch
     for i in range(warmup):
         path.step(i)
@@ -802,11 +820,11 @@ def _time_path(path, steps, warmup, stream):
         path.step(i, ev_a[i], ev_b[i], stream)
     t1.record(stream)
     torch.cuda.synchronize()
-    attn = statistics.mean(a.elapsed_time(b) for a, b in zip(ev_a, ev_b))
-    return t0.elapsed_time(t1) / steps, attn
+    per = [a.elapsed_time(b) for a, b in zip(ev_a, ev_b)]
+    return t0.elapsed_time(t1) / steps, statistics.median(per), statistics.mean(per)
 
 
-def _config_records(fv, ctx, dev, peaks, stream, steps=5, warmup=3):
+def _config_records(fv, ctx, dev, peaks, stream, steps=20, warmup=3):
     """Every target workload's own step, timed in the same run as the headline
     (attention TFLOP/s and its fraction of the FP8 denominator, step time), with
     torch's BF16 SDPA on the same inputs beside the single-image workloads."""
@@ -823,17 +841,23 @@ def _config_records(fv, ctx, dev, peaks, stream, steps=5, warmup=3):
                    .to(dev) for x in w.qkv(f)] for f in range(n_in)]
         path = _Path(fv, ctx, w, inputs, dev)
         n_steps = n_in if w.per_layer_rings else steps  # one pass over all 27 layers
-        ms, attn_ms = _time_path(path, n_steps, min(warmup, n_steps), stream)
+        ms, attn_ms, attn_mean = _time_path(path, n_steps, min(warmup, n_steps), stream)
         st, site = ctx.check()
         if st != fv.OK:
             raise RuntimeError(f"device fault in {name}: {fv.status_string(st)} site {site}")
         tf = w.attn_flops() / (attn_ms * 1e-3) / 1e12
         rec = {"workload": w.name, "step": _step_description(w), "ms_per_step": ms,
-               "steps_timed": n_steps, "attn_ms": attn_ms, "attn_tflops": tf,
+               "steps_timed": n_steps, "attn_ms": attn_ms, "attn_ms_mean": attn_mean,
+               "attn_timing": "median of the steps' attention events", "attn_tflops": tf,
                "attn_frac_of_fp8_peak": tf / fp8_peak,
                "step_tflops": w.attn_flops() / (ms * 1e-3) / 1e12}
         if len(w.seg_lens) == 1:
             rec["torch_bf16_sdpa"] = _sdpa_comparator(w, inputs, dev)
+        if w.fp8_out:
+            # the same attention with BF16 output (the run before the FP8-out one)
+            b_ms = _events_median(lambda: path._attend(path.out, None), steps, stream)
+            rec["bf16_out"] = {"attn_ms": b_ms,
+                               "attn_tflops": w.attn_flops() / (b_ms * 1e-3) / 1e12}
         if w.tokens <= 4096:
             rec["graph"] = _graph_times(path, w, inputs)
             st, site = ctx.check()
@@ -845,7 +869,7 @@ def _config_records(fv, ctx, dev, peaks, stream, steps=5, warmup=3):
             # tail: one launch instead of attention + per_token_group_quant_fp8
             del path
             path = _Path(fv, ctx, w, inputs, dev, group_tail=True)
-            ms_t, attn_t = _time_path(path, n_steps, min(warmup, n_steps), stream)
+            ms_t, attn_t, _ = _time_path(path, n_steps, min(warmup, n_steps), stream)
             st, site = ctx.check()
             if st != fv.OK:
                 raise RuntimeError(f"device fault in {name} (group tail): "
@@ -1051,7 +1075,8 @@ def run_ours(args):
                      "achieved": attn_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
                      "frac": attn_tflops / fp8_peak, "traffic": traffic,
                      "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16']} x 2 (fp8/bf16)",
-                     "kernel_ms": attn_avg_s * 1e3},
+                     "kernel_ms": attn_avg_s * 1e3,
+                     "kernel_ms_median": statistics.median(attn_ms)},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "copies": "pinned host buffers; uploads, compute and read-backs on three "
