@@ -29,6 +29,10 @@
 // 16-byte aligned x coordinate); bytes of the window outside the head are
 // zeroed in Q, so the neighbouring head's K bytes contribute exactly 0.  PV
 // runs with N = 80 and the epilogue picks the head's 72 columns.
+// Epilogues (one per instance): BF16 o; e4m3 o / output_scale; at head_dim
+// 128 the per-token-group quantizer on each head's row (a group is a head);
+// and, with tile counters, the BF16 instance's group tail, where the CTA that
+// completes a 128-column group across heads quantizes it (group_tail below).
 #include <math.h>
 
 #include <atomic>
