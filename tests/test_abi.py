@@ -356,3 +356,28 @@ def test_layer_constructor_runs_without_a_gpu(monkeypatch):
     dyn = fv.FP8EncoderAttention(4, 128, device="cpu", ctx=ctx, group_tail=True)
     assert dyn.ring is not None and dyn.ring.numel() * dyn.ring.element_size() == fv.RING_BYTES
     assert dyn.group_tail and float(dyn.descale.abs().sum()) == 0.0
+
+
+def test_tile_counter_workspace_covers_every_counter_index():
+    """The counter workspace the binding sizes for the group tail holds every
+    counter the kernel indexes: the kernel counts (query tile, group) pairs at
+    (seg_start / 128 + tile + segment) * groups + group, distinct for distinct
+    pairs because cu_seqlens is a cumulative sum.  Random ragged layouts,
+    empty images and single tokens included."""
+    rng = np.random.default_rng(7)
+    for trial in range(300):
+        n = int(rng.integers(1, 12))
+        lens = rng.integers(0, 700, size=n)
+        lens[rng.random(n) < 0.2] = int(rng.integers(0, 3))
+        cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+        T = int(cu[-1])
+        groups = int(rng.choice([9, 16, 18]))
+        size = fv.tile_counters_size(T, n, groups * 128)
+        seen = set()
+        for seg in range(n):
+            for qt in range((int(lens[seg]) + 127) // 128):
+                for g in range(groups):
+                    idx = ((int(cu[seg]) >> 7) + qt + seg) * groups + g
+                    assert 0 <= idx < size, (trial, seg, qt, g, idx, size)
+                    assert idx not in seen
+                    seen.add(idx)
